@@ -1,0 +1,264 @@
+"""Pins for the double-precision oracle (CPU only).
+
+Each test ties the oracle to something other than itself: hand-worked golden
+cases, an exact integer brute force written independently here, closed forms
+(FRM with stride 1 equals the reciprocal set; an identity warp matches every
+pixel to itself) and the invariants the pages state (every FRM pair is a
+mutual match, FRM output is a subset of M, scores never decrease along a
+trajectory).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from reciprocal_nearest_neighbour_b200 import synth
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+def _chain_maps(g):
+    S = np.array(g["scores"], dtype=np.float64)
+    D1 = S.reshape(g["H1"], g["W1"], g["d"])
+    D2 = np.eye(g["d"]).reshape(g["H2"], g["W2"], g["d"])
+    return D1, D2
+
+
+# ---------------------------------------------------------------- golden cases
+
+def test_golden_chain_nn_and_mnn(golden_dir):
+    g = _load(golden_dir, "frm_chain_2x2_1x4.json")
+    D1, D2 = _chain_maps(g)
+    r = oracle.mnn(D1, D2)
+    assert r.row.arg.tolist() == g["nn2"]
+    assert r.col.arg.tolist() == g["nn1"]
+    assert r.pairs.tolist() == g["mnn"]
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_golden_chain_frm(golden_dir, case):
+    g = _load(golden_dir, "frm_chain_2x2_1x4.json")
+    c = g["frm"][case]
+    D1, D2 = _chain_maps(g)
+    r = oracle.frm(D1, D2, seed_stride=c["stride"], max_iter=c["max_iter"])
+    assert r.pairs.reshape(-1, 2).tolist() == c["pairs"]
+    if "seed_queries" in c:
+        assert r.seed_queries.tolist() == c["seed_queries"]
+    if "seed_converged" in c:
+        assert r.seed_converged.tolist() == c["seed_converged"]
+    if "traj" in c:
+        assert r.traj.tolist() == c["traj"]
+
+
+def test_golden_seed_grid(golden_dir):
+    g = _load(golden_dir, "seed_grid.json")
+    for c in g["cases"]:
+        s = oracle.frm_seeds(c["H"], c["W"], c["S"])
+        if "seeds" in c:
+            assert s.tolist() == c["seeds"], c
+        else:
+            assert len(s) == c["count"] and s[0] == c["first"] and s[-1] == c["last"], c
+        assert np.all(np.diff(s) > 0)
+
+
+def test_golden_nn_ties(golden_dir):
+    g = _load(golden_dir, "nn_ties.json")
+    for c in g["cases"]:
+        sc = np.array(c["scores"], dtype=np.float64)
+        X = np.zeros((len(sc), 4))
+        X[:, 0] = sc
+        q = np.zeros((1, 4))
+        q[0, 0] = 1.0
+        r = oracle.nn(q, X)
+        assert r.arg[0] == c["arg"], c
+        want = math.inf if c["gap"] == "inf" else c["gap"]
+        assert r.gap[0] == want, c
+
+
+# ------------------------------------------------------- exact integer brute force
+
+def _int_codes(H, W, d, seed):
+    rng = np.random.default_rng(seed)
+    return synth.quantised_map(rng, H, W, d)
+
+
+def _brute(K1, K2):
+    """Exact integer scores (k1 . k2) and lowest-index argmax both ways."""
+    A = np.rint(K1.reshape(-1, K1.shape[-1]) * 64).astype(np.int64)
+    B = np.rint(K2.reshape(-1, K2.shape[-1]) * 64).astype(np.int64)
+    S = A @ B.T
+    rowarg = S.argmax(axis=1)          # numpy argmax returns the first maximum
+    colarg = S.argmax(axis=0)
+    mutual = [(i, int(rowarg[i])) for i in range(S.shape[0]) if colarg[rowarg[i]] == i]
+    return S, rowarg, colarg, mutual
+
+
+@pytest.mark.parametrize("shape", [((7, 9), (8, 6), 16), ((16, 16), (16, 16), 8),
+                                   ((5, 13), (11, 3), 24), ((32, 32), (32, 32), 16)])
+def test_mnn_matches_integer_bruteforce(shape):
+    (H1, W1), (H2, W2), d = shape
+    rng = np.random.default_rng(11 + d)
+    D1 = synth.quantised_map(rng, H1, W1, d)
+    D2 = synth.quantised_map(rng, H2, W2, d)
+    S, ra, ca, mutual = _brute(D1, D2)
+    r = oracle.mnn(D1, D2)
+    assert np.array_equal(r.row.arg, ra)
+    assert np.array_equal(r.col.arg, ca)
+    assert [tuple(p) for p in r.pairs.tolist()] == mutual
+    # scores are exact: best * 4096 is the integer maximum
+    assert np.array_equal(r.row.best * 4096, S.max(axis=1).astype(np.float64))
+    assert np.array_equal(r.col.best * 4096, S.max(axis=0).astype(np.float64))
+    srt = np.sort(S, axis=1)
+    assert np.array_equal(r.row.gap * 4096, (srt[:, -1] - srt[:, -2]).astype(np.float64))
+
+
+def test_tiny_workload_matches_bruteforce():
+    w = synth.WORKLOADS["tiny_q32"]
+    D1, D2 = synth.make_workload(w)
+    _, ra, ca, mutual = _brute(D1, D2)
+    r = oracle.mnn(D1, D2)
+    assert np.array_equal(r.row.arg, ra) and np.array_equal(r.col.arg, ca)
+    assert [tuple(p) for p in r.pairs.tolist()] == mutual
+
+
+def test_ties_on_duplicated_candidates():
+    rng = np.random.default_rng(5)
+    D1 = synth.quantised_map(rng, 4, 4, 8)
+    base = synth.quantised_map(rng, 2, 4, 8)
+    D2 = np.concatenate([base, base], axis=0)        # candidates j and j+8 are equal
+    r = oracle.mnn(D1, D2)
+    assert np.all(r.row.arg < 8)                      # lowest index wins
+    assert np.all(r.row.gap == 0)
+    zeros = np.zeros((3, 3, 8))
+    z = oracle.mnn(zeros, zeros)                      # every score is 0
+    assert np.all(z.row.arg == 0) and np.all(z.col.arg == 0)
+    assert z.pairs.tolist() == [[0, 0]]
+
+
+# ------------------------------------------------------------------ closed forms
+
+@pytest.mark.parametrize("max_iter", [1, 3, 10])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_frm_stride1_equals_mnn(seed, max_iter):
+    rng = np.random.default_rng(100 + seed)
+    D1 = synth.quantised_map(rng, 9, 11, 16)
+    D2 = synth.quantised_map(rng, 10, 7, 16)
+    m = oracle.mnn(D1, D2)
+    f = oracle.frm(D1, D2, seed_stride=1, max_iter=max_iter)
+    assert f.pairs.tolist() == m.pairs.tolist()
+
+
+def _unit_iid(rng, H, W, d):
+    v = rng.standard_normal((H, W, d))
+    v /= np.linalg.norm(v, axis=-1, keepdims=True)
+    return synth.to_storage(v, "f16").double().numpy()
+
+
+def test_identity_warp():
+    rng = np.random.default_rng(7)
+    D = _unit_iid(rng, 20, 24, 32)
+    m = oracle.mnn(D, D)
+    n = 20 * 24
+    assert m.pairs.tolist() == [[i, i] for i in range(n)]
+    f = oracle.frm(D, D, seed_stride=4, max_iter=10)
+    seeds = oracle.frm_seeds(20, 24, 4)
+    assert f.pairs.tolist() == [[s, s] for s in seeds]
+    assert np.all(f.seed_queries == 2)               # converged in the first iteration
+    assert np.all(f.seed_converged)
+
+
+def test_identity_warp_quantised():
+    # for vectors that are not unit length, (i,i) is in M iff NN2(i) = i, and M
+    # only holds diagonal pairs or symmetric off-diagonal pairs
+    rng = np.random.default_rng(8)
+    D = synth.quantised_map(rng, 12, 12, 16)
+    m = oracle.mnn(D, D)
+    P = {tuple(p) for p in m.pairs.tolist()}
+    for i in range(144):
+        assert ((i, i) in P) == (m.row.arg[i] == i)
+    for (i, j) in P:
+        assert i == j or (j, i) in P
+
+
+# ------------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("seed", range(4))
+def test_frm_subset_mutual_monotone(seed):
+    rng = np.random.default_rng(200 + seed)
+    D1 = synth.quantised_map(rng, 16, 20, 16)
+    D2 = synth.quantised_map(rng, 18, 14, 16)
+    S, ra, ca, mutual = _brute(D1, D2)
+    f = oracle.frm(D1, D2, seed_stride=2, max_iter=10)
+    for (u, v) in f.pairs.tolist():
+        assert ra[u] == v and ca[v] == u              # every output pair is mutual
+    assert set(map(tuple, f.pairs.tolist())) <= set(mutual)
+    assert f.pairs.tolist() == sorted(map(list, set(map(tuple, f.pairs.tolist()))))
+    # scores never decrease along a trajectory
+    for s in range(len(f.seeds)):
+        seq = []
+        prev_u = f.seeds[s]
+        for t in range(10):
+            u_in, v, u_out = f.traj[s, t]
+            if u_in < 0:
+                break
+            assert u_in == prev_u
+            seq.append(S[u_in, v])
+            if u_out >= 0:
+                seq.append(S[u_out, v])
+                prev_u = u_out
+        assert all(a <= b for a, b in zip(seq, seq[1:])), seq
+
+
+def test_mnn_symmetry_and_uniqueness():
+    rng = np.random.default_rng(9)
+    D1 = synth.quantised_map(rng, 13, 17, 24)
+    D2 = synth.quantised_map(rng, 15, 12, 24)
+    a = oracle.mnn(D1, D2).pairs
+    b = oracle.mnn(D2, D1).pairs
+    assert sorted(map(tuple, a.tolist())) == sorted((j, i) for i, j in b.tolist())
+    assert len(set(a[:, 0])) == len(a) and len(set(a[:, 1])) == len(a)
+
+
+def test_frm_on_smooth_pair_converges_and_is_mutual():
+    D1, D2 = synth.smooth_pair(3, 48, 64, 24)
+    D1 = synth.to_storage(D1, "f16")
+    D2 = synth.to_storage(D2, "f16")
+    f = oracle.frm(D1, D2, seed_stride=8, max_iter=10)
+    m = oracle.mnn(D1, D2)
+    assert len(f.pairs) > 0.5 * len(f.seeds)
+    assert set(map(tuple, f.pairs.tolist())) <= set(map(tuple, m.pairs.tolist()))
+    # the active counts shrink and match the per-seed query counts
+    assert f.active_per_half.sum() == f.seed_queries.sum()
+
+
+def test_thread_count_does_not_change_results():
+    D1, D2 = synth.quantised_pair(4, 20, 20, 18, 22, 16)
+    a = oracle.frm(D1, D2, seed_stride=3, max_iter=10, threads=1)
+    b = oracle.frm(D1, D2, seed_stride=3, max_iter=10, threads=0)
+    assert np.array_equal(a.pairs, b.pairs) and np.array_equal(a.traj, b.traj)
+    m1 = oracle.mnn(D1, D2, threads=1)
+    m2 = oracle.mnn(D1, D2, threads=0)
+    assert np.array_equal(m1.pairs, m2.pairs)
+
+
+def test_quantised_values_exact_in_storage_types():
+    rng = np.random.default_rng(1)
+    q = synth.quantised_map(rng, 8, 8, 16)
+    k = q * 64
+    assert np.all(np.abs(k) <= 127) and np.array_equal(k, np.rint(k))
+    for dt in ("f16", "bf16"):
+        assert np.array_equal(synth.to_storage(q, dt).double().numpy(), q)
+
+
+def test_workloads_have_stated_shapes():
+    w = synth.WORKLOADS["frm_512x384"]
+    assert (w.H, w.W, w.d, w.seed_stride, w.max_iter) == (384, 512, 24, 8, 10)
+    assert len(oracle.frm_seeds(w.H, w.W, w.seed_stride)) == 3072
+    b = synth.WORKLOADS["frm_batched_64x512x288"]
+    assert (b.pairs, b.H, b.W, b.occlusion) == (64, 288, 512, 0.30)
