@@ -1,0 +1,166 @@
+/*
+ * rnn.h - reciprocal nearest-neighbour matching on B200 (sm_100a).
+ *
+ * A C ABI over hand-written CUDA kernels.  The operations are those of dense
+ * descriptor matching in MASt3R:
+ *
+ *   descriptors   D1 in R^{H1 x W1 x d}, D2 in R^{H2 x W2 x d}, one d-vector
+ *                 per pixel (cv-learn.com "MASt3R" note, section "Method and
+ *                 architecture", matching head).  Stored channel-last and
+ *                 row-major as fp16 or bf16: element (y, x, c) of a map is at
+ *                 offset (y*W + x)*d + c.  Pixel index p = y*W + x.
+ *   score         s(i, j) = sum_c D1[i][c] * D2[j][c], accumulated in fp32.
+ *   NN2(i)        the lowest j with the largest s(i, j); NN1(j) likewise over
+ *                 i.  (The pages name nearest neighbours without a metric or a
+ *                 tie rule; the descriptors are unit vectors, so the largest
+ *                 dot product is also the smallest Euclidean distance.)
+ *   M             {(i, j) : j = NN2(i) and i = NN1(j)}, the reciprocal set
+ *                 (same note, paragraph "Fast reciprocal matching (FRM)").
+ *
+ * Conventions for every entry point:
+ *   - Every array argument is a DEVICE pointer owned by the caller; the
+ *     library never allocates, frees or synchronises, and every result
+ *     (including counts) is ordered on `stream` like a kernel's output.
+ *   - Descriptor pointers must be 16-byte aligned and d a multiple of 8
+ *     (RNN_EALIGN otherwise); 8 <= d <= 256 (RNN_EUNSUPPORTED above).
+ *   - Inputs must be finite and their scores finite in fp32; NaN or Inf gives
+ *     undefined matches (but no out-of-bounds access).
+ *   - Argument errors are returned before anything is launched.  A launch
+ *     failure returns RNN_ECUDA.  The kernels' internal waits are bounded;
+ *     if one runs out the kernel stops early and records it in the workspace,
+ *     which rnn_workspace_status() reports as RNN_ETIMEOUT.
+ *   - Calls that share a workspace must not overlap on the device.
+ *   - The GPU must be sm_100 (B200); otherwise RNN_EUNSUPPORTED.
+ *   - Pairs are written as int32 (i, j) = (image-1 pixel, image-2 pixel).
+ */
+#ifndef RNN_H
+#define RNN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *rnn_stream_t;
+
+typedef enum rnn_status {
+  RNN_OK = 0,
+  RNN_EINVAL = 1,       /* null pointer, non-positive size, bad stride or count */
+  RNN_EALIGN = 2,       /* d not a multiple of 8, or a pointer not 16-byte aligned */
+  RNN_ECAPACITY = 3,    /* output capacity below the guaranteed maximum */
+  RNN_ECUDA = 4,        /* a CUDA runtime or driver call failed */
+  RNN_ETIMEOUT = 5,     /* a kernel's bounded wait ran out (see rnn_workspace_status) */
+  RNN_EUNSUPPORTED = 6, /* d > 256, too many pairs in a batch, or not an sm_100 GPU */
+  RNN_EWORKSPACE = 7    /* workspace missing, too small or not 256-byte aligned */
+} rnn_status;
+
+typedef enum rnn_dtype { RNN_F16 = 0, RNN_BF16 = 1 } rnn_dtype;
+
+/* Largest batch of the batched FRM entry point. */
+#define RNN_MAX_BATCH 1024
+
+/* Human-readable name of a status. */
+const char *rnn_status_string(rnn_status s);
+
+/* Version of this ABI (incremented on any signature change). */
+int rnn_abi_version(void);
+
+/*
+ * Device-side status of the most recent call that used `workspace`:
+ * synchronises `stream`, then returns RNN_ETIMEOUT if a kernel of that call
+ * gave up on a bounded wait, else RNN_OK (RNN_ECUDA if the copy fails).
+ */
+rnn_status rnn_workspace_status(const void *workspace, rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Nearest neighbours of a set of queries (the NN1 / NN2 operator).
+ *
+ *   Q          [nq][d] query descriptors.
+ *   X          [nx][d] candidate descriptors.
+ *   idx_out    [nq] int32: NN of each query among the rows of X (lowest index
+ *              among equal largest scores).
+ *   score_out  [nq] float: that largest score (may be NULL).
+ *   workspace  at least rnn_nn_workspace_size(nq) bytes, 256-byte aligned.
+ * nq may be 0 (then Q and idx_out may be NULL and only the workspace status is
+ * reset); nx must be >= 1.
+ */
+size_t rnn_nn_workspace_size(int64_t nq);
+rnn_status rnn_nn_argmax(const void *Q, int64_t nq, const void *X, int64_t nx, int d,
+                         rnn_dtype dtype, int32_t *idx_out, float *score_out, void *workspace,
+                         size_t ws_bytes, rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Exhaustive reciprocal set M between two maps (cv-learn.com "MASt3R" note,
+ * paragraph "Fast reciprocal matching (FRM)": the O(W^2 H^2) mutual-NN set).
+ *
+ *   pairs_out  [cap][2] int32: M in increasing i.  cap >= min(H1*W1, H2*W2)
+ *              (RNN_ECAPACITY otherwise), which no M can exceed.
+ *   count_out  [1] int32: |M|.
+ *   rowarg_out [H1*W1] NN2 of every D1 pixel, rowmax_out its score,
+ *   colarg_out [H2*W2] NN1 of every D2 pixel, colmax_out its score;
+ *              each of these four may be NULL.
+ *   workspace  at least rnn_mnn_workspace_size(H1, W1, H2, W2) bytes.
+ */
+size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2);
+rnn_status rnn_mnn_exhaustive(const void *D1, int H1, int W1, const void *D2, int H2, int W2,
+                              int d, rnn_dtype dtype, int32_t *pairs_out, int64_t cap,
+                              int32_t *count_out, int32_t *rowarg_out, float *rowmax_out,
+                              int32_t *colarg_out, float *colmax_out, void *workspace,
+                              size_t ws_bytes, rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fast Reciprocal Matching (cv-learn.com "MASt3R" note, paragraph "Fast
+ * reciprocal matching (FRM)"; loop semantics of the fast_reciprocal_NNs
+ * function quoted in the staskaer.github.io DUSt3R/MASt3R blog, MASt3R
+ * matching section):
+ *
+ *   seeds  u on image 1 at rows y = S/2, S/2+S, ... < H1 and columns
+ *          x = S/2, S/2+S, ... < W1 (S = seed_stride, integer halving),
+ *          ascending; U = seeds, V = -1, U_old = U, V_old = V, all active.
+ *   loop   for t = 1 .. max_iter, while some seed is active:
+ *            V = NN2(U) for the active seeds; deactivate those with V == V_old;
+ *            U = NN1(V) for the still-active seeds; deactivate those with
+ *            U == U_old; stop after iteration max_iter; else U_old = U,
+ *            V_old = V.
+ *   output the (U, V) of the seeds that are no longer active, unique, sorted
+ *          by U.  Every output pair is in M.
+ *
+ * The whole loop runs on the device: 4*max_iter + 2 kernel launches, no host
+ * synchronisation.
+ *
+ *   seed_stride >= 1, max_iter >= 1 (RNN_EINVAL otherwise).
+ *   pairs_out   [cap][2] int32, cap >= rnn_frm_max_pairs(...).
+ *   count_out   [1] int32.
+ *   seed_state_out  (may be NULL) [k][4] int32 per seed: final U, final V,
+ *               number of NN queries made for it, 1 if converged else 0.
+ *   workspace   at least rnn_frm_workspace_size(1, H1, W1, H2, W2, seed_stride).
+ */
+int64_t rnn_frm_num_seeds(int H1, int W1, int seed_stride);
+int64_t rnn_frm_max_pairs(int H1, int W1, int H2, int W2, int seed_stride);
+size_t rnn_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int seed_stride);
+rnn_status rnn_frm_match(const void *D1, int H1, int W1, const void *D2, int H2, int W2, int d,
+                         rnn_dtype dtype, int seed_stride, int max_iter, int32_t *pairs_out,
+                         int64_t cap, int32_t *count_out, int32_t *seed_state_out,
+                         void *workspace, size_t ws_bytes, rnn_stream_t stream);
+
+/*
+ * FRM over B independent pairs in one launch sequence.  Pair b reads
+ * D1 + b*d1_batch_stride and D2 + b*d2_batch_stride (strides in elements,
+ * multiples of 8, at least H*W*d) and writes pairs_out + b*cap*2,
+ * count_out[b] and seed_state_out + b*k*4.  1 <= B <= RNN_MAX_BATCH.
+ */
+rnn_status rnn_frm_match_batched(int B, const void *D1, int64_t d1_batch_stride, const void *D2,
+                                 int64_t d2_batch_stride, int H1, int W1, int H2, int W2, int d,
+                                 rnn_dtype dtype, int seed_stride, int max_iter,
+                                 int32_t *pairs_out, int64_t cap, int32_t *count_out,
+                                 int32_t *seed_state_out, void *workspace, size_t ws_bytes,
+                                 rnn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RNN_H */

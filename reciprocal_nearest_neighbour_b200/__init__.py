@@ -1,1 +1,259 @@
-"""Reciprocal nearest-neighbour matching on B200 (sm_100a)."""
+"""Reciprocal nearest-neighbour matching on B200 (sm_100a).
+
+Thin PyTorch binding of ``librnn.so`` (C ABI in ``include/rnn.h``): it checks
+shapes, allocates outputs and workspaces with torch (device memory only) and
+passes raw pointers and the current CUDA stream.  Every step of the matching
+runs in the library's CUDA kernels; there is no CPU path.
+
+Descriptor maps are ``[H, W, d]`` (or ``[B, H, W, d]`` for the batched FRM)
+contiguous fp16/bf16 CUDA tensors; pixel index ``p = y*W + x``.
+
+* ``nn_argmax(Q, X)``: NN of every query row among the rows of X (largest dot
+  product, lowest index on ties) and its score.
+* ``mnn_exhaustive(D1, D2)``: the reciprocal set
+  M = {(i, j) | j = NN2(D1_i) and i = NN1(D2_j)} (cv-learn.com "MASt3R"
+  note, paragraph "Fast reciprocal matching (FRM)").
+* ``frm_match`` / ``frm_match_batched``: Fast Reciprocal Matching from grid
+  seeds, with the loop of the quoted ``fast_reciprocal_NNs``
+  (staskaer.github.io DUSt3R/MASt3R blog, MASt3R matching section).
+
+Results stay on the device; pair lists come back as ``(pairs, count)`` with
+``pairs`` a ``[cap, 2]`` int32 buffer and ``count`` a device int32 tensor;
+``trim(pairs, count)`` cuts the buffer to length (this synchronises).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import RNNError, RNNLibraryError  # noqa: F401
+
+__all__ = [
+    "nn_argmax", "mnn_exhaustive", "frm_match", "frm_match_batched", "frm_num_seeds",
+    "frm_max_pairs", "workspace_status", "trim", "MNNResult", "FRMResult", "RNNError",
+    "RNNLibraryError", "FRMPlan",
+]
+
+_DT = {torch.float16: _lib.RNN_F16, torch.bfloat16: _lib.RNN_BF16}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"descriptors must be float16 or bfloat16, got {t.dtype}")
+    return _DT[t.dtype]
+
+
+def _check_map(t: torch.Tensor, name: str, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns blocks aligned to at least 512 bytes
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def workspace_status(workspace: torch.Tensor) -> None:
+    """Raise RNNError(RNN_ETIMEOUT) if the last call on `workspace` gave up on a wait."""
+    lib = _lib.load()
+    _lib.check(lib.rnn_workspace_status(workspace.data_ptr(), _stream(workspace)),
+               "rnn_workspace_status")
+
+
+def trim(pairs: torch.Tensor, count: torch.Tensor) -> torch.Tensor:
+    """``pairs[:count]`` (reads the count back to the host)."""
+    return pairs[: int(count.reshape(-1)[0].item())]
+
+
+def nn_argmax(Q: torch.Tensor, X: torch.Tensor, *, workspace: Optional[torch.Tensor] = None,
+              idx_out: Optional[torch.Tensor] = None, score_out: Optional[torch.Tensor] = None,
+              with_scores: bool = True):
+    """NN of each row of ``Q [nq, d]`` among the rows of ``X [nx, d]``.
+
+    Returns ``(idx int32 [nq], score float32 [nq] or None)``.
+    """
+    _check_map(Q, "Q", 2)
+    _check_map(X, "X", 2)
+    if Q.dtype != X.dtype or Q.shape[1] != X.shape[1]:
+        raise ValueError("Q and X must share dtype and d")
+    lib = _lib.load()
+    nq, d = Q.shape
+    nx = X.shape[0]
+    dev = Q.device
+    if idx_out is None:
+        idx_out = torch.empty(nq, dtype=torch.int32, device=dev)
+    if score_out is None and with_scores:
+        score_out = torch.empty(nq, dtype=torch.float32, device=dev)
+    need = lib.rnn_nn_workspace_size(nq)
+    if workspace is None:
+        workspace = _workspace(need, dev)
+    _lib.check(lib.rnn_nn_argmax(Q.data_ptr(), nq, X.data_ptr(), nx, d, _dtype_code(Q),
+                                 idx_out.data_ptr(), _ptr(score_out), workspace.data_ptr(),
+                                 workspace.numel(), _stream(Q)), "rnn_nn_argmax")
+    return idx_out, score_out
+
+
+@dataclass
+class MNNResult:
+    pairs: torch.Tensor            # [cap, 2] int32 buffer; the first `count` rows hold M
+    count: torch.Tensor            # [1] int32 on the device
+    rowarg: Optional[torch.Tensor] = None   # [H1*W1] NN2 of every D1 pixel
+    rowmax: Optional[torch.Tensor] = None
+    colarg: Optional[torch.Tensor] = None   # [H2*W2] NN1 of every D2 pixel
+    colmax: Optional[torch.Tensor] = None
+
+    def trimmed(self) -> torch.Tensor:
+        return trim(self.pairs, self.count)
+
+
+def mnn_exhaustive(D1: torch.Tensor, D2: torch.Tensor, *, with_nn: bool = False,
+                   workspace: Optional[torch.Tensor] = None,
+                   out: Optional[MNNResult] = None) -> MNNResult:
+    """Exhaustive reciprocal NN set between ``D1 [H1, W1, d]`` and ``D2 [H2, W2, d]``."""
+    _check_map(D1, "D1", 3)
+    _check_map(D2, "D2", 3)
+    if D1.dtype != D2.dtype or D1.shape[2] != D2.shape[2]:
+        raise ValueError("D1 and D2 must share dtype and d")
+    lib = _lib.load()
+    H1, W1, d = D1.shape
+    H2, W2, _ = D2.shape
+    n1, n2 = H1 * W1, H2 * W2
+    dev = D1.device
+    if out is None:
+        out = MNNResult(torch.empty((min(n1, n2), 2), dtype=torch.int32, device=dev),
+                        torch.zeros(1, dtype=torch.int32, device=dev))
+        if with_nn:
+            out.rowarg = torch.empty(n1, dtype=torch.int32, device=dev)
+            out.rowmax = torch.empty(n1, dtype=torch.float32, device=dev)
+            out.colarg = torch.empty(n2, dtype=torch.int32, device=dev)
+            out.colmax = torch.empty(n2, dtype=torch.float32, device=dev)
+    need = lib.rnn_mnn_workspace_size(H1, W1, H2, W2)
+    if workspace is None:
+        workspace = _workspace(need, dev)
+    _lib.check(lib.rnn_mnn_exhaustive(
+        D1.data_ptr(), H1, W1, D2.data_ptr(), H2, W2, d, _dtype_code(D1), out.pairs.data_ptr(),
+        out.pairs.shape[0], out.count.data_ptr(), _ptr(out.rowarg), _ptr(out.rowmax),
+        _ptr(out.colarg), _ptr(out.colmax), workspace.data_ptr(), workspace.numel(),
+        _stream(D1)), "rnn_mnn_exhaustive")
+    return out
+
+
+def frm_num_seeds(H1: int, W1: int, seed_stride: int) -> int:
+    return int(_lib.load().rnn_frm_num_seeds(H1, W1, seed_stride))
+
+
+def frm_max_pairs(H1: int, W1: int, H2: int, W2: int, seed_stride: int) -> int:
+    return int(_lib.load().rnn_frm_max_pairs(H1, W1, H2, W2, seed_stride))
+
+
+@dataclass
+class FRMResult:
+    pairs: torch.Tensor                      # [B, cap, 2] int32 (B = 1 for frm_match)
+    count: torch.Tensor                      # [B] int32 on the device
+    seed_state: Optional[torch.Tensor] = None  # [B, k, 4]: U, V, queries, converged
+
+    def trimmed(self, b: int = 0) -> torch.Tensor:
+        return self.pairs[b, : int(self.count[b].item())]
+
+
+class FRMPlan:
+    """Preallocated workspace and outputs for repeated FRM calls of one shape.
+
+    ``plan.run(D1, D2)`` only marshals pointers into the ABI, so it can be
+    captured in a CUDA graph.
+    """
+
+    def __init__(self, B: int, H1: int, W1: int, H2: int, W2: int, d: int, dtype: torch.dtype,
+                 seed_stride: int = 8, max_iter: int = 10, device="cuda",
+                 with_seed_state: bool = False):
+        lib = _lib.load()
+        self.B, self.H1, self.W1, self.H2, self.W2, self.d = B, H1, W1, H2, W2, d
+        self.dtype, self.seed_stride, self.max_iter = dtype, seed_stride, max_iter
+        self.k = int(lib.rnn_frm_num_seeds(H1, W1, seed_stride))
+        self.cap = max(1, int(lib.rnn_frm_max_pairs(H1, W1, H2, W2, seed_stride)))
+        dev = torch.device(device)
+        self.workspace = _workspace(lib.rnn_frm_workspace_size(B, H1, W1, H2, W2, seed_stride),
+                                    dev)
+        self.result = FRMResult(
+            torch.empty((B, self.cap, 2), dtype=torch.int32, device=dev),
+            torch.zeros(B, dtype=torch.int32, device=dev),
+            torch.empty((B, max(self.k, 1), 4), dtype=torch.int32, device=dev)
+            if with_seed_state else None)
+
+    def run(self, D1: torch.Tensor, D2: torch.Tensor) -> FRMResult:
+        batched = D1.dim() == 4
+        _check_map(D1, "D1", 4 if batched else 3)
+        _check_map(D2, "D2", 4 if batched else 3)
+        B = D1.shape[0] if batched else 1
+        if (B, *D1.shape[-3:]) != (self.B, self.H1, self.W1, self.d) or \
+                tuple(D2.shape[-3:]) != (self.H2, self.W2, self.d) or \
+                (batched and D2.shape[0] != B):
+            raise ValueError("maps do not match the plan's shape")
+        if D1.dtype != self.dtype or D2.dtype != self.dtype:
+            raise ValueError("maps do not match the plan's dtype")
+        lib = _lib.load()
+        r = self.result
+        n1, n2 = self.H1 * self.W1 * self.d, self.H2 * self.W2 * self.d
+        _lib.check(lib.rnn_frm_match_batched(
+            B, D1.data_ptr(), n1, D2.data_ptr(), n2, self.H1, self.W1, self.H2, self.W2, self.d,
+            _DT[self.dtype], self.seed_stride, self.max_iter, r.pairs.data_ptr(), self.cap,
+            r.count.data_ptr(), _ptr(r.seed_state), self.workspace.data_ptr(),
+            self.workspace.numel(), _stream(D1)), "rnn_frm_match_batched")
+        return r
+
+
+def frm_match(D1: torch.Tensor, D2: torch.Tensor, seed_stride: int = 8, max_iter: int = 10, *,
+              with_seed_state: bool = False, workspace: Optional[torch.Tensor] = None
+              ) -> FRMResult:
+    """Fast Reciprocal Matching of ``D1 [H1, W1, d]`` against ``D2 [H2, W2, d]``."""
+    _check_map(D1, "D1", 3)
+    _check_map(D2, "D2", 3)
+    if D1.dtype != D2.dtype or D1.shape[2] != D2.shape[2]:
+        raise ValueError("D1 and D2 must share dtype and d")
+    lib = _lib.load()
+    H1, W1, d = D1.shape
+    H2, W2, _ = D2.shape
+    dev = D1.device
+    k = int(lib.rnn_frm_num_seeds(H1, W1, seed_stride)) if seed_stride >= 1 else 0
+    cap = max(1, int(lib.rnn_frm_max_pairs(H1, W1, H2, W2, seed_stride)) if seed_stride >= 1
+              else 1)
+    out = FRMResult(torch.empty((1, cap, 2), dtype=torch.int32, device=dev),
+                    torch.zeros(1, dtype=torch.int32, device=dev),
+                    torch.empty((1, max(k, 1), 4), dtype=torch.int32, device=dev)
+                    if with_seed_state else None)
+    if workspace is None:
+        workspace = _workspace(lib.rnn_frm_workspace_size(1, H1, W1, H2, W2, seed_stride), dev)
+    _lib.check(lib.rnn_frm_match(
+        D1.data_ptr(), H1, W1, D2.data_ptr(), H2, W2, d, _dtype_code(D1), seed_stride, max_iter,
+        out.pairs.data_ptr(), cap, out.count.data_ptr(), _ptr(out.seed_state),
+        workspace.data_ptr(), workspace.numel(), _stream(D1)), "rnn_frm_match")
+    return out
+
+
+def frm_match_batched(D1: torch.Tensor, D2: torch.Tensor, seed_stride: int = 8,
+                      max_iter: int = 10, *, with_seed_state: bool = False) -> FRMResult:
+    """FRM over ``B`` independent pairs: ``D1 [B, H1, W1, d]``, ``D2 [B, H2, W2, d]``."""
+    _check_map(D1, "D1", 4)
+    _check_map(D2, "D2", 4)
+    if D1.shape[0] != D2.shape[0] or D1.dtype != D2.dtype or D1.shape[3] != D2.shape[3]:
+        raise ValueError("D1 and D2 must share B, dtype and d")
+    B, H1, W1, d = D1.shape
+    _, H2, W2, _ = D2.shape
+    plan = FRMPlan(B, H1, W1, H2, W2, d, D1.dtype, seed_stride, max_iter, D1.device,
+                   with_seed_state)
+    return plan.run(D1, D2)

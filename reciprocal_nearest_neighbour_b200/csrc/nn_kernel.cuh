@@ -1,0 +1,646 @@
+// Fused similarity + argmax on the 5th-generation tensor cores.
+//
+// For a tile of 128 query descriptors and a stream of candidate tiles, the
+// scores S = Q * X^T are accumulated in fp32 in tensor memory (tcgen05.mma,
+// kind::f16) and reduced on the fly to the largest score of each query row
+// and the lowest candidate index that reaches it.  No score ever leaves the
+// SM.  This is the NN1/NN2 operator of the reciprocal set and of Fast
+// Reciprocal Matching (cv-learn.com "MASt3R" note, paragraph "Fast reciprocal
+// matching (FRM)"), on the dot-product reading of "nearest".
+//
+// Work decomposition.  A launch holds up to two "families" of problems (the
+// two sweeps of the exhaustive set, or the pairs of a batched FRM half-step).
+// A family has `nbatch` independent problems; problem b has `count_b`
+// queries (fixed, or read from device memory) and `n_cand` candidates.  Each
+// problem's queries are cut into 128-row m-tiles; each m-tile's candidate
+// range is cut into S contiguous splits.  A work unit is one (m-tile, split);
+// CTAs take units round-robin.  Partial results meet in one 64-bit key per
+// query: the score bits in the upper word (ordered as unsigned integers) and
+// the complement of the index in the lower word, merged with atomicMax, so
+// the merge gives the largest score and then the lowest index whatever the
+// order of arrival.
+//
+// Warp roles (12 warps):
+//   warp 0      TMA producer: candidate tiles into a ring of shared-memory stages
+//   warp 1      tensor-memory owner and MMA issuer
+//   warp 2      query tiles: a TMA box when the rows are contiguous, else
+//               indexed rows gathered with plain loads into the same swizzle
+//   warp 3      idle
+//   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. and quarter
+//               (w-4)/4 of the columns of each accumulator, 32 columns at a
+//               time.  Each thread keeps its row's running maximum; when a
+//               chunk beats it, the chunk's 32 scores are kept (in a private
+//               shared-memory slot, or located at once in registers) and the
+//               lowest index reaching the maximum is found from them.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include "ptx.cuh"
+
+namespace rnn {
+
+constexpr int kBlockM = 128;
+constexpr int kThreads = 640;
+constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 16;
+constexpr int kSlotBytes = kEpiWarps * 32 * 32 * 4;  // 32 saved scores per epilogue thread
+constexpr int kMaxBatchTable = 1024;
+
+// Error bits written to the device error word.
+constexpr int kErrWaitProducer = 1 << 0;
+constexpr int kErrWaitMma = 1 << 1;
+constexpr int kErrWaitGather = 1 << 2;
+constexpr int kErrWaitEpilogue = 1 << 3;
+constexpr int kErrDrain = 1 << 4;
+
+struct NNFamily {
+  const uint16_t* q_base;       // query rows (fp16/bf16 bits), problem b at q_base + b*q_bstride
+  int64_t q_bstride;            // elements
+  const int32_t* q_list;        // optional: query position -> slot
+  const int32_t* q_index;       // optional: slot -> query row
+  int64_t slot_bstride;         // elements between problems in q_list / q_index
+  const int32_t* q_count_dev;   // optional: per-problem query counts in device memory
+  int32_t q_count;              // query count when q_count_dev is null
+  int32_t n_cand;               // candidates per problem
+  int32_t nbatch;               // problems
+  unsigned long long* keys;     // per-query packed result, problem b at keys + b*key_bstride
+  int64_t key_bstride;
+  int32_t q_tma;                // 1: query rows are contiguous, load them with the Q tensor map
+};
+
+struct NNParams {
+  NNFamily fam[2];
+  int nfam;
+  int d;            // channels (multiple of 8)
+  int kb;           // K-block width in elements: 16, 32 or 64 (32/64/128-byte swizzle)
+  int nkb;          // K-blocks; padded depth K = kb * nkb
+  int block_n;      // candidates per stage: 256 or 128
+  int stages;       // candidate ring depth
+  int qbufs;        // query tile buffers: 1 or 2
+  uint32_t idesc;   // tcgen05 instruction descriptor
+  int target_units; // units to aim for when choosing the split count
+  int min_tiles;    // fewest candidate tiles per unit (amortises the query-tile load)
+  int* err;         // device error word
+  unsigned long long wait_limit_ns;
+};
+
+// Packed key: larger is better (higher score, then lower index).
+__device__ __forceinline__ unsigned long long pack_key(float s, int idx) {
+  s = __fadd_rn(s, 0.0f);  // -0 -> +0 so that equal scores pack equally
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<unsigned long long>(o) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(idx));
+}
+__device__ __forceinline__ int key_index(unsigned long long k) {
+  return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(k));
+}
+__device__ __forceinline__ float key_score(unsigned long long k) {
+  const uint32_t o = static_cast<uint32_t>(k >> 32);
+  const uint32_t b = (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
+  return __uint_as_float(b);
+}
+
+// Shared-memory descriptor of a K-major operand tile stored with the
+// 32/64/128-byte swizzle (rows of kb elements, 8-row groups).
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, int kb) {
+  const uint32_t row_bytes = static_cast<uint32_t>(kb) * 2u;
+  const uint64_t sbo = (8u * row_bytes) >> 4;
+  const uint64_t layout = (kb == 64) ? 2u : (kb == 32) ? 4u : 6u;
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  desc |= static_cast<uint64_t>(1u) << 16;  // leading byte offset (unused with swizzle)
+  desc |= sbo << 32;
+  desc |= static_cast<uint64_t>(1u) << 46;  // descriptor version for sm_100
+  desc |= layout << 61;
+  return desc;
+}
+
+// Index of the 16-byte chunk `c` of row `r` after the swizzle of a tile with
+// kb-element rows (the same pattern the TMA unit writes).
+__device__ __forceinline__ int swz_chunk(int r, int c, int kb) {
+  if (kb == 64) return c ^ (r & 7);
+  if (kb == 32) return c ^ ((r >> 1) & 3);
+  return c ^ ((r >> 2) & 1);
+}
+
+struct UnitInfo {
+  int f, b, m, t0, t1, nrows;
+};
+
+struct SharedTables {
+  int mt_prefix[2][kMaxBatchTable + 1];  // per family: m-tile prefix over problems
+  int fam_tiles[2];                      // m-tiles per family
+  int split[2];                          // splits per m-tile per family
+  int fam_units[2];
+  int total_units;
+  int ntiles[2];                         // candidate tiles per problem
+};
+
+__device__ __forceinline__ int family_count(const NNFamily& F, int b) {
+  return F.q_count_dev ? F.q_count_dev[b] : F.q_count;
+}
+
+__device__ __forceinline__ UnitInfo decode_unit(const NNParams& p, const SharedTables& T, int u) {
+  UnitInfo ui;
+  int f = 0;
+  if (u >= T.fam_units[0]) {
+    u -= T.fam_units[0];
+    f = 1;
+  }
+  const NNFamily& F = p.fam[f];
+  const int S = T.split[f];
+  const int mt = u / S, sp = u - (u / S) * S;
+  // problem b: last b with mt_prefix[f][b] <= mt
+  int lo = 0, hi = F.nbatch;  // invariant: prefix[lo] <= mt < prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (T.mt_prefix[f][mid] <= mt) lo = mid; else hi = mid;
+  }
+  ui.f = f;
+  ui.b = lo;
+  ui.m = mt - T.mt_prefix[f][lo];
+  const int cnt = family_count(F, lo);
+  ui.nrows = min(kBlockM, cnt - ui.m * kBlockM);
+  const int nt = T.ntiles[f];
+  ui.t0 = static_cast<int>((static_cast<long long>(sp) * nt) / S);
+  ui.t1 = static_cast<int>((static_cast<long long>(sp + 1) * nt) / S);
+  return ui;
+}
+
+// Exclusive scan of `n` values (n <= kMaxBatchTable) of m-tile counts into
+// T.mt_prefix[f][0..n], by all kThreads threads.
+__device__ void build_prefix(const NNFamily& F, int* prefix, int* scratch_warp) {
+  const int n = F.nbatch;
+  const int per = (n + kThreads - 1) / kThreads;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  int vals[4];
+  int local = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int b = t * per + e;
+    int v = 0;
+    if (e < per && b < n) {
+      const int c = family_count(F, b);
+      v = (c + kBlockM - 1) / kBlockM;
+    }
+    vals[e] = v;
+    local += v;
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) scratch_warp[warp] = incl;
+  __syncthreads();
+  if (t == 0) {
+    int run = 0;
+    for (int w = 0; w < kThreads / 32; ++w) {
+      const int x = scratch_warp[w];
+      scratch_warp[w] = run;
+      run += x;
+    }
+    scratch_warp[kThreads / 32] = run;
+  }
+  __syncthreads();
+  int run = scratch_warp[warp] + incl - local;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int b = t * per + e;
+    if (e < per && b < n) prefix[b] = run;
+    run += vals[e];
+  }
+  if (t == 0) prefix[n] = scratch_warp[kThreads / 32];
+  __syncthreads();
+}
+
+// Largest of 32 values with three-input maxima (17 instructions).
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float a[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) a[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  a[10] = fmaxf(v[30], v[31]);
+  const float b0 = fmax3(a[0], a[1], a[2]), b1 = fmax3(a[3], a[4], a[5]);
+  const float b2 = fmax3(a[6], a[7], a[8]), b3 = fmaxf(a[9], a[10]);
+  return fmaxf(fmax3(b0, b1, b2), b3);
+}
+
+// Lowest k with v[k] == m (m is one of the values).
+__device__ __forceinline__ int first_equal32(const float (&v)[32], float m) {
+  int pos = 31;
+#pragma unroll
+  for (int k = 30; k >= 0; --k) pos = (v[k] == m) ? k : pos;
+  return pos;
+}
+
+template <bool kSlotLocate>
+__global__ void __launch_bounds__(kThreads, 1)
+nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUtensorMap tmap0,
+                 const __grid_constant__ CUtensorMap tmap1,
+                 const __grid_constant__ CUtensorMap qmap0,
+                 const __grid_constant__ CUtensorMap qmap1) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int kpad = p.kb * p.nkb;
+  const uint32_t stage_bytes = static_cast<uint32_t>(p.block_n) * kpad * 2;
+  const uint32_t kblk_bytes_x = static_cast<uint32_t>(p.block_n) * p.kb * 2;
+  const uint32_t q_bytes = static_cast<uint32_t>(kBlockM) * kpad * 2;
+  const uint32_t kblk_bytes_q = static_cast<uint32_t>(kBlockM) * p.kb * 2;
+
+  uint8_t* x_tiles = smem;
+  uint8_t* q_tiles = x_tiles + static_cast<size_t>(p.stages) * stage_bytes;
+  float* slots = reinterpret_cast<float*>(q_tiles + static_cast<size_t>(p.qbufs) * q_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(slots) +
+                                               (kSlotLocate ? kSlotBytes : 0));
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + p.stages;
+  uint64_t* qfull_bar = bars + 2 * p.stages;
+  uint64_t* qempty_bar = qfull_bar + 2;
+  uint64_t* tfull_bar = qempty_bar + 2;
+  uint64_t* tempty_bar = tfull_bar + 2;
+  uint64_t* drain_bar = tempty_bar + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* qrows = reinterpret_cast<int*>(misc + 4);            // [128]
+  int* scan_scratch = qrows + kBlockM;                       // [kThreads/32 + 1]
+  SharedTables* T = reinterpret_cast<SharedTables*>(scan_scratch + 32);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = static_cast<uint32_t>(2 * p.block_n);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&qfull_bar[i]), 1);
+      mbar_init(smem_u32(&qempty_bar[i]), 1);
+      mbar_init(smem_u32(&tfull_bar[i]), 1);
+      mbar_init(smem_u32(&tempty_bar[i]), kEpiWarps);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap0);
+    if (p.nfam > 1) tma_prefetch_desc(&tmap1);
+    if (p.fam[0].q_tma) tma_prefetch_desc(&qmap0);
+    if (p.nfam > 1 && p.fam[1].q_tma) tma_prefetch_desc(&qmap1);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(misc), ncols);
+    tmem_relinquish();
+  }
+
+  // unit table
+  for (int f = 0; f < 2; ++f) {
+    if (f < p.nfam) {
+      build_prefix(p.fam[f], T->mt_prefix[f], scan_scratch);
+    }
+  }
+  if (threadIdx.x == 0) {
+    int tiles_total = 0;
+    for (int f = 0; f < 2; ++f) {
+      if (f < p.nfam) {
+        T->fam_tiles[f] = T->mt_prefix[f][p.fam[f].nbatch];
+        T->ntiles[f] = (p.fam[f].n_cand + p.block_n - 1) / p.block_n;
+      } else {
+        T->fam_tiles[f] = 0;
+        T->ntiles[f] = 1;
+      }
+      tiles_total += T->fam_tiles[f];
+    }
+    int S = tiles_total > 0 ? (p.target_units + tiles_total - 1) / tiles_total : 1;
+    if (S < 1) S = 1;
+    int total = 0;
+    for (int f = 0; f < 2; ++f) {
+      const int Sf = max(1, min(S, T->ntiles[f] / max(1, p.min_tiles)));
+      T->split[f] = Sf;
+      T->fam_units[f] = T->fam_tiles[f] * Sf;
+      total += T->fam_units[f];
+    }
+    T->total_units = total;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+  const int total_units = T->total_units;
+  const uint64_t lim = p.wait_limit_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const UnitInfo ui = decode_unit(p, *T, u);
+        const CUtensorMap* map = ui.f == 0 ? &tmap0 : &tmap1;
+        for (int t = ui.t0; t < ui.t1; ++t) {
+          if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
+                         kErrWaitProducer, lim)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full_bar[stage]);
+          mbar_arrive_expect_tx(fb, stage_bytes);
+          const uint32_t dst = smem_u32(x_tiles + static_cast<size_t>(stage) * stage_bytes);
+          for (int kk = 0; kk < p.nkb; ++kk)
+            tma_load_3d(dst + kk * kblk_bytes_x, map, fb, kk * p.kb, t * p.block_n, ui.b);
+          ++issued;
+          if (++stage == p.stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // wait (bounded) for the loads still in flight before the CTA exits
+        const long long n = issued < p.stages ? issued : p.stages;
+        for (long long q = issued - n; q < issued; ++q) {
+          const int s = static_cast<int>(q % p.stages);
+          const uint32_t ph = static_cast<uint32_t>((q / p.stages) & 1);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(smem_u32(&full_bar[s]), ph)) {
+            if (globaltimer_ns() - t0 > lim) {
+              atomicOr(p.err, kErrDrain);
+              break;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    // The issue loop is latency-critical (two MMAs per 256-cycle tile at
+    // K = 32).  The whole warp runs it on warp-uniform values (so they live
+    // in uniform registers, where tcgen05.mma reads its operands), the
+    // descriptors are built once, only their 16-byte start-address field
+    // moves, and one elected lane issues.
+    int stage = 0, acc = 0, qb = 0;
+    uint32_t phase = 0, acc_phase = 0, qphase = 0;
+    bool ok = true, any = false;
+    const int ksteps = kpad / 16;
+    const int spk = p.kb / 16;                                   // K-steps per K-block
+    const uint64_t a_desc0 = make_sdesc(smem_u32(q_tiles), p.kb);
+    const uint64_t b_desc0 = make_sdesc(smem_u32(x_tiles), p.kb);
+    const uint32_t a_jump = (kblk_bytes_q - (spk - 1) * 32) >> 4;  // to the next K-block
+    const uint32_t b_jump = (kblk_bytes_x - (spk - 1) * 32) >> 4;
+    const uint32_t q_step = q_bytes >> 4, x_step = stage_bytes >> 4;
+    const uint32_t idesc = p.idesc;
+    uint64_t b_stage = b_desc0;
+    uint64_t a_unit = a_desc0;
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+      const UnitInfo ui = decode_unit(p, *T, u);
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(smem_u32(&qfull_bar[qb]), qphase, abort_flag, p.err, kErrWaitMma,
+                                lim));
+      if (!ok) break;
+      for (int t = ui.t0; t < ui.t1; ++t) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err,
+                                  kErrWaitMma, lim) &&
+                            mbar_wait(smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag,
+                                      p.err, kErrWaitMma, lim));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (acc ? static_cast<uint32_t>(p.block_n) : 0u);
+        uint64_t a = a_unit, b = b_stage;
+        if (elect_one()) {
+          int w = 0;
+          for (int k = 0; k < ksteps; ++k) {
+            umma_f16(d_tmem, a, b, idesc, k > 0 ? 1u : 0u);
+            if (++w == spk) {
+              w = 0;
+              a += a_jump;
+              b += b_jump;
+            } else {
+              a += 2;
+              b += 2;
+            }
+          }
+          umma_commit(smem_u32(&empty_bar[stage]));
+          umma_commit(smem_u32(&tfull_bar[acc]));
+        }
+        __syncwarp();
+        any = true;
+        b_stage += x_step;
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1u;
+          b_stage = b_desc0;
+        }
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) umma_commit(smem_u32(&qempty_bar[qb]));
+      __syncwarp();
+      a_unit += q_step;
+      if (++qb == p.qbufs) {
+        qb = 0;
+        qphase ^= 1u;
+        a_unit = a_desc0;
+      }
+    }
+    if (!ok && any) {
+      // let every MMA issued so far finish before tensor memory is released
+      if (elect_one()) umma_commit(smem_u32(drain_bar));
+      __syncwarp();
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(drain_bar), 0)) {
+        if (globaltimer_ns() - t0 > lim) {
+          if (lane == 0) atomicOr(p.err, kErrDrain);
+          break;
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------------------------------------------- query gather
+    int qb = 0;
+    uint32_t qphase = 0;
+    int q_last = 0;
+    uint32_t q_last_phase = 0;
+    bool q_any = false;
+    const int nch_real = p.d / 8;       // 16-byte chunks holding data
+    const int nch_row = kpad / 8;       // chunks per padded row
+    const int ch_per_kblk = p.kb / 8;
+    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+      const UnitInfo ui = decode_unit(p, *T, u);
+      if (!mbar_wait(smem_u32(&qempty_bar[qb]), qphase ^ 1u, abort_flag, p.err, kErrWaitGather,
+                     lim))
+        break;
+      const NNFamily& F = p.fam[ui.f];
+      if (F.q_tma) {
+        // contiguous query rows: one TMA box per K-block, rows past the end are zero
+        if (lane == 0) {
+          const uint32_t qf = smem_u32(&qfull_bar[qb]);
+          mbar_arrive_expect_tx(qf, q_bytes);
+          const uint32_t dst = smem_u32(q_tiles + static_cast<size_t>(qb) * q_bytes);
+          const CUtensorMap* qm = ui.f == 0 ? &qmap0 : &qmap1;
+          for (int kk = 0; kk < p.nkb; ++kk)
+            tma_load_3d(dst + kk * kblk_bytes_q, qm, qf, kk * p.kb, ui.m * kBlockM, ui.b);
+        }
+        __syncwarp();
+        q_last = qb;
+        q_last_phase = qphase;
+        q_any = true;
+        if (++qb == p.qbufs) {
+          qb = 0;
+          qphase ^= 1u;
+        }
+        continue;
+      }
+      for (int r = lane; r < kBlockM; r += 32) {
+        int row = -1;
+        if (r < ui.nrows) {
+          int pos = ui.m * kBlockM + r;
+          int slot = F.q_list ? __ldg(F.q_list + ui.b * F.slot_bstride + pos) : pos;
+          row = F.q_index ? __ldg(F.q_index + ui.b * F.slot_bstride + slot) : slot;
+        }
+        qrows[r] = row;
+      }
+      __syncwarp();
+      const uint16_t* qsrc = F.q_base + ui.b * F.q_bstride;
+      uint8_t* qdst = q_tiles + static_cast<size_t>(qb) * q_bytes;
+      const int items = kBlockM * nch_row;
+      for (int it0 = 0; it0 < items; it0 += 32 * 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int it = it0 + j * 32 + lane;
+          v[j] = make_uint4(0, 0, 0, 0);
+          if (it < items) {
+            const int r = it / nch_row, c = it - (it / nch_row) * nch_row;
+            const int row = qrows[r];
+            if (row >= 0 && c < nch_real)
+              v[j] = __ldg(reinterpret_cast<const uint4*>(qsrc + static_cast<int64_t>(row) * p.d) + c);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int it = it0 + j * 32 + lane;
+          if (it < items) {
+            const int r = it / nch_row, c = it - (it / nch_row) * nch_row;
+            const int kblk = c / ch_per_kblk, cw = c - kblk * ch_per_kblk;
+            uint8_t* dst = qdst + kblk * kblk_bytes_q + r * (p.kb * 2) +
+                           swz_chunk(r, cw, p.kb) * 16;
+            *reinterpret_cast<uint4*>(dst) = v[j];
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&qfull_bar[qb]));
+      if (++qb == p.qbufs) {
+        qb = 0;
+        qphase ^= 1u;
+      }
+    }
+    if (*abort_flag && q_any && lane == 0) {
+      // a query-tile TMA load may still be in flight: wait for it (bounded)
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(&qfull_bar[q_last]), q_last_phase)) {
+        if (globaltimer_ns() - t0 > lim) {
+          atomicOr(p.err, kErrDrain);
+          break;
+        }
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // --------------------------------------------------------- epilogue
+    const int ew = warp - kEpiWarp0;
+    const int quad = warp & 3;
+    const int part = ew >> 2;
+    const int row = quad * 32 + lane;
+    const int cols_part = p.block_n / 4;
+    // private slot of 32 floats; 16-byte unit q lives at (q ^ lane) & 7
+    float* slot = slots + (ew * 32 + lane) * 32;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+      const UnitInfo ui = decode_unit(p, *T, u);
+      const NNFamily& F = p.fam[ui.f];
+      float best = -__int_as_float(0x7f800000);
+      int arg = -1;  // slot mode: first column of the kept chunk; else the index
+      for (int t = ui.t0; t < ui.t1; ++t) {
+        if (!mbar_wait(smem_u32(&tfull_bar[acc]), acc_phase, abort_flag, p.err, kErrWaitEpilogue,
+                       lim)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int col0 = t * p.block_n + part * cols_part;   // first candidate of this part
+        const int valid = F.n_cand - col0;                    // candidates left from col0
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(acc * p.block_n + part * cols_part);
+        for (int c = 0; c < cols_part; c += 32) {
+          float v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld_regs(v);
+          if (valid - c < 32) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (c + k >= valid) v[k] = -__int_as_float(0x7f800000);
+          }
+          const float m = max32(v);
+          if (m > best) {
+            best = m;
+            if (kSlotLocate) {
+              arg = col0 + c;
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(slot + ((q ^ lane) & 7) * 4) =
+                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            } else {
+              arg = col0 + c + first_equal32(v, m);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (row < ui.nrows && arg >= 0) {
+        if (kSlotLocate) {
+          float w[32];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 x = *reinterpret_cast<const float4*>(slot + ((q ^ lane) & 7) * 4);
+            w[4 * q] = x.x;
+            w[4 * q + 1] = x.y;
+            w[4 * q + 2] = x.z;
+            w[4 * q + 3] = x.w;
+          }
+          arg += first_equal32(w, best);
+        }
+        unsigned long long* kp = F.keys + ui.b * F.key_bstride + ui.m * kBlockM + row;
+        atomicMax(kp, pack_key(best, arg));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, ncols);
+  }
+}
+
+}  // namespace rnn

@@ -1,0 +1,786 @@
+// C ABI of the reciprocal nearest-neighbour library (declared in include/rnn.h).
+//
+// Every entry point validates its arguments on the host, builds the TMA
+// descriptors of the candidate maps, and enqueues a fixed sequence of kernels
+// on the caller's stream.  No allocation, no synchronisation: scratch lives in
+// the caller's workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "nn_kernel.cuh"
+#include "rnn.h"
+
+namespace rnn {
+
+// ------------------------------------------------------------------ helpers
+constexpr size_t kAlign = 256;
+constexpr int kSmallThreads = 1024;
+constexpr int kMnnChunk = 4096;  // rows per block in the mutual test (4 per thread)
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
+
+static size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+struct Carve {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off = align_up(off + count * sizeof(T));
+    return p;
+  }
+};
+
+struct DeviceInfo {
+  int sms = 0;
+  bool sm100 = false;
+  bool smem_set = false;
+};
+
+static std::mutex g_mu;
+static DeviceInfo g_dev[64];
+
+static rnn_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RNN_ECUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (di.sms == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return RNN_ECUDA;
+    di.sm100 = (major == 10 && minor == 0);
+    di.sms = sms;
+  }
+  if (!di.sm100) return RNN_EUNSUPPORTED;
+  *out = &di;
+  return RNN_OK;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Operand geometry for a channel count d.
+struct Geometry {
+  int kb, nkb, kpad, block_n, stages, qbufs;
+  bool slot_locate;  // epilogue keeps improving chunks in shared memory
+  size_t smem;
+};
+
+static size_t tables_bytes() { return sizeof(SharedTables); }
+
+static Geometry geometry(int d) {
+  Geometry g;
+  if (d <= 16) {
+    g.kb = 16; g.nkb = 1;
+  } else if (d <= 32) {
+    g.kb = 32; g.nkb = 1;
+  } else if (d % 64 == 0) {
+    g.kb = 64; g.nkb = d / 64;
+  } else if (d % 32 == 0) {
+    g.kb = 32; g.nkb = d / 32;
+  } else {
+    g.kb = 16; g.nkb = (d + 15) / 16;
+  }
+  g.kpad = g.kb * g.nkb;
+  // small d: the argmax epilogue bounds the kernel, so it gets the 64 KB of
+  // score slots; large d: the tensor cores bound it and the slots would not fit
+  g.slot_locate = g.kpad <= 64;
+  g.block_n = g.kpad <= 64 ? 256 : 128;
+  const size_t stage = static_cast<size_t>(g.block_n) * g.kpad * 2;
+  const size_t qb = static_cast<size_t>(kBlockM) * g.kpad * 2;
+  const size_t slots = g.slot_locate ? kSlotBytes : 0;
+  const size_t fixed = 1024 /*align slack*/ + 16 + kBlockM * 4 + 32 * 4 + tables_bytes();
+  const size_t budget = 227 * 1024;
+  const size_t bars = (2 * 8 + 9) * 8;
+  const size_t avail = budget - fixed - bars - slots;
+  g.qbufs = (2 * qb + 2 * stage <= avail) ? 2 : 1;
+  size_t st = (avail - g.qbufs * qb) / stage;
+  if (st > 8) st = 8;
+  g.stages = static_cast<int>(st);
+  g.smem = fixed + (2 * g.stages + 9) * 8 + g.stages * stage + g.qbufs * qb + slots;
+  // at least half the SM's shared memory, so that two CTAs never share an SM
+  // (each one allocates all 512 tensor-memory columns)
+  if (g.smem < 116 * 1024) g.smem = 116 * 1024;
+  return g;
+}
+
+static uint32_t make_idesc(rnn_dtype dt, int block_n) {
+  const uint32_t fmt = dt == RNN_BF16 ? 1u : 0u;
+  uint32_t d = 0;
+  d |= 1u << 4;                                      // accumulator: f32
+  d |= fmt << 7;                                     // A format
+  d |= fmt << 10;                                    // B format
+  d |= static_cast<uint32_t>(block_n >> 3) << 17;    // N
+  d |= static_cast<uint32_t>(kBlockM >> 4) << 24;    // M
+  return d;
+}
+
+// [nbatch][rows][d] map with batch stride `bstride` elements, boxes of
+// `box_rows` rows (candidate tiles: g.block_n; query tiles: 128).
+static rnn_status make_map(CUtensorMap* m, const void* base, int d, int64_t rows, int nbatch,
+                           int64_t bstride, const Geometry& g, int box_rows = 0) {
+  auto fn = encode_fn();
+  if (!fn) return RNN_ECUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(nbatch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(bstride) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(g.kb),
+                       static_cast<cuuint32_t>(box_rows > 0 ? box_rows : g.block_n), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = g.kb == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : g.kb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                             : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RNN_OK : RNN_ECUDA;
+}
+
+static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const CUtensorMap& m1,
+                            const CUtensorMap& q0, const CUtensorMap& q1, const Geometry& g,
+                            DeviceInfo* di, cudaStream_t s) {
+  NNParams p = p_in;
+  p.kb = g.kb;
+  p.nkb = g.nkb;
+  p.block_n = g.block_n;
+  p.stages = g.stages;
+  p.qbufs = g.qbufs;
+  p.target_units = 8 * di->sms;
+  {
+    // a unit should hold about 4096 tensor-core cycles of work
+    const int tile_cycles = (g.kpad / 16) * (g.block_n / 2);
+    p.min_tiles = 4096 / tile_cycles > 2 ? 4096 / tile_cycles : 2;
+  }
+  p.wait_limit_ns = kWaitLimitNs;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!di->smem_set) {
+      if (cudaFuncSetAttribute(nn_argmax_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) != cudaSuccess ||
+          cudaFuncSetAttribute(nn_argmax_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) != cudaSuccess)
+        return RNN_ECUDA;
+      di->smem_set = true;
+    }
+  }
+  if (g.slot_locate)
+    nn_argmax_kernel<true><<<di->sms, kThreads, g.smem, s>>>(p, m0, m1, q0, q1);
+  else
+    nn_argmax_kernel<false><<<di->sms, kThreads, g.smem, s>>>(p, m0, m1, q0, q1);
+  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+static rnn_status check_desc(const void* p, int d) {
+  if (!p) return RNN_EINVAL;
+  if (d <= 0) return RNN_EINVAL;
+  if (d % 8 != 0 || !aligned16(p)) return RNN_EALIGN;
+  if (d > 256) return RNN_EUNSUPPORTED;
+  return RNN_OK;
+}
+
+static bool valid_dtype(rnn_dtype dt) { return dt == RNN_F16 || dt == RNN_BF16; }
+
+// -------------------------------------------------------------- small kernels
+__global__ void zero_keys_kernel(unsigned long long* a, int64_t na, unsigned long long* b,
+                                 int64_t nb, int* err) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < na + nb;
+       i += stride) {
+    if (i < na) a[i] = 0ull; else b[i - na] = 0ull;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
+}
+
+__global__ void unpack_kernel(const unsigned long long* keys, int64_t n, int32_t* idx,
+                              float* score) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += stride) {
+    const unsigned long long k = keys[i];
+    idx[i] = key_index(k);
+    if (score) score[i] = key_score(k);
+  }
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
+__device__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int warp_sums[33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? warp_sums[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    if (lane < nw) warp_sums[lane] = wi - w;
+    if (lane == nw - 1) warp_sums[32] = wi;
+  }
+  __syncthreads();
+  const int r = warp_sums[warp] + incl - v;
+  *total = warp_sums[32];
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ bool is_mutual(const unsigned long long* rowk,
+                                          const unsigned long long* colk, int64_t i, int* j) {
+  *j = key_index(rowk[i]);
+  return key_index(colk[*j]) == static_cast<int>(i);
+}
+
+// Pass 1 of the reciprocal test: mutual count per block of kMnnChunk rows,
+// and the optional per-pixel outputs.
+__global__ void mnn_count_kernel(const unsigned long long* rowk, int64_t n1,
+                                 const unsigned long long* colk, int64_t n2, int* block_counts,
+                                 int nblocks1,
+                                 int32_t* rowarg, float* rowmax, int32_t* colarg,
+                                 float* colmax) {
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kMnnChunk;
+  int c = 0;
+  for (int e = 0; e < kMnnChunk / kSmallThreads; ++e) {
+    const int64_t i = base + static_cast<int64_t>(e) * kSmallThreads + threadIdx.x;
+    if (i < n1) {
+      int j;
+      c += is_mutual(rowk, colk, i, &j) ? 1 : 0;
+      if (rowarg) rowarg[i] = j;
+      if (rowmax) rowmax[i] = key_score(rowk[i]);
+    }
+    if (i < n2) {
+      if (colarg) colarg[i] = key_index(colk[i]);
+      if (colmax) colmax[i] = key_score(colk[i]);
+    }
+  }
+  // block total
+  int total;
+  (void)block_exclusive_scan(c, &total);
+  if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < nblocks1) block_counts[blockIdx.x] = total;
+}
+
+// Pass 2: each block finds its offset from the counts of the blocks before
+// it and writes its mutual pairs in increasing i.
+__global__ void mnn_write_kernel(const unsigned long long* rowk, int64_t n1,
+                                 const unsigned long long* colk, const int* block_counts,
+                                 int nblocks, int32_t* pairs, int32_t* count_out) {
+  __shared__ int s_off;
+  int part = 0;
+  for (int b = threadIdx.x; b < blockIdx.x; b += blockDim.x) part += block_counts[b];
+  int tot;
+  (void)block_exclusive_scan(part, &tot);
+  if (threadIdx.x == 0) s_off = tot;
+  __syncthreads();
+  int off = s_off;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kMnnChunk;
+  // rows of this thread: kMnnChunk/kSmallThreads consecutive rows, so that a
+  // thread-order scan keeps increasing i
+  constexpr int per = kMnnChunk / kSmallThreads;
+  int js[per];
+  bool ms[per];
+  int c = 0;
+#pragma unroll
+  for (int e = 0; e < per; ++e) {
+    const int64_t i = base + static_cast<int64_t>(threadIdx.x) * per + e;
+    ms[e] = false;
+    if (i < n1) ms[e] = is_mutual(rowk, colk, i, &js[e]);
+    c += ms[e] ? 1 : 0;
+  }
+  int btot;
+  int pos = off + block_exclusive_scan(c, &btot);
+#pragma unroll
+  for (int e = 0; e < per; ++e) {
+    if (ms[e]) {
+      const int64_t i = base + static_cast<int64_t>(threadIdx.x) * per + e;
+      pairs[2 * static_cast<int64_t>(pos)] = static_cast<int32_t>(i);
+      pairs[2 * static_cast<int64_t>(pos) + 1] = js[e];
+      ++pos;
+    }
+  }
+  if (blockIdx.x == nblocks - 1 && threadIdx.x == 0) *count_out = off + btot;
+}
+
+// ------------------------------------------------------------------- FRM
+struct FrmState {
+  int* err;
+  int32_t* count;   // [B] active seeds
+  int32_t* U;       // [B][k]
+  int32_t* V;
+  int32_t* Uold;
+  int32_t* Vold;
+  int32_t* list;    // [B][k] active slots, compacted
+  int32_t* nq;      // [B][k] queries made per seed
+  uint8_t* act;     // [B][k] 1 while active
+  unsigned long long* keys;  // [B][k] NN result per list position
+  uint32_t* bitmap; // [B][nwords] converged image-1 pixels
+  int32_t* partner; // [B][N1] image-2 partner of a converged pixel
+  int B, k, N1, nwords;
+};
+
+// Workspace layout of a batched FRM call; returns the bytes it needs.
+static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, FrmState* st) {
+  Carve c(ws);
+  st->err = c.take<int>(64);
+  st->count = c.take<int32_t>(B);
+  st->U = c.take<int32_t>(B * k);
+  st->V = c.take<int32_t>(B * k);
+  st->Uold = c.take<int32_t>(B * k);
+  st->Vold = c.take<int32_t>(B * k);
+  st->list = c.take<int32_t>(B * k);
+  st->nq = c.take<int32_t>(B * k);
+  st->act = c.take<uint8_t>(B * k);
+  st->keys = c.take<unsigned long long>(B * k);
+  const int64_t nwords = (N1 + 31) / 32;
+  st->bitmap = c.take<uint32_t>(B * nwords);
+  st->partner = c.take<int32_t>(B * N1);
+  st->B = B;
+  st->k = static_cast<int>(k);
+  st->N1 = static_cast<int>(N1);
+  st->nwords = static_cast<int>(nwords);
+  return c.off;
+}
+
+static size_t frm_bytes(int B, int64_t k, int64_t N1) {
+  FrmState st;
+  return frm_layout(nullptr, B, k, N1, &st);
+}
+
+__global__ void frm_init_kernel(FrmState st, int W1, int S) {
+  const int x0 = S / 2;
+  const int nx = W1 > x0 ? (W1 - x0 + S - 1) / S : 0;
+  const int64_t nseed = static_cast<int64_t>(st.B) * st.k;
+  const int64_t nbits = static_cast<int64_t>(st.B) * st.nwords;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+       t < nseed + nbits; t += stride) {
+    if (t < nseed) {
+      const int s = static_cast<int>(t % st.k);
+      const int iy = s / nx, ix = s - (s / nx) * nx;
+      const int32_t u = (x0 + iy * S) * W1 + (x0 + ix * S);
+      st.U[t] = u;
+      st.Uold[t] = u;
+      st.V[t] = -1;
+      st.Vold[t] = -1;
+      st.list[t] = s;
+      st.nq[t] = 0;
+      st.act[t] = 1;
+      st.keys[t] = 0ull;
+    } else {
+      st.bitmap[t - nseed] = 0u;
+    }
+  }
+  if (blockIdx.x == 0) {
+    for (int b = threadIdx.x; b < st.B; b += blockDim.x) st.count[b] = st.k;
+    if (threadIdx.x == 0) *st.err = 0;
+  }
+}
+
+// Result of one half-step for pair blockIdx.x: store the NN found for every
+// active seed, apply the convergence test, refresh the old copies at the end
+// of an iteration, and compact the list of seeds that stay active.
+__global__ void frm_update_kernel(FrmState st, int nn2_half, int last_iter) {
+  __shared__ int s_out;
+  const int b = blockIdx.x;
+  const int64_t base = static_cast<int64_t>(b) * st.k;
+  const int n = st.count[b];
+  if (threadIdx.x == 0) s_out = 0;
+  __syncthreads();
+  for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    int s = -1, still = 0;
+    if (i < n) {
+      s = st.list[base + i];
+      const unsigned long long key = st.keys[base + i];
+      st.keys[base + i] = 0ull;
+      const int j = key_index(key);
+      st.nq[base + s] += 1;
+      if (nn2_half) {
+        st.V[base + s] = j;
+        still = j != st.Vold[base + s];
+      } else {
+        st.U[base + s] = j;
+        still = j != st.Uold[base + s];
+        if (still && !last_iter) {
+          st.Uold[base + s] = j;
+          st.Vold[base + s] = st.V[base + s];
+        }
+      }
+      if (!still) st.act[base + s] = 0;
+    }
+    int tot;
+    const int pos = block_exclusive_scan(still, &tot);  // also orders reads before writes
+    if (still) st.list[base + s_out + pos] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) s_out += tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) st.count[b] = s_out;
+}
+
+// Unique converged pairs of pair blockIdx.x, sorted by the image-1 pixel.
+__global__ void frm_merge_kernel(FrmState st, int32_t* pairs, int64_t cap, int32_t* count_out,
+                                 int32_t* seed_state) {
+  const int b = blockIdx.x;
+  const int64_t base = static_cast<int64_t>(b) * st.k;
+  uint32_t* bm = st.bitmap + static_cast<int64_t>(b) * st.nwords;
+  int32_t* partner = st.partner + static_cast<int64_t>(b) * st.N1;
+  for (int s = threadIdx.x; s < st.k; s += blockDim.x) {
+    const int conv = st.act[base + s] == 0;
+    const int32_t u = st.U[base + s], v = st.V[base + s];
+    if (conv) {
+      atomicOr(bm + (u >> 5), 1u << (u & 31));
+      partner[u] = v;
+    }
+    if (seed_state) {
+      int32_t* o = seed_state + (base + s) * 4;
+      o[0] = u;
+      o[1] = v;
+      o[2] = st.nq[base + s];
+      o[3] = conv;
+    }
+  }
+  __syncthreads();
+  const int per = (st.nwords + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * per;
+  const int w1 = min(st.nwords, w0 + per);
+  int c = 0;
+  for (int w = w0; w < w1; ++w) c += __popc(__ldcg(bm + w));
+  int tot;
+  int pos = block_exclusive_scan(c, &tot);
+  int32_t* out = pairs + static_cast<int64_t>(b) * cap * 2;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = __ldcg(bm + w);
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      const int u = w * 32 + bit;
+      out[2 * static_cast<int64_t>(pos)] = u;
+      out[2 * static_cast<int64_t>(pos) + 1] = __ldcg(partner + u);
+      ++pos;
+    }
+  }
+  if (threadIdx.x == 0) count_out[b] = tot;
+}
+
+static int grid_for(int64_t n, int sms) {
+  int64_t g = (n + kSmallThreads - 1) / kSmallThreads;
+  if (g > 4LL * sms) g = 4LL * sms;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+static int64_t num_seeds(int H, int W, int S) {
+  const int o = S / 2;
+  const int64_t ny = H > o ? (H - o + S - 1) / S : 0;
+  const int64_t nx = W > o ? (W - o + S - 1) / S : 0;
+  return ny * nx;
+}
+
+static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, int64_t bs2, int H1,
+                          int W1, int H2, int W2, int d, rnn_dtype dt, int S, int max_iter,
+                          int32_t* pairs, int64_t cap, int32_t* count_out, int32_t* seed_state,
+                          void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (B < 1) return RNN_EINVAL;
+  if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
+  if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || S < 1 || max_iter < 1) return RNN_EINVAL;
+  if (!valid_dtype(dt)) return RNN_EINVAL;
+  rnn_status st0 = check_desc(D1, d);
+  if (st0 != RNN_OK) return st0;
+  st0 = check_desc(D2, d);
+  if (st0 != RNN_OK) return st0;
+  const int64_t N1 = static_cast<int64_t>(H1) * W1, N2 = static_cast<int64_t>(H2) * W2;
+  if (N1 > INT32_MAX || N2 > INT32_MAX) return RNN_EINVAL;
+  if (bs1 < N1 * d || bs2 < N2 * d || bs1 % 8 != 0 || bs2 % 8 != 0) return RNN_EINVAL;
+  if (!pairs || !count_out) return RNN_EINVAL;
+  const int64_t k = num_seeds(H1, W1, S);
+  const int64_t need = k < N2 ? k : N2;
+  if (cap < need) return RNN_ECAPACITY;
+  if (!ws || !aligned256(ws) || ws_bytes < frm_bytes(B, k, N1)) return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  rnn_status r = device_info(&di);
+  if (r != RNN_OK) return r;
+
+  FrmState st;
+  frm_layout(ws, B, k, N1, &st);
+  const Geometry g = geometry(d);
+  if (k == 0) {
+    // no seeds: every count is zero
+    if (cudaMemsetAsync(count_out, 0, sizeof(int32_t) * B, s) != cudaSuccess) return RNN_ECUDA;
+    if (cudaMemsetAsync(st.err, 0, sizeof(int), s) != cudaSuccess) return RNN_ECUDA;
+    return RNN_OK;
+  }
+  CUtensorMap map1, map2;
+  if ((r = make_map(&map1, D1, d, N1, B, bs1, g)) != RNN_OK) return r;
+  if ((r = make_map(&map2, D2, d, N2, B, bs2, g)) != RNN_OK) return r;
+
+  frm_init_kernel<<<grid_for(B * k + B * st.nwords, di->sms), kSmallThreads, 0, s>>>(st, W1, S);
+  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+
+  NNParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.nfam = 1;
+  p.d = d;
+  p.idesc = make_idesc(dt, g.block_n);
+  p.err = st.err;
+  NNFamily& F = p.fam[0];
+  F.slot_bstride = k;
+  F.q_list = st.list;
+  F.q_count_dev = st.count;
+  F.nbatch = B;
+  F.keys = st.keys;
+  F.key_bstride = k;
+  for (int it = 1; it <= max_iter; ++it) {
+    // half-step 1: V = NN2(U)
+    F.q_base = static_cast<const uint16_t*>(D1);
+    F.q_bstride = bs1;
+    F.q_index = st.U;
+    F.n_cand = static_cast<int32_t>(N2);
+    if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s)) != RNN_OK) return r;
+    frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 1, 0);
+    if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+    // half-step 2: U = NN1(V)
+    F.q_base = static_cast<const uint16_t*>(D2);
+    F.q_bstride = bs2;
+    F.q_index = st.V;
+    F.n_cand = static_cast<int32_t>(N1);
+    if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s)) != RNN_OK) return r;
+    frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 0, it == max_iter ? 1 : 0);
+    if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  }
+  frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, pairs, cap, count_out, seed_state);
+  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+}
+
+}  // namespace rnn
+
+// ====================================================================== ABI
+using namespace rnn;
+
+extern "C" {
+
+const char* rnn_status_string(rnn_status s) {
+  switch (s) {
+    case RNN_OK: return "RNN_OK";
+    case RNN_EINVAL: return "RNN_EINVAL: invalid argument";
+    case RNN_EALIGN: return "RNN_EALIGN: d must be a multiple of 8 and pointers 16-byte aligned";
+    case RNN_ECAPACITY: return "RNN_ECAPACITY: output capacity below the guaranteed maximum";
+    case RNN_ECUDA: return "RNN_ECUDA: a CUDA call failed";
+    case RNN_ETIMEOUT: return "RNN_ETIMEOUT: a kernel's bounded wait ran out";
+    case RNN_EUNSUPPORTED: return "RNN_EUNSUPPORTED: unsupported size or device";
+    case RNN_EWORKSPACE: return "RNN_EWORKSPACE: workspace missing, too small or misaligned";
+  }
+  return "unknown rnn_status";
+}
+
+int rnn_abi_version(void) { return 1; }
+
+rnn_status rnn_workspace_status(const void* workspace, rnn_stream_t stream) {
+  if (!workspace) return RNN_EINVAL;
+  int err = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return RNN_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RNN_ECUDA;
+  return err ? RNN_ETIMEOUT : RNN_OK;
+}
+
+size_t rnn_nn_workspace_size(int64_t nq) {
+  Carve c(nullptr);
+  c.take<int>(64);
+  c.take<unsigned long long>(nq > 0 ? nq : 1);
+  return c.off;
+}
+
+rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, int d,
+                         rnn_dtype dtype, int32_t* idx_out, float* score_out, void* workspace,
+                         size_t ws_bytes, rnn_stream_t stream) {
+  if (nq < 0 || nx < 1 || nq > INT32_MAX || nx > INT32_MAX) return RNN_EINVAL;
+  if (!valid_dtype(dtype)) return RNN_EINVAL;
+  rnn_status r = check_desc(X, d);
+  if (r != RNN_OK) return r;
+  if (nq > 0) {  // with no queries, Q and idx_out may be null
+    if ((r = check_desc(Q, d)) != RNN_OK) return r;
+    if (!idx_out) return RNN_EINVAL;
+  }
+  if (!workspace || !aligned256(workspace) || ws_bytes < rnn_nn_workspace_size(nq))
+    return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  if ((r = device_info(&di)) != RNN_OK) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(workspace);
+  int* err = c.take<int>(64);
+  unsigned long long* keys = c.take<unsigned long long>(nq > 0 ? nq : 1);
+  zero_keys_kernel<<<grid_for(nq, di->sms), kSmallThreads, 0, s>>>(keys, nq, nullptr, 0, err);
+  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  if (nq == 0) return RNN_OK;
+  const Geometry g = geometry(d);
+  CUtensorMap mx, mq;
+  if ((r = make_map(&mx, X, d, nx, 1, nx * d, g)) != RNN_OK) return r;
+  if ((r = make_map(&mq, Q, d, nq, 1, nq * d, g, kBlockM)) != RNN_OK) return r;
+  NNParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.nfam = 1;
+  p.d = d;
+  p.idesc = make_idesc(dtype, g.block_n);
+  p.err = err;
+  NNFamily& F = p.fam[0];
+  F.q_base = static_cast<const uint16_t*>(Q);
+  F.q_count = static_cast<int32_t>(nq);
+  F.n_cand = static_cast<int32_t>(nx);
+  F.nbatch = 1;
+  F.keys = keys;
+  F.q_tma = 1;
+  if ((r = launch_nn(p, mx, mx, mq, mq, g, di, s)) != RNN_OK) return r;
+  unpack_kernel<<<grid_for(nq, di->sms), kSmallThreads, 0, s>>>(keys, nq, idx_out, score_out);
+  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+}
+
+size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2) {
+  const int64_t n1 = static_cast<int64_t>(H1 > 0 ? H1 : 0) * (W1 > 0 ? W1 : 0);
+  const int64_t n2 = static_cast<int64_t>(H2 > 0 ? H2 : 0) * (W2 > 0 ? W2 : 0);
+  Carve c(nullptr);
+  c.take<int>(64);
+  c.take<unsigned long long>(n1 > 0 ? n1 : 1);
+  c.take<unsigned long long>(n2 > 0 ? n2 : 1);
+  c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
+  return c.off;
+}
+
+rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, int H2, int W2,
+                              int d, rnn_dtype dtype, int32_t* pairs_out, int64_t cap,
+                              int32_t* count_out, int32_t* rowarg_out, float* rowmax_out,
+                              int32_t* colarg_out, float* colmax_out, void* workspace,
+                              size_t ws_bytes, rnn_stream_t stream) {
+  if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0) return RNN_EINVAL;
+  if (!valid_dtype(dtype)) return RNN_EINVAL;
+  rnn_status r = check_desc(D1, d);
+  if (r != RNN_OK) return r;
+  if ((r = check_desc(D2, d)) != RNN_OK) return r;
+  const int64_t n1 = static_cast<int64_t>(H1) * W1, n2 = static_cast<int64_t>(H2) * W2;
+  if (n1 > INT32_MAX || n2 > INT32_MAX) return RNN_EINVAL;
+  if (!pairs_out || !count_out) return RNN_EINVAL;
+  if (cap < (n1 < n2 ? n1 : n2)) return RNN_ECAPACITY;
+  if (!workspace || !aligned256(workspace) || ws_bytes < rnn_mnn_workspace_size(H1, W1, H2, W2))
+    return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  if ((r = device_info(&di)) != RNN_OK) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(workspace);
+  int* err = c.take<int>(64);
+  unsigned long long* rowk = c.take<unsigned long long>(n1);
+  unsigned long long* colk = c.take<unsigned long long>(n2);
+  const int nblk1 = static_cast<int>((n1 + kMnnChunk - 1) / kMnnChunk);
+  const int nblk2 = static_cast<int>((n2 + kMnnChunk - 1) / kMnnChunk);
+  int* counts = c.take<int>(nblk1 + 1);
+
+  const Geometry g = geometry(d);
+  CUtensorMap m1, m2, q1, q2;
+  if ((r = make_map(&m1, D1, d, n1, 1, n1 * d, g)) != RNN_OK) return r;
+  if ((r = make_map(&m2, D2, d, n2, 1, n2 * d, g)) != RNN_OK) return r;
+  if ((r = make_map(&q1, D1, d, n1, 1, n1 * d, g, kBlockM)) != RNN_OK) return r;
+  if ((r = make_map(&q2, D2, d, n2, 1, n2 * d, g, kBlockM)) != RNN_OK) return r;
+
+  zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(rowk, n1, colk, n2, err);
+  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  NNParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.nfam = 2;
+  p.d = d;
+  p.idesc = make_idesc(dtype, g.block_n);
+  p.err = err;
+  // sweep 1: rows of D1 against D2 -> NN2; sweep 2: rows of D2 against D1 -> NN1
+  p.fam[0].q_base = static_cast<const uint16_t*>(D1);
+  p.fam[0].q_count = static_cast<int32_t>(n1);
+  p.fam[0].n_cand = static_cast<int32_t>(n2);
+  p.fam[0].nbatch = 1;
+  p.fam[0].keys = rowk;
+  p.fam[1].q_base = static_cast<const uint16_t*>(D2);
+  p.fam[1].q_count = static_cast<int32_t>(n2);
+  p.fam[1].n_cand = static_cast<int32_t>(n1);
+  p.fam[1].nbatch = 1;
+  p.fam[1].keys = colk;
+  p.fam[0].q_tma = 1;
+  p.fam[1].q_tma = 1;
+  if ((r = launch_nn(p, m2, m1, q1, q2, g, di, s)) != RNN_OK) return r;
+  const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
+  mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, counts, nblk1, rowarg_out,
+                                                rowmax_out, colarg_out, colmax_out);
+  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  mnn_write_kernel<<<nblk1, kSmallThreads, 0, s>>>(rowk, n1, colk, counts, nblk1, pairs_out,
+                                                   count_out);
+  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+}
+
+int64_t rnn_frm_num_seeds(int H1, int W1, int seed_stride) {
+  if (H1 <= 0 || W1 <= 0 || seed_stride < 1) return 0;
+  return num_seeds(H1, W1, seed_stride);
+}
+
+int64_t rnn_frm_max_pairs(int H1, int W1, int H2, int W2, int seed_stride) {
+  const int64_t k = rnn_frm_num_seeds(H1, W1, seed_stride);
+  const int64_t n2 = static_cast<int64_t>(H2 > 0 ? H2 : 0) * (W2 > 0 ? W2 : 0);
+  return k < n2 ? k : n2;
+}
+
+size_t rnn_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int seed_stride) {
+  (void)H2;
+  (void)W2;
+  if (B < 1 || H1 <= 0 || W1 <= 0 || seed_stride < 1) return 0;
+  return frm_bytes(B, num_seeds(H1, W1, seed_stride), static_cast<int64_t>(H1) * W1);
+}
+
+rnn_status rnn_frm_match(const void* D1, int H1, int W1, const void* D2, int H2, int W2, int d,
+                         rnn_dtype dtype, int seed_stride, int max_iter, int32_t* pairs_out,
+                         int64_t cap, int32_t* count_out, int32_t* seed_state_out,
+                         void* workspace, size_t ws_bytes, rnn_stream_t stream) {
+  const int64_t n1 = static_cast<int64_t>(H1) * W1, n2 = static_cast<int64_t>(H2) * W2;
+  return frm_run(1, D1, n1 * d, D2, n2 * d, H1, W1, H2, W2, d, dtype, seed_stride, max_iter,
+                 pairs_out, cap, count_out, seed_state_out, workspace, ws_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+rnn_status rnn_frm_match_batched(int B, const void* D1, int64_t d1_batch_stride, const void* D2,
+                                 int64_t d2_batch_stride, int H1, int W1, int H2, int W2, int d,
+                                 rnn_dtype dtype, int seed_stride, int max_iter,
+                                 int32_t* pairs_out, int64_t cap, int32_t* count_out,
+                                 int32_t* seed_state_out, void* workspace, size_t ws_bytes,
+                                 rnn_stream_t stream) {
+  return frm_run(B, D1, d1_batch_stride, D2, d2_batch_stride, H1, W1, H2, W2, d, dtype,
+                 seed_stride, max_iter, pairs_out, cap, count_out, seed_state_out, workspace,
+                 ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -142,15 +142,25 @@ def smooth_pair(seed: int, H: int, W: int, d: int, *, sigma: float = 2.0,
 def to_storage(a: np.ndarray, dtype: str):
     """Round a float64 map to the storage type; returns a CPU torch tensor.
 
-    ``dtype`` is ``"f16"`` or ``"bf16"``; rounding is to nearest even.
+    ``dtype`` is ``"f16"`` (numpy's float64 -> float16 conversion, one
+    round-to-nearest-even step) or ``"bf16"`` (torch's conversion, which goes
+    through float32; each step rounds to nearest even).
     """
     import torch
 
-    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    return torch.from_numpy(_storage_bits(a, dtype)).view(
+        torch.float16 if dtype == "f16" else torch.bfloat16)
+
+
+def _storage_bits(a: np.ndarray, dtype: str) -> np.ndarray:
+    """16-bit patterns of ``a`` rounded to ``dtype`` (int16 array)."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
     if dtype == "f16":
-        return t.to(torch.float16)
+        return a.astype(np.float16).view(np.int16)
     if dtype == "bf16":
-        return t.to(torch.bfloat16)
+        import torch
+
+        return torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy()
     raise ValueError(f"unknown storage dtype {dtype!r}")
 
 
@@ -200,3 +210,37 @@ def make_workload(w: Workload, pair: int = 0):
     if w.kind == "quantised":
         return quantised_pair(seed, w.H, w.W, w.H, w.W, w.d)
     return smooth_pair(seed, w.H, w.W, w.d, occlusion=w.occlusion, outliers=w.outliers)
+
+
+def _pair_storage(args):
+    w, pair, dtype = args
+    d1, d2 = make_workload(w, pair)
+    # ship raw 16-bit patterns (bf16 has no numpy type)
+    return _storage_bits(d1, dtype), _storage_bits(d2, dtype)
+
+
+def make_workload_storage(w: Workload, dtype: str = "f16", pairs=None, workers: int = 0):
+    """Pairs of workload ``w`` rounded to ``dtype``, as CPU tensors ``[P, H, W, d]``.
+
+    ``pairs`` is an iterable of pair indices (default: all ``w.pairs``).  With
+    ``workers > 1`` the pairs are drawn in a process pool started with the
+    ``spawn`` method, so it is safe after CUDA has been initialised; the result
+    does not depend on the worker count.
+    """
+    import torch
+
+    idx = list(range(w.pairs)) if pairs is None else list(pairs)
+    jobs = [(w, p, dtype) for p in idx]
+    if workers and workers > 1 and len(jobs) > 1:
+        import multiprocessing as mp
+        from concurrent.futures import ProcessPoolExecutor
+
+        with ProcessPoolExecutor(max_workers=min(workers, len(jobs)),
+                                 mp_context=mp.get_context("spawn")) as ex:
+            parts = list(ex.map(_pair_storage, jobs))
+    else:
+        parts = [_pair_storage(j) for j in jobs]
+    tdt = torch.float16 if dtype == "f16" else torch.bfloat16
+    A = torch.from_numpy(np.stack([p[0] for p in parts])).view(tdt)
+    B = torch.from_numpy(np.stack([p[1] for p in parts])).view(tdt)
+    return A, B

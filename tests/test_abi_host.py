@@ -1,0 +1,133 @@
+"""Host-side checks of the C ABI (no GPU needed, nothing is launched).
+
+The library must load without a GPU, export every function ``include/rnn.h``
+declares, compute workspace sizes and seed counts on the host, and reject bad
+arguments before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from reciprocal_nearest_neighbour_b200 import _lib, build as rnn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rnn_build.build()
+    return _lib.load()
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(rnn_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert declared, "no declarations found"
+    assert declared == set(_lib.EXPORTS)
+    so = ctypes.CDLL(_lib.LIB_PATH)
+    for name in declared:
+        assert hasattr(so, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert lib.rnn_abi_version() == 1
+    for code, name in _lib.STATUS.items():
+        assert lib.rnn_status_string(code).decode().startswith(name)
+
+
+@pytest.mark.parametrize("H,W,S", [(5, 7, 2), (4, 4, 3), (1, 4, 2), (3, 3, 1), (384, 512, 8),
+                                   (288, 512, 8), (768, 1024, 8), (32, 32, 4), (17, 9, 5)])
+def test_seed_counts_match_oracle(lib, H, W, S):
+    assert lib.rnn_frm_num_seeds(H, W, S) == len(oracle.frm_seeds(H, W, S))
+    k = len(oracle.frm_seeds(H, W, S))
+    assert lib.rnn_frm_max_pairs(H, W, H, W, S) == min(k, H * W)
+
+
+def test_workspace_sizes(lib):
+    assert lib.rnn_nn_workspace_size(1000) >= 1000 * 8
+    assert lib.rnn_mnn_workspace_size(384, 512, 384, 512) >= 2 * 384 * 512 * 8
+    one = lib.rnn_frm_workspace_size(1, 384, 512, 384, 512, 8)
+    many = lib.rnn_frm_workspace_size(64, 288, 512, 288, 512, 8)
+    assert one > 0 and many > 64 * 2304 * 8
+    assert lib.rnn_frm_workspace_size(0, 384, 512, 384, 512, 8) == 0
+    for v in (one, many):
+        assert v % 256 == 0
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+EINVAL, EALIGN, ECAP, EUNSUP, EWS = 1, 2, 3, 6, 7
+
+
+def test_nn_argmax_argument_errors(lib):
+    ws = lib.rnn_nn_workspace_size(10)
+    f = lib.rnn_nn_argmax
+    assert f(None, 10, FAKE, 10, 24, 0, FAKE, None, FAKE, ws, None) == EINVAL
+    assert f(FAKE, 10, FAKE, 0, 24, 0, FAKE, None, FAKE, ws, None) == EINVAL
+    assert f(FAKE, -1, FAKE, 10, 24, 0, FAKE, None, FAKE, ws, None) == EINVAL
+    assert f(FAKE, 10, FAKE, 10, 20, 0, FAKE, None, FAKE, ws, None) == EALIGN
+    assert f(FAKE + 8, 10, FAKE, 10, 24, 0, FAKE, None, FAKE, ws, None) == EALIGN
+    assert f(FAKE, 10, FAKE, 10, 264, 0, FAKE, None, FAKE, ws, None) == EUNSUP
+    assert f(FAKE, 10, FAKE, 10, 24, 7, FAKE, None, FAKE, ws, None) == EINVAL
+    assert f(FAKE, 10, FAKE, 10, 24, 0, None, None, FAKE, ws, None) == EINVAL
+    assert f(FAKE, 10, FAKE, 10, 24, 0, FAKE, None, None, ws, None) == EWS
+    assert f(FAKE, 10, FAKE, 10, 24, 0, FAKE, None, FAKE, ws - 8, None) == EWS
+    assert f(FAKE, 10, FAKE, 10, 24, 0, FAKE, None, FAKE + 16, ws, None) == EWS
+
+
+def test_mnn_argument_errors(lib):
+    ws = lib.rnn_mnn_workspace_size(4, 4, 4, 4)
+    f = lib.rnn_mnn_exhaustive
+
+    def call(**kw):
+        a = dict(D1=FAKE, H1=4, W1=4, D2=FAKE, H2=4, W2=4, d=16, dt=0, pairs=FAKE, cap=16,
+                 count=FAKE, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return f(a["D1"], a["H1"], a["W1"], a["D2"], a["H2"], a["W2"], a["d"], a["dt"],
+                 a["pairs"], a["cap"], a["count"], None, None, None, None, a["ws"], a["wsb"], None)
+
+    assert call(H1=0) == EINVAL
+    assert call(D2=None) == EINVAL
+    assert call(pairs=None) == EINVAL
+    assert call(count=None) == EINVAL
+    assert call(d=12) == EALIGN
+    assert call(cap=15) == ECAP
+    assert call(wsb=ws - 1) == EWS
+
+
+def test_frm_argument_errors(lib):
+    ws = lib.rnn_frm_workspace_size(2, 8, 8, 8, 8, 2)
+    f = lib.rnn_frm_match_batched
+
+    def call(**kw):
+        a = dict(B=2, D1=FAKE, s1=8 * 8 * 16, D2=FAKE, s2=8 * 8 * 16, H1=8, W1=8, H2=8, W2=8,
+                 d=16, dt=0, S=2, it=10, pairs=FAKE, cap=16, count=FAKE, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return f(a["B"], a["D1"], a["s1"], a["D2"], a["s2"], a["H1"], a["W1"], a["H2"], a["W2"],
+                 a["d"], a["dt"], a["S"], a["it"], a["pairs"], a["cap"], a["count"], None,
+                 a["ws"], a["wsb"], None)
+
+    assert call(B=0) == EINVAL
+    assert call(B=_lib.RNN_MAX_BATCH + 1) == EUNSUP
+    assert call(S=0) == EINVAL
+    assert call(it=0) == EINVAL
+    assert call(s1=8 * 8 * 16 - 8) == EINVAL
+    assert call(s2=8 * 8 * 16 + 4) == EINVAL
+    assert call(cap=15) == ECAP
+    assert call(ws=None) == EWS
+    assert call(d=4) == EALIGN
+    single = lib.rnn_frm_match
+    assert single(FAKE, 8, 8, FAKE, 8, 8, 16, 0, 2, 0, FAKE, 16, FAKE, None, FAKE, ws,
+                  None) == EINVAL
