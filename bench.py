@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark: FRM image pairs/s at 512x384, d=24 (plus exhaustive MNN pair-scores/s).
+
+One step = Fast Reciprocal Matching of a batch of distinct synthetic image
+pairs (512x384, d=24, unit-norm fp16 descriptors, seed stride 8 -> 3072
+seeds, max_iter 10) through the batched C-ABI entry point: seed init, 10 x
+(NN2 half-step + update, NN1 half-step + update), merge.  The batch's inputs
+(8 pairs = 151 MB) exceed the 126 MB L2, so no flush is needed between steps.
+
+Printed: one JSON line (rank 0).  ``value`` = pairs/s over all ranks (each
+rank matches its own pairs: weak scaling, no data-path collective), timed on
+the device with CUDA events between barriers, max over ranks.  Extra keys:
+``e2e`` (host buffers, copies inside the timed region), ``roofline`` (the
+fused similarity+argmax kernel, timed live with CUDA events), ``mnn`` (the
+exhaustive reciprocal set at 512x384 with its own roofline), ``cpu_baseline``
+(the double-precision oracle on a bounded sample), ``clocks``,
+``gpu_launches``.
+
+``--impl reference`` times the oracle itself (host cores) on the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("FRM image pairs/s at 512×384, d=24; exhaustive MNN pair-scores/s; "
+          "% roofline")
+WORKLOAD = "frm_512x384"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "sm_max_mhz": p.get("sm_max_mhz", 1965.0), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """SM clock and throttle reasons of one GPU, polled every 5 ms while running.
+
+    Reads NVML (the data nvidia-smi prints); the GPU is matched by UUID so a
+    remapped CUDA_VISIBLE_DEVICES does not matter.  Reading changes nothing.
+    """
+
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, device):
+        self.device = device
+        self.samples = []
+        self._stop = None
+        self._thread = None
+        self._nvml = None
+        self._handle = None
+        self.max_mhz = None
+
+    def __enter__(self):
+        import threading
+
+        import torch
+
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self._handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+            self._nvml = pynvml
+        except Exception:  # no NVML: clocks are reported as null
+            self._nvml = None
+            return self
+        self._stop = threading.Event()
+
+        def poll():
+            nv = self._nvml
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            while not self._stop.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM)
+                    mask = get_reasons(self._handle) if get_reasons else 0
+                    self.samples.append((mhz, mask))
+                except Exception:
+                    pass
+                self._stop.wait(0.005)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+        if self._nvml is not None:
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return None
+        mx = self.max_mhz or max(m for m, _ in self.samples)
+        loaded = [s for s in self.samples if s[0] > 0.5 * mx] or self.samples
+        reasons = sorted(name for name, attr in self.REASONS.items()
+                         if any(mask & getattr(self._nvml, attr, 0) for _, mask in loaded))
+        return {"sm_mhz": statistics.median(m for m, _ in loaded), "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _oracle_frm_pairs_per_s(maps, budget_s: float, max_pairs: int):
+    """Time the oracle's FRM on whole pairs until `budget_s` is spent."""
+    import oracle
+
+    t0 = time.perf_counter()
+    n = 0
+    for D1, D2 in maps[:max_pairs]:
+        oracle.frm(D1, D2, 8, 10)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return n, dt, oracle.max_threads()
+
+
+def run_reference(args):
+    """The oracle as the reference arm: same metric, host cores, bounded steps."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    from reciprocal_nearest_neighbour_b200 import synth
+    import oracle
+
+    w = synth.WORKLOADS[WORKLOAD]
+    npairs = max(1, min(args.pairs, args.warmup + args.steps))
+    A, B = synth.make_workload_storage(w, "f16", pairs=range(npairs),
+                                       workers=min(npairs, os.cpu_count() or 1))
+    for s in range(args.warmup):
+        oracle.frm(A[s % npairs], B[s % npairs], w.seed_stride, w.max_iter)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        oracle.frm(A[s % npairs], B[s % npairs], w.seed_stride, w.max_iter)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "pairs/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "pairs_per_step": 1, "H": w.H, "W": w.W, "d": w.d,
+                   "seed_stride": w.seed_stride, "max_iter": w.max_iter,
+                   "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": "pairs/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"one 512x384 pair per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": "pairs/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _event_ms(evs_a, evs_b, n):
+    return [evs_a[i].elapsed_time(evs_b[i]) for i in range(n)]
+
+
+def run_native(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import reciprocal_nearest_neighbour_b200 as rnn
+    from reciprocal_nearest_neighbour_b200 import _lib, synth
+
+    world, rank, local = _dist()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    lib = _lib.load()
+    peaks = _peaks()
+    w = synth.WORKLOADS[WORKLOAD]
+    P = args.pairs
+    pair_ids = range(rank * P, rank * P + P)      # each rank matches its own pairs
+    A_h, B_h = synth.make_workload_storage(w, "f16", pairs=pair_ids,
+                                           workers=min(P, max(1, (os.cpu_count() or 2) // world)))
+    A_h, B_h = A_h.pin_memory(), B_h.pin_memory()
+    A = A_h.to(dev)
+    B = B_h.to(dev)
+    plan = rnn.FRMPlan(P, w.H, w.W, w.H, w.W, w.d, torch.float16, w.seed_stride, w.max_iter,
+                       dev, with_seed_state=True)
+    n_per_call_nn = 2 * w.max_iter
+
+    for _ in range(args.warmup):
+        plan.run(A, B)
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------------------- timed region
+    cap = n_per_call_nn * min(args.steps, 20)
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    for e in ev_a + ev_b:
+        e.record()
+    torch.cuda.synchronize()
+    import ctypes
+
+    h_a = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_a])
+    h_b = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_b])
+    rec = ctypes.c_int(0)
+    t0e = torch.cuda.Event(enable_timing=True)
+    t1e = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        launches0 = lib.rnn_launch_count()
+        lib.rnn_set_kernel_timer(h_a, h_b, cap, ctypes.byref(rec))
+        t0e.record()
+        for _ in range(args.steps):
+            plan.run(A, B)
+        t1e.record()
+        torch.cuda.synchronize()
+        lib.rnn_set_kernel_timer(None, None, 0, None)
+        launches = lib.rnn_launch_count() - launches0
+        barrier()
+    clocks = clk.summary()
+    step_ms = t0e.elapsed_time(t1e) / args.steps
+    step_ms = max_over_ranks(step_ms)
+    value = world * P / (step_ms * 1e-3)
+    rnn.workspace_status(plan.workspace)
+
+    # roofline of the fused similarity+argmax kernel over the recorded launches
+    nrec = min(rec.value, cap)
+    nn_ms = _event_ms(ev_a, ev_b, nrec)
+    seed_state = plan.result.seed_state.cpu().numpy()
+    queries_per_call = int(seed_state[:, :, 2].sum())          # sum of active seeds per half-step
+    calls_recorded = nrec / n_per_call_nn
+    n_cand = w.H * w.W
+    flops = 2.0 * w.d * n_cand * queries_per_call * calls_recorded
+    nn_time_s = sum(nn_ms) * 1e-3
+    achieved_tf = flops / nn_time_s / 1e12
+    peak_tf = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved_tf / peak_tf, "traffic": None,
+                "kernel": "nn_argmax_kernel (FRM half-steps)",
+                "launches": nrec, "avg_launch_us": 1e3 * sum(nn_ms) / max(nrec, 1),
+                "flops_per_launch": flops / max(nrec, 1),
+                "peak_source": f"bf16 sustained, {peaks['source']} (fp16 runs at the bf16 rate)",
+                "active_queries_per_pair": queries_per_call / P}
+
+    # ------------------------------------------------------ end to end (host)
+    pairs_h = torch.empty_like(plan.result.pairs, device="cpu").pin_memory()
+    count_h = torch.empty_like(plan.result.count, device="cpu").pin_memory()
+
+    def e2e_step():
+        A.copy_(A_h, non_blocking=True)
+        B.copy_(B_h, non_blocking=True)
+        r = plan.run(A, B)
+        pairs_h.copy_(r.pairs, non_blocking=True)
+        count_h.copy_(r.count, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    barrier()
+    e2e = {"value": world * P / (e2e_ms * 1e-3), "unit": "pairs/s",
+           "h2d_bytes_per_step": int(A_h.numel() * 2 + B_h.numel() * 2),
+           "d2h_bytes_per_step": int(pairs_h.numel() * 4 + count_h.numel() * 4),
+           "ms_per_step": e2e_ms}
+
+    # --------------------------------------- exhaustive reciprocal set (rank 0 shape)
+    mnn = None
+    if not args.skip_mnn:
+        mnn = {}
+        props = torch.cuda.get_device_properties(dev)
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        for mode, wl in (("quantised", "mnn_512x384_q"), ("fp16", "mnn_512x384_f")):
+            ww = synth.WORKLOADS[wl]
+            a, b = synth.make_workload_storage(ww, "f16", pairs=[0])
+            a, b = a[0].to(dev), b[0].to(dev)
+            out = rnn.mnn_exhaustive(a, b)
+            ws = torch.empty(lib.rnn_mnn_workspace_size(ww.H, ww.W, ww.H, ww.W),
+                             dtype=torch.uint8, device=dev)
+            reps = args.mnn_reps
+            ka = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            kb = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            ca = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            cb = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            for e in ka + kb:
+                e.record()
+            torch.cuda.synchronize()
+            ha = (ctypes.c_void_p * reps)(*[e.cuda_event for e in ka])
+            hb = (ctypes.c_void_p * reps)(*[e.cuda_event for e in kb])
+            r2 = ctypes.c_int(0)
+            for _ in range(2):
+                rnn.mnn_exhaustive(a, b, workspace=ws, out=out)
+            lib.rnn_set_kernel_timer(ha, hb, reps, ctypes.byref(r2))
+            for i in range(reps):
+                flush.fill_(i & 0xFF)                   # evict the maps from L2
+                ca[i].record()
+                rnn.mnn_exhaustive(a, b, workspace=ws, out=out)
+                cb[i].record()
+            torch.cuda.synchronize()
+            lib.rnn_set_kernel_timer(None, None, 0, None)
+            call_ms = statistics.median(_event_ms(ca, cb, reps))
+            kern_ms = statistics.median(_event_ms(ka, kb, min(r2.value, reps)))
+            n1 = ww.H * ww.W
+            scores = float(n1) * n1
+            compares = 2.0 * scores                      # both directions
+            peak_cmp = props.multi_processor_count * 128 * peaks["sm_max_mhz"] * 1e6
+            achieved_cmp = compares / (kern_ms * 1e-3)
+            mnn[mode] = {
+                "metric": "exhaustive MNN pair-scores/s at 512x384, d=24",
+                "value": scores / (call_ms * 1e-3), "unit": "pair-scores/s",
+                "ms_per_call": call_ms, "pairs": int(out.count.item()),
+                "roofline": {"bound": "alu", "achieved": achieved_cmp / 1e12,
+                             "peak": peak_cmp / 1e12, "unit": "Tcompare/s",
+                             "frac": achieved_cmp / peak_cmp, "traffic": None,
+                             "kernel_ms": kern_ms,
+                             "peak_basis": "1 compare per score per direction at "
+                                           f"{props.multi_processor_count} SMs x 128 lanes x "
+                                           f"{peaks['sm_max_mhz']:.0f} MHz"},
+                "l2": "256 MB flush before every call"}
+        del flush
+
+    # ----------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        maps = [(A_h[i], B_h[i]) for i in range(min(P, 4))]
+        n, dt, cores = _oracle_frm_pairs_per_s(maps, args.cpu_budget_s, 4)
+        cpu = {"value": n / dt, "unit": "pairs/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} of this step's 512x384 pairs, whole FRM loop, double precision"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "pairs_per_step": P, "H": w.H, "W": w.W,
+                       "d": w.d, "seed_stride": w.seed_stride, "max_iter": w.max_iter,
+                       "global_batch": world * P, "parallelism": f"replicas x{world}",
+                       "l2": f"step inputs {2 * A_h.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
+            "e2e": e2e, "roofline": roofline, "mnn": mnn, "cpu_baseline": cpu,
+            "clocks": clocks, "gpu_launches": int(launches),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--pairs", type=int, default=8, help="image pairs per step and rank")
+    ap.add_argument("--mnn-reps", type=int, default=10)
+    ap.add_argument("--skip-mnn", action="store_true")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

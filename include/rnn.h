@@ -159,6 +159,24 @@ rnn_status rnn_frm_match_batched(int B, const void *D1, int64_t d1_batch_stride,
                                  int32_t *seed_state_out, void *workspace, size_t ws_bytes,
                                  rnn_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Diagnostics for benchmarking (no effect on results).
+ *
+ * rnn_launch_count: number of kernels this library has launched in this
+ *   process (all entry points, all devices).
+ * rnn_set_kernel_timer: while set, every launch of the fused
+ *   similarity+argmax kernel is bracketed by cudaEventRecord(start_events[i])
+ *   and cudaEventRecord(stop_events[i]) on the launch stream, with
+ *   i = (*recorded)++ for i < capacity (launches past capacity are still
+ *   counted).  The events (cudaEvent_t, created by the caller with timing
+ *   enabled) and the host counter stay owned by the caller; pass NULL
+ *   pointers or capacity 0 to switch the timer off.  The setting is global to
+ *   the process and not thread-safe against concurrent calls.
+ */
+uint64_t rnn_launch_count(void);
+void rnn_set_kernel_timer(void *const *start_events, void *const *stop_events, int capacity,
+                          int *recorded);
+
 #ifdef __cplusplus
 }
 #endif

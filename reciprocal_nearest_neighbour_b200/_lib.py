@@ -25,6 +25,8 @@ EXPORTS = (
     "rnn_frm_workspace_size",
     "rnn_frm_match",
     "rnn_frm_match_batched",
+    "rnn_launch_count",
+    "rnn_set_kernel_timer",
 )
 
 STATUS = {
@@ -77,6 +79,8 @@ def load():
         "rnn_frm_match": (I, [P, I, I, P, I, I, I, I, I, I, P, I64, P, P, P, SZ, P]),
         "rnn_frm_match_batched": (I, [I, P, I64, P, I64, I, I, I, I, I, I, I, I, P, I64, P, P, P,
                                       SZ, P]),
+        "rnn_launch_count": (ctypes.c_uint64, []),
+        "rnn_set_kernel_timer": (None, [P, P, I, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

@@ -157,6 +157,20 @@ static rnn_status make_map(CUtensorMap* m, const void* base, int d, int64_t rows
   return r == CUDA_SUCCESS ? RNN_OK : RNN_ECUDA;
 }
 
+// ------------------------------------------------------------- diagnostics
+static std::atomic<uint64_t> g_launches{0};
+static void* const* g_timer_start = nullptr;
+static void* const* g_timer_stop = nullptr;
+static int g_timer_cap = 0;
+static int* g_timer_count = nullptr;
+
+// Check the last launch and count it.
+static rnn_status launched() {
+  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return RNN_OK;
+}
+
 static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const CUtensorMap& m1,
                             const CUtensorMap& q0, const CUtensorMap& q1, const Geometry& g,
                             DeviceInfo* di, cudaStream_t s) {
@@ -186,11 +200,25 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
       di->smem_set = true;
     }
   }
+  int slot = -1;
+  if (g_timer_count && g_timer_start && g_timer_stop) {
+    slot = (*g_timer_count)++;
+    if (slot < g_timer_cap) {
+      if (cudaEventRecord(static_cast<cudaEvent_t>(g_timer_start[slot]), s) != cudaSuccess)
+        return RNN_ECUDA;
+    } else {
+      slot = -1;
+    }
+  }
   if (g.slot_locate)
     nn_argmax_kernel<true><<<di->sms, kThreads, g.smem, s>>>(p, m0, m1, q0, q1);
   else
     nn_argmax_kernel<false><<<di->sms, kThreads, g.smem, s>>>(p, m0, m1, q0, q1);
-  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+  const rnn_status r = launched();
+  if (r == RNN_OK && slot >= 0 &&
+      cudaEventRecord(static_cast<cudaEvent_t>(g_timer_stop[slot]), s) != cudaSuccess)
+    return RNN_ECUDA;
+  return r;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -547,7 +575,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   if ((r = make_map(&map2, D2, d, N2, B, bs2, g)) != RNN_OK) return r;
 
   frm_init_kernel<<<grid_for(B * k + B * st.nwords, di->sms), kSmallThreads, 0, s>>>(st, W1, S);
-  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  if ((r = launched()) != RNN_OK) return r;
 
   NNParams p;
   std::memset(&p, 0, sizeof(p));
@@ -570,7 +598,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.n_cand = static_cast<int32_t>(N2);
     if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s)) != RNN_OK) return r;
     frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 1, 0);
-    if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+    if ((r = launched()) != RNN_OK) return r;
     // half-step 2: U = NN1(V)
     F.q_base = static_cast<const uint16_t*>(D2);
     F.q_bstride = bs2;
@@ -578,10 +606,10 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.n_cand = static_cast<int32_t>(N1);
     if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s)) != RNN_OK) return r;
     frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 0, it == max_iter ? 1 : 0);
-    if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+    if ((r = launched()) != RNN_OK) return r;
   }
   frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, pairs, cap, count_out, seed_state);
-  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+  return launched();
 }
 
 }  // namespace rnn
@@ -606,6 +634,18 @@ const char* rnn_status_string(rnn_status s) {
 }
 
 int rnn_abi_version(void) { return 1; }
+
+uint64_t rnn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void rnn_set_kernel_timer(void* const* start_events, void* const* stop_events, int capacity,
+                          int* recorded) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const bool on = start_events && stop_events && recorded && capacity > 0;
+  g_timer_start = on ? start_events : nullptr;
+  g_timer_stop = on ? stop_events : nullptr;
+  g_timer_cap = on ? capacity : 0;
+  g_timer_count = on ? recorded : nullptr;
+}
 
 rnn_status rnn_workspace_status(const void* workspace, rnn_stream_t stream) {
   if (!workspace) return RNN_EINVAL;
@@ -644,7 +684,7 @@ rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, i
   int* err = c.take<int>(64);
   unsigned long long* keys = c.take<unsigned long long>(nq > 0 ? nq : 1);
   zero_keys_kernel<<<grid_for(nq, di->sms), kSmallThreads, 0, s>>>(keys, nq, nullptr, 0, err);
-  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  if ((r = launched()) != RNN_OK) return r;
   if (nq == 0) return RNN_OK;
   const Geometry g = geometry(d);
   CUtensorMap mx, mq;
@@ -665,7 +705,7 @@ rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, i
   F.q_tma = 1;
   if ((r = launch_nn(p, mx, mx, mq, mq, g, di, s)) != RNN_OK) return r;
   unpack_kernel<<<grid_for(nq, di->sms), kSmallThreads, 0, s>>>(keys, nq, idx_out, score_out);
-  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+  return launched();
 }
 
 size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2) {
@@ -714,7 +754,7 @@ rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, in
   if ((r = make_map(&q2, D2, d, n2, 1, n2 * d, g, kBlockM)) != RNN_OK) return r;
 
   zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(rowk, n1, colk, n2, err);
-  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  if ((r = launched()) != RNN_OK) return r;
   NNParams p;
   std::memset(&p, 0, sizeof(p));
   p.nfam = 2;
@@ -738,10 +778,10 @@ rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, in
   const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
   mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, counts, nblk1, rowarg_out,
                                                 rowmax_out, colarg_out, colmax_out);
-  if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
+  if ((r = launched()) != RNN_OK) return r;
   mnn_write_kernel<<<nblk1, kSmallThreads, 0, s>>>(rowk, n1, colk, counts, nblk1, pairs_out,
                                                    count_out);
-  return cudaGetLastError() == cudaSuccess ? RNN_OK : RNN_ECUDA;
+  return launched();
 }
 
 int64_t rnn_frm_num_seeds(int H1, int W1, int seed_stride) {
