@@ -160,6 +160,34 @@ rnn_status rnn_frm_match_batched(int B, const void *D1, int64_t d1_batch_stride,
                                  rnn_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Nearest neighbours without any allocation.  (The matching method itself
+ * has no counterpart of this: it exists for callers, not for the algorithm.)
+ *
+ * Same computation, arguments, results and errors as rnn_nn_argmax, minus the
+ * workspace: its scratch lives in a fixed array inside the library, which
+ * every GPU that loads the library keeps for the life of the process
+ * (256 + 8 * RNN_NN_NOALLOC_MAX_QUERIES bytes, about 512 KB).  It is meant for
+ * callers that cannot allocate device memory themselves: a plugin whose host
+ * framework owns all device buffers, or a latency-bound loop in which
+ * cudaMalloc/cudaFree would synchronise the device.  The function itself calls
+ * no allocator.
+ *
+ *   nq > RNN_NN_NOALLOC_MAX_QUERIES  -> RNN_EUNSUPPORTED (nothing launched).
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.
+ *   All calls share the one array, which keeps the last call's contents (each
+ *   call clears what must start at zero): calls that overlap on the GPU, on
+ *   any streams, race and give undefined results.  Serialise them.
+ *   rnn_workspace_status() does not apply; a timed-out wait shows as an
+ *   undefined result only.
+ */
+#define RNN_NN_NOALLOC_MAX_QUERIES 65536
+rnn_status rnn_nn_argmax_noalloc(const void *Q, int64_t nq, const void *X, int64_t nx, int d,
+                                 rnn_dtype dtype, int32_t *idx_out, float *score_out,
+                                 rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Diagnostics for benchmarking (no effect on results).
  *
  * rnn_launch_count: number of kernels this library has launched in this

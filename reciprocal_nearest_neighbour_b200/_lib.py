@@ -27,6 +27,7 @@ EXPORTS = (
     "rnn_frm_match_batched",
     "rnn_launch_count",
     "rnn_set_kernel_timer",
+    "rnn_nn_argmax_noalloc",
 )
 
 STATUS = {
@@ -35,6 +36,7 @@ STATUS = {
 }
 RNN_F16, RNN_BF16 = 0, 1
 RNN_MAX_BATCH = 1024
+RNN_NN_NOALLOC_MAX_QUERIES = 65536
 
 
 class RNNLibraryError(RuntimeError):
@@ -81,6 +83,7 @@ def load():
                                       SZ, P]),
         "rnn_launch_count": (ctypes.c_uint64, []),
         "rnn_set_kernel_timer": (None, [P, P, I, P]),
+        "rnn_nn_argmax_noalloc": (I, [P, I64, P, I64, I, I, P, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

@@ -824,3 +824,53 @@ rnn_status rnn_frm_match_batched(int B, const void* D1, int64_t d1_batch_stride,
 }
 
 }  // extern "C"
+
+// ============================================== nearest neighbours, no allocation
+//
+// Some callers cannot allocate device memory: a plugin whose host framework
+// owns every device buffer and only lends it the inputs and outputs, or a
+// latency-bound serving loop in which cudaMalloc/cudaFree would synchronise
+// the device and stall other work.  For them rnn_nn_argmax_noalloc keeps its
+// scratch (the packed per-query keys and the status word) in the fixed array
+// below instead of a caller workspace.  The array is part of the library's
+// device image, so every GPU that loads the library holds it until the
+// process exits.
+namespace rnn {
+
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[256 + RNN_NN_NOALLOC_MAX_QUERIES * sizeof(unsigned long long)];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[64];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code only knows the array by a host-side stand-in name).
+static rnn_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RNN_ECUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return RNN_ECUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return RNN_OK;
+}
+
+}  // namespace rnn
+
+extern "C" rnn_status rnn_nn_argmax_noalloc(const void* Q, int64_t nq, const void* X, int64_t nx,
+                                            int d, rnn_dtype dtype, int32_t* idx_out,
+                                            float* score_out, rnn_stream_t stream) {
+  if (nq > RNN_NN_NOALLOC_MAX_QUERIES) return RNN_EUNSUPPORTED;
+  if (nq < 0) return RNN_EINVAL;
+  void* scratch = nullptr;
+  const rnn_status r = rnn::noalloc_scratch(&scratch);
+  if (r != RNN_OK) return r;
+  static_assert(sizeof(rnn::g_noalloc_scratch) >= 256 + RNN_NN_NOALLOC_MAX_QUERIES * 8,
+                "scratch array too small");
+  return rnn_nn_argmax(Q, nq, X, nx, d, dtype, idx_out, score_out, scratch,
+                       sizeof(rnn::g_noalloc_scratch), stream);
+}
