@@ -408,6 +408,20 @@ def run_native(args):
     return 0
 
 
+def run_nn_case(nq, d, nx):
+    """One small nearest-neighbour case for an ncu capture of the fused kernel."""
+    import torch
+    import reciprocal_nearest_neighbour_b200 as rnn
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    Q = torch.randn(nq, d, device="cuda", generator=gen).half()
+    X = torch.randn(nx, d, device="cuda", generator=gen).half()
+    for _ in range(3):
+        idx, sc = rnn.nn_argmax(Q, X)
+    torch.cuda.synchronize()
+    print(f"nn-case {nq}x{nx} d={d}: idx[0]={int(idx[0])} score[0]={float(sc[0]):.6f}")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -419,7 +433,12 @@ def main(argv=None):
     ap.add_argument("--skip-mnn", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--nn-case", type=int, nargs=3, metavar=("NQ", "D", "NX"),
+                    help="profiling aid: run nn_argmax three times on seeded fp16 "
+                         "queries/candidates of these sizes and exit (no timing)")
     args = ap.parse_args(argv)
+    if args.nn_case:
+        return run_nn_case(*args.nn_case)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":

@@ -3,7 +3,7 @@
 // For a tile of 128 query descriptors and a stream of candidate tiles, the
 // scores S = Q * X^T are accumulated in fp32 in tensor memory (tcgen05.mma,
 // kind::f16) and reduced on the fly to the largest score of each query row
-// and the lowest candidate index that reaches it.  No score ever leaves the
+// and the first 32-column chunk that reaches it.  No score ever leaves the
 // SM.  This is the NN1/NN2 operator of the reciprocal set and of Fast
 // Reciprocal Matching (cv-learn.com "MASt3R" note, paragraph "Fast reciprocal
 // matching (FRM)"), on the dot-product reading of "nearest".
@@ -20,18 +20,29 @@
 // the merge gives the largest score and then the lowest index whatever the
 // order of arrival.
 //
-// Warp roles (12 warps):
+// Warp roles (4 + kEpiWarps warps):
 //   warp 0      TMA producer: candidate tiles into a ring of shared-memory stages
-//   warp 1      tensor-memory owner and MMA issuer
-//   warp 2      query tiles: a TMA box when the rows are contiguous, else
+//   warps 1-2   MMA issuers, alternating tiles (warp 1 owns tensor memory).
+//               Every wait, fence and commit in an issuing thread costs it
+//               hundreds of cycles of latency, which one warp would pay
+//               serially on every tile; two warps overlap them.
+//   warp 3      query tiles: a TMA box when the rows are contiguous, else
 //               indexed rows gathered with plain loads into the same swizzle
-//   warp 3      idle
-//   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. and quarter
-//               (w-4)/4 of the columns of each accumulator, 32 columns at a
-//               time.  Each thread keeps its row's running maximum; when a
-//               chunk beats it, the chunk's 32 scores are kept (in a private
-//               shared-memory slot, or located at once in registers) and the
-//               lowest index reaching the maximum is found from them.
+//   warps 4..   epilogue (8 or 16 warps), in groups that each own one
+//               accumulator (tiles g, g+nacc, ...), so that one group reduces
+//               while another waits.  Warp w reads TMEM lanes 32*(w%4).. and
+//               its part of the columns, folds them 32 at a time into its
+//               row's running maximum, and keeps the first 32-column chunk
+//               that reached it.
+//
+// The exact lowest index inside the kept chunk is not resolved here: the
+// packed key carries the chunk's first column, and a small pass afterwards
+// recomputes that chunk's 32 scores (locate_chunk, in rnn.cu).  Keeping the
+// locate out of the loop leaves the epilogue with one maximum per score and
+// three instructions per chunk, with no branches and no shared-memory
+// traffic.  Whole chunks compare by their maxima with a strict '>' in
+// increasing column order, so the kept chunk is the first that holds the row
+// maximum and its lowest maximal column is the lowest-index argmax.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -40,11 +51,13 @@
 namespace rnn {
 
 constexpr int kBlockM = 128;
-constexpr int kThreads = 640;
+constexpr int kMmaWarps = 2;     // warps 1..kMmaWarps issue MMAs
+constexpr int kGatherWarp = 3;
 constexpr int kEpiWarp0 = 4;
-constexpr int kEpiWarps = 16;
-constexpr int kSlotBytes = kEpiWarps * 32 * 32 * 4;  // 32 saved scores per epilogue thread
+constexpr int kChunk = 32;       // columns folded per maximum; the locate pass resolves within one
 constexpr int kMaxBatchTable = 1024;
+constexpr int kMaxStages = 16;   // candidate ring depth limit
+constexpr int kMaxAcc = 4;       // accumulator buffers in tensor memory (512 columns in all)
 
 // Error bits written to the device error word.
 constexpr int kErrWaitProducer = 1 << 0;
@@ -76,6 +89,8 @@ struct NNParams {
   int nkb;          // K-blocks; padded depth K = kb * nkb
   int block_n;      // candidates per stage: 256 or 128
   int stages;       // candidate ring depth
+  int nacc;         // accumulators of block_n columns: 2 or 4, nacc * block_n <= 512,
+                    // stages a multiple of nacc
   int qbufs;        // query tile buffers: 1 or 2
   uint32_t idesc;   // tcgen05 instruction descriptor
   int target_units; // units to aim for when choosing the split count
@@ -168,10 +183,12 @@ __device__ __forceinline__ UnitInfo decode_unit(const NNParams& p, const SharedT
 }
 
 // Exclusive scan of `n` values (n <= kMaxBatchTable) of m-tile counts into
-// T.mt_prefix[f][0..n], by all kThreads threads.
+// T.mt_prefix[f][0..n], by all threads of the block (at least 256, at most
+// 32 warps).
 __device__ void build_prefix(const NNFamily& F, int* prefix, int* scratch_warp) {
   const int n = F.nbatch;
-  const int per = (n + kThreads - 1) / kThreads;
+  const int nthreads = blockDim.x, nwarps = nthreads >> 5;
+  const int per = (n + nthreads - 1) / nthreads;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   int vals[4];
   int local = 0;
@@ -196,12 +213,12 @@ __device__ void build_prefix(const NNFamily& F, int* prefix, int* scratch_warp) 
   __syncthreads();
   if (t == 0) {
     int run = 0;
-    for (int w = 0; w < kThreads / 32; ++w) {
+    for (int w = 0; w < nwarps; ++w) {
       const int x = scratch_warp[w];
       scratch_warp[w] = run;
       run += x;
     }
-    scratch_warp[kThreads / 32] = run;
+    scratch_warp[nwarps] = run;
   }
   __syncthreads();
   int run = scratch_warp[warp] + incl - local;
@@ -211,7 +228,7 @@ __device__ void build_prefix(const NNFamily& F, int* prefix, int* scratch_warp) 
     if (e < per && b < n) prefix[b] = run;
     run += vals[e];
   }
-  if (t == 0) prefix[n] = scratch_warp[kThreads / 32];
+  if (t == 0) prefix[n] = scratch_warp[nwarps];
   __syncthreads();
 }
 
@@ -226,16 +243,11 @@ __device__ __forceinline__ float max32(const float (&v)[32]) {
   return fmaxf(fmax3(b0, b1, b2), b3);
 }
 
-// Lowest k with v[k] == m (m is one of the values).
-__device__ __forceinline__ int first_equal32(const float (&v)[32], float m) {
-  int pos = 31;
-#pragma unroll
-  for (int k = 30; k >= 0; --k) pos = (v[k] == m) ? k : pos;
-  return pos;
-}
-
-template <bool kSlotLocate>
-__global__ void __launch_bounds__(kThreads, 1)
+// kEpiWarps: epilogue warps (8 or 16); kChunks: 32-column chunks of each
+// tile read by one of them (block_n * nacc / (8 * kEpiWarps)); kBatch:
+// chunks per copy from tensor memory to registers.
+template <int kEpiWarps, int kChunks, int kBatch>
+__global__ void __launch_bounds__((kEpiWarp0 + kEpiWarps) * 32, 1)
 nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUtensorMap tmap0,
                  const __grid_constant__ CUtensorMap tmap1,
                  const __grid_constant__ CUtensorMap qmap0,
@@ -252,37 +264,40 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
 
   uint8_t* x_tiles = smem;
   uint8_t* q_tiles = x_tiles + static_cast<size_t>(p.stages) * stage_bytes;
-  float* slots = reinterpret_cast<float*>(q_tiles + static_cast<size_t>(p.qbufs) * q_bytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(slots) +
-                                               (kSlotLocate ? kSlotBytes : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(q_tiles + static_cast<size_t>(p.qbufs) * q_bytes);
   uint64_t* full_bar = bars;
-  uint64_t* empty_bar = bars + p.stages;
+  // done_bar[s]: the MMAs that read stage s have completed.  One commit per
+  // tile tells both the producer (the stage may be refilled) and the
+  // epilogue (the accumulator of that tile is ready): every tcgen05.commit
+  // costs the tensor pipe tens of cycles, and a tile is only a few hundred.
+  uint64_t* done_bar = bars + p.stages;
   uint64_t* qfull_bar = bars + 2 * p.stages;
   uint64_t* qempty_bar = qfull_bar + 2;
-  uint64_t* tfull_bar = qempty_bar + 2;
-  uint64_t* tempty_bar = tfull_bar + 2;
-  uint64_t* drain_bar = tempty_bar + 2;
-  uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* tempty_bar = qempty_bar + 2;
+  uint64_t* drain_bar = tempty_bar + kMaxAcc;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(drain_bar + kMmaWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   int* qrows = reinterpret_cast<int*>(misc + 4);            // [128]
-  int* scan_scratch = qrows + kBlockM;                       // [kThreads/32 + 1]
+  int* scan_scratch = qrows + kBlockM;                       // [warps + 1]
   SharedTables* T = reinterpret_cast<SharedTables*>(scan_scratch + 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ncols = static_cast<uint32_t>(2 * p.block_n);
+  const int epi_per_group = kEpiWarps / p.nacc;  // epilogue warps sharing one accumulator
+  // tensor-memory allocation: a power of two of at least 32 columns
+  uint32_t ncols = 32;
+  while (ncols < static_cast<uint32_t>(p.nacc * p.block_n)) ncols <<= 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
-      mbar_init(smem_u32(&empty_bar[s]), 1);
+      mbar_init(smem_u32(&done_bar[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&qfull_bar[i]), 1);
-      mbar_init(smem_u32(&qempty_bar[i]), 1);
-      mbar_init(smem_u32(&tfull_bar[i]), 1);
-      mbar_init(smem_u32(&tempty_bar[i]), kEpiWarps);
+      mbar_init(smem_u32(&qempty_bar[i]), kMmaWarps);
     }
-    mbar_init(smem_u32(drain_bar), 1);
+    for (int i = 0; i < p.nacc; ++i) mbar_init(smem_u32(&tempty_bar[i]), epi_per_group);
+    for (int i = 0; i < kMmaWarps; ++i) mbar_init(smem_u32(&drain_bar[i]), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -344,8 +359,8 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
         const UnitInfo ui = decode_unit(p, *T, u);
         const CUtensorMap* map = ui.f == 0 ? &tmap0 : &tmap1;
         for (int t = ui.t0; t < ui.t1; ++t) {
-          if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
-                         kErrWaitProducer, lim)) {
+          if (!mbar_wait_sleep(smem_u32(&done_bar[stage]), phase ^ 1u, abort_flag, p.err,
+                               kErrWaitProducer, lim)) {
             ok = false;
             break;
           }
@@ -377,13 +392,12 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    // The issue loop is latency-critical (two MMAs per 256-cycle tile at
-    // K = 32).  The whole warp runs it on warp-uniform values (so they live
-    // in uniform registers, where tcgen05.mma reads its operands), the
-    // descriptors are built once, only their 16-byte start-address field
-    // moves, and one elected lane issues.
+  } else if (warp <= kMmaWarps) {
+    // ------------------------------------------------------ MMA issuers
+    // Warp 1 takes the tiles g = 0, 2, 4, ... of this CTA's sequence, warp 2
+    // the odd ones (nacc is even, so each warp keeps its own accumulators).
+    // The loop runs on warp-uniform values and one elected lane issues.
+    const int mw = warp - 1;
     int stage = 0, acc = 0, qb = 0;
     uint32_t phase = 0, acc_phase = 0, qphase = 0;
     bool ok = true, any = false;
@@ -395,28 +409,27 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
     const uint32_t b_jump = (kblk_bytes_x - (spk - 1) * 32) >> 4;
     const uint32_t q_step = q_bytes >> 4, x_step = stage_bytes >> 4;
     const uint32_t idesc = p.idesc;
-    uint64_t b_stage = b_desc0;
-    uint64_t a_unit = a_desc0;
     for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       const UnitInfo ui = decode_unit(p, *T, u);
       ok = __all_sync(0xffffffffu,
                       mbar_wait(smem_u32(&qfull_bar[qb]), qphase, abort_flag, p.err, kErrWaitMma,
                                 lim));
       if (!ok) break;
+      const uint64_t a_unit = a_desc0 + static_cast<uint64_t>(qb) * q_step;
       for (int t = ui.t0; t < ui.t1; ++t) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err,
-                                  kErrWaitMma, lim) &&
-                            mbar_wait(smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag,
-                                      p.err, kErrWaitMma, lim));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (acc ? static_cast<uint32_t>(p.block_n) : 0u);
-        uint64_t a = a_unit, b = b_stage;
-        if (elect_one()) {
+        if ((acc & 1) == mw) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err,
+                                    kErrWaitMma, lim) &&
+                              mbar_wait_sleep(smem_u32(&tempty_bar[acc]), acc_phase ^ 1u,
+                                              abort_flag, p.err, kErrWaitMma, lim));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * p.block_n);
+          uint64_t a = a_unit, b = b_desc0 + static_cast<uint64_t>(stage) * x_step;
           int w = 0;
           for (int k = 0; k < ksteps; ++k) {
-            umma_f16(d_tmem, a, b, idesc, k > 0 ? 1u : 0u);
+            umma_f16_warp(d_tmem, a, b, idesc, k > 0 ? 1u : 0u);
             if (++w == spk) {
               w = 0;
               a += a_jump;
@@ -426,45 +439,41 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
               b += 2;
             }
           }
-          umma_commit(smem_u32(&empty_bar[stage]));
-          umma_commit(smem_u32(&tfull_bar[acc]));
+          umma_commit_warp(smem_u32(&done_bar[stage]));
+          __syncwarp();
+          any = true;
         }
-        __syncwarp();
-        any = true;
-        b_stage += x_step;
         if (++stage == p.stages) {
           stage = 0;
           phase ^= 1u;
-          b_stage = b_desc0;
         }
-        if (++acc == 2) {
+        if (++acc == p.nacc) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       if (!ok) break;
-      if (elect_one()) umma_commit(smem_u32(&qempty_bar[qb]));
+      // the query tile is free once both warps' MMAs of the unit are done
+      umma_commit_warp(smem_u32(&qempty_bar[qb]));
       __syncwarp();
-      a_unit += q_step;
       if (++qb == p.qbufs) {
         qb = 0;
         qphase ^= 1u;
-        a_unit = a_desc0;
       }
     }
     if (!ok && any) {
-      // let every MMA issued so far finish before tensor memory is released
-      if (elect_one()) umma_commit(smem_u32(drain_bar));
+      // let every MMA this warp issued finish before tensor memory is released
+      umma_commit_warp(smem_u32(&drain_bar[mw]));
       __syncwarp();
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(drain_bar), 0)) {
+      while (!mbar_try_wait(smem_u32(&drain_bar[mw]), 0)) {
         if (globaltimer_ns() - t0 > lim) {
           if (lane == 0) atomicOr(p.err, kErrDrain);
           break;
         }
       }
     }
-  } else if (warp == 2) {
+  } else if (warp == kGatherWarp) {
     // ---------------------------------------------------- query gather
     int qb = 0;
     uint32_t qphase = 0;
@@ -476,8 +485,8 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
     const int ch_per_kblk = p.kb / 8;
     for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
       const UnitInfo ui = decode_unit(p, *T, u);
-      if (!mbar_wait(smem_u32(&qempty_bar[qb]), qphase ^ 1u, abort_flag, p.err, kErrWaitGather,
-                     lim))
+      if (!mbar_wait_sleep(smem_u32(&qempty_bar[qb]), qphase ^ 1u, abort_flag, p.err,
+                           kErrWaitGather, lim))
         break;
       const NNFamily& F = p.fam[ui.f];
       if (F.q_tma) {
@@ -556,81 +565,85 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
         }
       }
     }
-  } else if (warp >= kEpiWarp0) {
+  } else {
     // --------------------------------------------------------- epilogue
+    // Group `grp` owns accumulator grp and reduces the tiles g with
+    // g % nacc == grp; within it, warp w covers TMEM lanes 32*(w%4).. and
+    // column part `part` of each tile, kBatch chunks of 32 columns per copy
+    // to registers.  After the last copy of a tile the accumulator goes back
+    // to the MMA warps, before that copy is folded.
     const int ew = warp - kEpiWarp0;
     const int quad = warp & 3;
-    const int part = ew >> 2;
+    const int grp = ew / epi_per_group;
+    const int part = (ew - grp * epi_per_group) >> 2;
     const int row = quad * 32 + lane;
-    const int cols_part = p.block_n / 4;
-    // private slot of 32 floats; 16-byte unit q lives at (q ^ lane) & 7
-    float* slot = slots + (ew * 32 + lane) * 32;
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    constexpr int cols_part = kChunk * kChunks;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(grp * p.block_n + part * cols_part);
+    int acc = 0, stage = 0;  // position of tile t in this CTA's tile sequence
+    uint32_t phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       const UnitInfo ui = decode_unit(p, *T, u);
       const NNFamily& F = p.fam[ui.f];
       float best = -__int_as_float(0x7f800000);
-      int arg = -1;  // slot mode: first column of the kept chunk; else the index
+      int bcol = -1;  // first column of the first chunk that reached `best`
       for (int t = ui.t0; t < ui.t1; ++t) {
-        if (!mbar_wait(smem_u32(&tfull_bar[acc]), acc_phase, abort_flag, p.err, kErrWaitEpilogue,
-                       lim)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int col0 = t * p.block_n + part * cols_part;   // first candidate of this part
-        const int valid = F.n_cand - col0;                    // candidates left from col0
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                               static_cast<uint32_t>(acc * p.block_n + part * cols_part);
-        for (int c = 0; c < cols_part; c += 32) {
-          float v[32];
-          tmem_ld32(taddr + c, v);
-          tmem_wait_ld_regs(v);
-          if (valid - c < 32) {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (c + k >= valid) v[k] = -__int_as_float(0x7f800000);
+        if (acc == grp) {
+          // stages is a multiple of nacc, so done_bar[stage] is only ever
+          // used by this group's tiles, and its next phase needs this tile's
+          // accumulator back: the parity below cannot be a phase behind
+          if (!mbar_wait_sleep(smem_u32(&done_bar[stage]), phase, abort_flag, p.err,
+                               kErrWaitEpilogue, lim)) {
+            ok = false;
+            break;
           }
-          const float m = max32(v);
-          if (m > best) {
-            best = m;
-            if (kSlotLocate) {
-              arg = col0 + c;
+          tc_fence_after();
+          const int col0 = t * p.block_n + part * cols_part;   // first candidate of this part
+          const int valid = F.n_cand - col0;                    // candidates left from col0
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4*>(slot + ((q ^ lane) & 7) * 4) =
-                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            } else {
-              arg = col0 + c + first_equal32(v, m);
+          for (int h = 0; h < kChunks; h += kBatch) {
+            float v[kBatch][kChunk];
+#pragma unroll
+            for (int c = 0; c < kBatch; ++c) tmem_ld32(lane_base + kChunk * (h + c), v[c]);
+            tmem_wait_ld_regs(v[0]);
+#pragma unroll
+            for (int c = 1; c < kBatch; ++c) reg_fence(v[c]);
+            if (h + kBatch == kChunks) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
+              // keep the reductions below the release
+#pragma unroll
+              for (int c = 0; c < kBatch; ++c) reg_fence(v[c]);
+            }
+            if (valid < kChunk * (h + kBatch)) {
+              // ragged last tile: columns past the candidates never win
+#pragma unroll
+              for (int c = 0; c < kBatch; ++c)
+#pragma unroll
+                for (int k = 0; k < kChunk; ++k)
+                  if (kChunk * (h + c) + k >= valid) v[c][k] = -__int_as_float(0x7f800000);
+            }
+#pragma unroll
+            for (int c = 0; c < kBatch; ++c) {
+              const float m = max32(v[c]);
+              const bool up = m > best;
+              best = up ? m : best;
+              bcol = up ? col0 + kChunk * (h + c) : bcol;
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1u;
         }
+        if (++acc == p.nacc) acc = 0;
       }
       if (!ok) break;
-      if (row < ui.nrows && arg >= 0) {
-        if (kSlotLocate) {
-          float w[32];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 x = *reinterpret_cast<const float4*>(slot + ((q ^ lane) & 7) * 4);
-            w[4 * q] = x.x;
-            w[4 * q + 1] = x.y;
-            w[4 * q + 2] = x.z;
-            w[4 * q + 3] = x.w;
-          }
-          arg += first_equal32(w, best);
-        }
+      if (row < ui.nrows && bcol >= 0) {
         unsigned long long* kp = F.keys + ui.b * F.key_bstride + ui.m * kBlockM + row;
-        atomicMax(kp, pack_key(best, arg));
+        atomicMax(kp, pack_key(best, bcol));
       }
     }
   }

@@ -5,6 +5,8 @@
 // on the caller's stream.  No allocation, no synchronisation: scratch lives in
 // the caller's workspace.
 #include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -82,12 +84,21 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Operand geometry for a channel count d.
 struct Geometry {
-  int kb, nkb, kpad, block_n, stages, qbufs;
-  bool slot_locate;  // epilogue keeps improving chunks in shared memory
+  int kb, nkb, kpad, block_n, nacc, stages, qbufs;
   size_t smem;
 };
 
 static size_t tables_bytes() { return sizeof(SharedTables); }
+
+// Epilogue warps of the fused kernel: 8 (two accumulators) or 16.
+#ifndef RNN_EPI_WARPS
+#define RNN_EPI_WARPS 8
+#endif
+
+// Candidate tile width for K <= 64: 128 (four accumulators) or 256 (two).
+#ifndef RNN_SMALL_K_BLOCK_N
+#define RNN_SMALL_K_BLOCK_N 256
+#endif
 
 static Geometry geometry(int d) {
   Geometry g;
@@ -103,22 +114,24 @@ static Geometry geometry(int d) {
     g.kb = 16; g.nkb = (d + 15) / 16;
   }
   g.kpad = g.kb * g.nkb;
-  // small d: the argmax epilogue bounds the kernel, so it gets the 64 KB of
-  // score slots; large d: the tensor cores bound it and the slots would not fit
-  g.slot_locate = g.kpad <= 64;
-  g.block_n = g.kpad <= 64 ? 256 : 128;
+  g.block_n = g.kpad <= 64 ? RNN_SMALL_K_BLOCK_N : 128;
+  g.nacc = 512 / g.block_n;
   const size_t stage = static_cast<size_t>(g.block_n) * g.kpad * 2;
   const size_t qb = static_cast<size_t>(kBlockM) * g.kpad * 2;
-  const size_t slots = g.slot_locate ? kSlotBytes : 0;
   const size_t fixed = 1024 /*align slack*/ + 16 + kBlockM * 4 + 32 * 4 + tables_bytes();
   const size_t budget = 227 * 1024;
-  const size_t bars = (2 * 8 + 9) * 8;
-  const size_t avail = budget - fixed - bars - slots;
+  const size_t bars = (2 * kMaxStages + 4 + kMaxAcc + kMmaWarps) * 8;
+  const size_t avail = budget - fixed - bars;
   g.qbufs = (2 * qb + 2 * stage <= avail) ? 2 : 1;
   size_t st = (avail - g.qbufs * qb) / stage;
-  if (st > 8) st = 8;
+  if (st > kMaxStages) st = kMaxStages;
+  // one barrier per stage also signals the accumulators: each epilogue group
+  // waits on the stages of its own tiles only, which needs the stage count
+  // to be a multiple of the accumulator count (2 or 4)
+  if (g.nacc > 2 && st < 4) g.nacc = 2;
+  st -= st % g.nacc;
   g.stages = static_cast<int>(st);
-  g.smem = fixed + (2 * g.stages + 9) * 8 + g.stages * stage + g.qbufs * qb + slots;
+  g.smem = fixed + bars + g.stages * stage + g.qbufs * qb;
   // at least half the SM's shared memory, so that two CTAs never share an SM
   // (each one allocates all 512 tensor-memory columns)
   if (g.smem < 116 * 1024) g.smem = 116 * 1024;
@@ -179,6 +192,7 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
   p.nkb = g.nkb;
   p.block_n = g.block_n;
   p.stages = g.stages;
+  p.nacc = g.nacc;
   p.qbufs = g.qbufs;
   p.target_units = 8 * di->sms;
   {
@@ -190,12 +204,12 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!di->smem_set) {
-      if (cudaFuncSetAttribute(nn_argmax_kernel<true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               227 * 1024) != cudaSuccess ||
-          cudaFuncSetAttribute(nn_argmax_kernel<false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               227 * 1024) != cudaSuccess)
+      const int sm = 227 * 1024;
+      const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+      if (cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2>, attr, sm) != cudaSuccess ||
+          cudaFuncSetAttribute(nn_argmax_kernel<16, 4, 2>, attr, sm) != cudaSuccess ||
+          cudaFuncSetAttribute(nn_argmax_kernel<8, 4, 4>, attr, sm) != cudaSuccess ||
+          cudaFuncSetAttribute(nn_argmax_kernel<8, 8, 4>, attr, sm) != cudaSuccess)
         return RNN_ECUDA;
       di->smem_set = true;
     }
@@ -210,10 +224,22 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
       slot = -1;
     }
   }
-  if (g.slot_locate)
-    nn_argmax_kernel<true><<<di->sms, kThreads, g.smem, s>>>(p, m0, m1, q0, q1);
-  else
-    nn_argmax_kernel<false><<<di->sms, kThreads, g.smem, s>>>(p, m0, m1, q0, q1);
+  // Epilogue layout: with two accumulators, eight warps (one per lane
+  // quadrant and accumulator) copying 128 columns per round trip to
+  // tensor memory; with four, sixteen warps copying 64.  Each row gets
+  // kEpiWarps / 4 warps, each covering block_n * nacc / (8 * kEpiWarps) chunks.
+  const bool wide = g.block_n * g.nacc == 512;
+  if (RNN_EPI_WARPS == 8 && g.nacc == 2) {
+    if (wide)
+      nn_argmax_kernel<8, 8, 4><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
+    else
+      nn_argmax_kernel<8, 4, 4><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
+  } else {
+    if (wide)
+      nn_argmax_kernel<16, 4, 2><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
+    else
+      nn_argmax_kernel<16, 2, 2><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
+  }
   const rnn_status r = launched();
   if (r == RNN_OK && slot >= 0 &&
       cudaEventRecord(static_cast<cudaEvent_t>(g_timer_stop[slot]), s) != cudaSuccess)
@@ -245,14 +271,84 @@ __global__ void zero_keys_kernel(unsigned long long* a, int64_t na, unsigned lon
   if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
 }
 
-__global__ void unpack_kernel(const unsigned long long* keys, int64_t n, int32_t* idx,
-                              float* score) {
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += stride) {
+// ------------------------------------------------------------------ locate
+// The fused kernel leaves, per query, the largest score and the first column
+// c0 of the first 32-column chunk that reaches it.  locate_chunk recomputes
+// the scores of that chunk (one candidate per lane, fp32 fused multiply-adds
+// over the channels in order) and returns the lowest column that reaches
+// their maximum.  On inputs whose products and partial sums are exact in
+// fp32 (the quantised k/64 maps) the recomputed scores equal the tensor
+// cores' bit for bit, so the result is the exact lowest-index argmax; on
+// other inputs the two roundings can differ only between scores within fp32
+// rounding of each other.  Warp-collective: all lanes pass the same query.
+__device__ __forceinline__ float h2f(uint16_t h, bool bf16) {
+  return bf16 ? __bfloat162float(__ushort_as_bfloat16(h)) : __half2float(__ushort_as_half(h));
+}
+
+template <bool kBf16>
+__device__ __forceinline__ float dot_rows(const uint16_t* a, const uint16_t* b, int d) {
+  float acc = 0.f;
+  for (int c = 0; c < d; c += 8) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(a + c));
+    const uint4 y = __ldg(reinterpret_cast<const uint4*>(b + c));
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(h2f(static_cast<uint16_t>(xs[e] & 0xFFFFu), kBf16),
+                 h2f(static_cast<uint16_t>(ys[e] & 0xFFFFu), kBf16), acc);
+      acc = fmaf(h2f(static_cast<uint16_t>(xs[e] >> 16), kBf16),
+                 h2f(static_cast<uint16_t>(ys[e] >> 16), kBf16), acc);
+    }
+  }
+  return acc;
+}
+
+template <bool kBf16>
+__device__ __forceinline__ int locate_chunk(const uint16_t* q, const uint16_t* X, int n_cand,
+                                            int d, int c0) {
+  const int lane = threadIdx.x & 31;
+  const int j = c0 + lane;
+  float sc = -__int_as_float(0x7f800000);
+  if (j < n_cand) sc = dot_rows<kBf16>(q, X + static_cast<int64_t>(j) * d, d);
+  float m = sc;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const unsigned hit = __ballot_sync(0xffffffffu, sc == m);
+  return c0 + __ffs(hit) - 1;
+}
+
+// nn_argmax results: locate every query's index, write index and score.
+template <bool kBf16>
+__global__ void locate_unpack_kernel(const unsigned long long* keys, int64_t n, const uint16_t* Q,
+                                     const uint16_t* X, int nx, int d, int32_t* idx,
+                                     float* score) {
+  const int64_t w0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t i = w0; i < n; i += nw) {
     const unsigned long long k = keys[i];
-    idx[i] = key_index(k);
-    if (score) score[i] = key_score(k);
+    const int j = locate_chunk<kBf16>(Q + i * d, X, nx, d, key_index(k));
+    if ((threadIdx.x & 31) == 0) {
+      idx[i] = j;
+      if (score) score[i] = key_score(k);
+    }
+  }
+}
+
+// Both sweeps of the reciprocal set: rewrite each packed key with its exact
+// index (rows of D1 against D2, then rows of D2 against D1).
+template <bool kBf16>
+__global__ void locate_mnn_kernel(unsigned long long* rowk, int64_t n1, unsigned long long* colk,
+                                  int64_t n2, const uint16_t* D1, const uint16_t* D2, int d) {
+  const int64_t w0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t i = w0; i < n1 + n2; i += nw) {
+    const bool row = i < n1;
+    const int64_t r = row ? i : i - n1;
+    unsigned long long* kp = row ? rowk + r : colk + r;
+    const unsigned long long k = *kp;
+    const int j = row ? locate_chunk<kBf16>(D1 + r * d, D2, static_cast<int>(n2), d, key_index(k))
+                      : locate_chunk<kBf16>(D2 + r * d, D1, static_cast<int>(n1), d, key_index(k));
+    if ((threadIdx.x & 31) == 0) *kp = pack_key(key_score(k), j);
   }
 }
 
@@ -375,7 +471,10 @@ struct FrmState {
   unsigned long long* keys;  // [B][k] NN result per list position
   uint32_t* bitmap; // [B][nwords] converged image-1 pixels
   int32_t* partner; // [B][N1] image-2 partner of a converged pixel
-  int B, k, N1, nwords;
+  const uint16_t* D1;  // descriptor maps (for the locate pass), pair b at D1 + b*bs1
+  const uint16_t* D2;
+  int64_t bs1, bs2;
+  int B, k, N1, N2, nwords, d;
 };
 
 // Workspace layout of a batched FRM call; returns the bytes it needs.
@@ -433,6 +532,30 @@ __global__ void frm_init_kernel(FrmState st, int W1, int S) {
   if (blockIdx.x == 0) {
     for (int b = threadIdx.x; b < st.B; b += blockDim.x) st.count[b] = st.k;
     if (threadIdx.x == 0) *st.err = 0;
+  }
+}
+
+// Exact index inside each kept chunk for every active seed of every pair
+// (one warp per seed): NN2 queries are rows U of D1 against D2, NN1 queries
+// rows V of D2 against D1.
+template <bool kBf16>
+__global__ void frm_locate_kernel(FrmState st, int nn2_half) {
+  const int64_t w0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int n_cand = nn2_half ? st.N2 : st.N1;
+  const int32_t* rows = nn2_half ? st.U : st.V;
+  for (int64_t x = w0; x < static_cast<int64_t>(st.B) * st.k; x += nw) {
+    const int b = static_cast<int>(x / st.k);
+    const int i = static_cast<int>(x - static_cast<int64_t>(b) * st.k);
+    if (i >= st.count[b]) continue;
+    const int64_t base = static_cast<int64_t>(b) * st.k;
+    const uint16_t* Dq = nn2_half ? st.D1 + b * st.bs1 : st.D2 + b * st.bs2;
+    const uint16_t* Dx = nn2_half ? st.D2 + b * st.bs2 : st.D1 + b * st.bs1;
+    const int sl = st.list[base + i];
+    const unsigned long long k = st.keys[base + i];
+    const int64_t qr = rows[base + sl];
+    const int j = locate_chunk<kBf16>(Dq + qr * st.d, Dx, n_cand, st.d, key_index(k));
+    if ((threadIdx.x & 31) == 0) st.keys[base + i] = pack_key(key_score(k), j);
   }
 }
 
@@ -530,6 +653,15 @@ static int grid_for(int64_t n, int sms) {
   return static_cast<int>(g);
 }
 
+static rnn_status frm_locate(const FrmState& st, int nn2_half, rnn_dtype dt, int grid,
+                             cudaStream_t s) {
+  if (dt == RNN_BF16)
+    frm_locate_kernel<true><<<grid, kSmallThreads, 0, s>>>(st, nn2_half);
+  else
+    frm_locate_kernel<false><<<grid, kSmallThreads, 0, s>>>(st, nn2_half);
+  return launched();
+}
+
 static int64_t num_seeds(int H, int W, int S) {
   const int o = S / 2;
   const int64_t ny = H > o ? (H - o + S - 1) / S : 0;
@@ -563,6 +695,12 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
 
   FrmState st;
   frm_layout(ws, B, k, N1, &st);
+  st.D1 = static_cast<const uint16_t*>(D1);
+  st.D2 = static_cast<const uint16_t*>(D2);
+  st.bs1 = bs1;
+  st.bs2 = bs2;
+  st.N2 = static_cast<int>(N2);
+  st.d = d;
   const Geometry g = geometry(d);
   if (k == 0) {
     // no seeds: every count is zero
@@ -575,6 +713,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   if ((r = make_map(&map2, D2, d, N2, B, bs2, g)) != RNN_OK) return r;
 
   frm_init_kernel<<<grid_for(B * k + B * st.nwords, di->sms), kSmallThreads, 0, s>>>(st, W1, S);
+  const int lgrid = grid_for(static_cast<int64_t>(B) * k * 32, di->sms);
   if ((r = launched()) != RNN_OK) return r;
 
   NNParams p;
@@ -597,6 +736,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_index = st.U;
     F.n_cand = static_cast<int32_t>(N2);
     if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s)) != RNN_OK) return r;
+    if ((r = frm_locate(st, 1, dt, lgrid, s)) != RNN_OK) return r;
     frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 1, 0);
     if ((r = launched()) != RNN_OK) return r;
     // half-step 2: U = NN1(V)
@@ -605,6 +745,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_index = st.V;
     F.n_cand = static_cast<int32_t>(N1);
     if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s)) != RNN_OK) return r;
+    if ((r = frm_locate(st, 0, dt, lgrid, s)) != RNN_OK) return r;
     frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 0, it == max_iter ? 1 : 0);
     if ((r = launched()) != RNN_OK) return r;
   }
@@ -704,7 +845,17 @@ rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, i
   F.keys = keys;
   F.q_tma = 1;
   if ((r = launch_nn(p, mx, mx, mq, mq, g, di, s)) != RNN_OK) return r;
-  unpack_kernel<<<grid_for(nq, di->sms), kSmallThreads, 0, s>>>(keys, nq, idx_out, score_out);
+  const int lg = grid_for(nq * 32, di->sms);
+  const uint16_t* q16 = static_cast<const uint16_t*>(Q);
+  const uint16_t* x16 = static_cast<const uint16_t*>(X);
+  if (dtype == RNN_BF16)
+    locate_unpack_kernel<true><<<lg, kSmallThreads, 0, s>>>(keys, nq, q16, x16,
+                                                           static_cast<int>(nx), d, idx_out,
+                                                           score_out);
+  else
+    locate_unpack_kernel<false><<<lg, kSmallThreads, 0, s>>>(keys, nq, q16, x16,
+                                                            static_cast<int>(nx), d, idx_out,
+                                                            score_out);
   return launched();
 }
 
@@ -776,6 +927,16 @@ rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, in
   p.fam[1].q_tma = 1;
   if ((r = launch_nn(p, m2, m1, q1, q2, g, di, s)) != RNN_OK) return r;
   const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
+  {
+    const int lg = grid_for((n1 + n2) * 32, di->sms);
+    const uint16_t* a16 = static_cast<const uint16_t*>(D1);
+    const uint16_t* b16 = static_cast<const uint16_t*>(D2);
+    if (dtype == RNN_BF16)
+      locate_mnn_kernel<true><<<lg, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, a16, b16, d);
+    else
+      locate_mnn_kernel<false><<<lg, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, a16, b16, d);
+    if ((r = launched()) != RNN_OK) return r;
+  }
   mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, counts, nblk1, rowarg_out,
                                                 rowmax_out, colarg_out, colmax_out);
   if ((r = launched()) != RNN_OK) return r;
