@@ -337,7 +337,7 @@ def run_native(args):
             a, b = synth.make_workload_storage(ww, "f16", pairs=[0])
             a, b = a[0].to(dev), b[0].to(dev)
             out = rnn.mnn_exhaustive(a, b)
-            ws = torch.empty(lib.rnn_mnn_workspace_size(ww.H, ww.W, ww.H, ww.W),
+            ws = torch.empty(lib.rnn_mnn_workspace_size(ww.H, ww.W, ww.H, ww.W, ww.d),
                              dtype=torch.uint8, device=dev)
             reps = args.mnn_reps
             ka = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]

@@ -102,9 +102,12 @@ rnn_status rnn_nn_argmax(const void *Q, int64_t nq, const void *X, int64_t nx, i
  *   rowarg_out [H1*W1] NN2 of every D1 pixel, rowmax_out its score,
  *   colarg_out [H2*W2] NN1 of every D2 pixel, colmax_out its score;
  *              each of these four may be NULL.
- *   workspace  at least rnn_mnn_workspace_size(H1, W1, H2, W2) bytes.
+ *   workspace  at least rnn_mnn_workspace_size(H1, W1, H2, W2, d) bytes,
+ *              256-byte aligned.  When d is not a whole number of the
+ *              tensor-core K-blocks (d = 8, 24, 40, ...) it also holds
+ *              zero-padded copies of both maps, made by the call.
  */
-size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2);
+size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2, int d);
 rnn_status rnn_mnn_exhaustive(const void *D1, int H1, int W1, const void *D2, int H2, int W2,
                               int d, rnn_dtype dtype, int32_t *pairs_out, int64_t cap,
                               int32_t *count_out, int32_t *rowarg_out, float *rowmax_out,
@@ -128,19 +131,21 @@ rnn_status rnn_mnn_exhaustive(const void *D1, int H1, int W1, const void *D2, in
  *   output the (U, V) of the seeds that are no longer active, unique, sorted
  *          by U.  Every output pair is in M.
  *
- * The whole loop runs on the device: 4*max_iter + 2 kernel launches, no host
- * synchronisation.
+ * The whole loop runs on the device: 6*max_iter + 2 kernel launches (2 more
+ * when d needs padded copies), no host synchronisation.
  *
  *   seed_stride >= 1, max_iter >= 1 (RNN_EINVAL otherwise).
  *   pairs_out   [cap][2] int32, cap >= rnn_frm_max_pairs(...).
  *   count_out   [1] int32.
  *   seed_state_out  (may be NULL) [k][4] int32 per seed: final U, final V,
  *               number of NN queries made for it, 1 if converged else 0.
- *   workspace   at least rnn_frm_workspace_size(1, H1, W1, H2, W2, seed_stride).
+ *   workspace   at least rnn_frm_workspace_size(1, H1, W1, H2, W2, d, seed_stride)
+ *               bytes, 256-byte aligned (it holds zero-padded copies of the
+ *               maps when d is not a whole number of K-blocks).
  */
 int64_t rnn_frm_num_seeds(int H1, int W1, int seed_stride);
 int64_t rnn_frm_max_pairs(int H1, int W1, int H2, int W2, int seed_stride);
-size_t rnn_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int seed_stride);
+size_t rnn_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int d, int seed_stride);
 rnn_status rnn_frm_match(const void *D1, int H1, int W1, const void *D2, int H2, int W2, int d,
                          rnn_dtype dtype, int seed_stride, int max_iter, int32_t *pairs_out,
                          int64_t cap, int32_t *count_out, int32_t *seed_state_out,

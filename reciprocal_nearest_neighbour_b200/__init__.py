@@ -142,7 +142,7 @@ def mnn_exhaustive(D1: torch.Tensor, D2: torch.Tensor, *, with_nn: bool = False,
             out.rowmax = torch.empty(n1, dtype=torch.float32, device=dev)
             out.colarg = torch.empty(n2, dtype=torch.int32, device=dev)
             out.colmax = torch.empty(n2, dtype=torch.float32, device=dev)
-    need = lib.rnn_mnn_workspace_size(H1, W1, H2, W2)
+    need = lib.rnn_mnn_workspace_size(H1, W1, H2, W2, d)
     if workspace is None:
         workspace = _workspace(need, dev)
     _lib.check(lib.rnn_mnn_exhaustive(
@@ -187,8 +187,8 @@ class FRMPlan:
         self.k = int(lib.rnn_frm_num_seeds(H1, W1, seed_stride))
         self.cap = max(1, int(lib.rnn_frm_max_pairs(H1, W1, H2, W2, seed_stride)))
         dev = torch.device(device)
-        self.workspace = _workspace(lib.rnn_frm_workspace_size(B, H1, W1, H2, W2, seed_stride),
-                                    dev)
+        self.workspace = _workspace(
+            lib.rnn_frm_workspace_size(B, H1, W1, H2, W2, d, seed_stride), dev)
         self.result = FRMResult(
             torch.empty((B, self.cap, 2), dtype=torch.int32, device=dev),
             torch.zeros(B, dtype=torch.int32, device=dev),
@@ -237,7 +237,8 @@ def frm_match(D1: torch.Tensor, D2: torch.Tensor, seed_stride: int = 8, max_iter
                     torch.empty((1, max(k, 1), 4), dtype=torch.int32, device=dev)
                     if with_seed_state else None)
     if workspace is None:
-        workspace = _workspace(lib.rnn_frm_workspace_size(1, H1, W1, H2, W2, seed_stride), dev)
+        workspace = _workspace(lib.rnn_frm_workspace_size(1, H1, W1, H2, W2, d, seed_stride),
+                               dev)
     _lib.check(lib.rnn_frm_match(
         D1.data_ptr(), H1, W1, D2.data_ptr(), H2, W2, d, _dtype_code(D1), seed_stride, max_iter,
         out.pairs.data_ptr(), cap, out.count.data_ptr(), _ptr(out.seed_state),

@@ -73,11 +73,11 @@ def load():
         "rnn_workspace_status": (I, [P, P]),
         "rnn_nn_workspace_size": (SZ, [I64]),
         "rnn_nn_argmax": (I, [P, I64, P, I64, I, I, P, P, P, SZ, P]),
-        "rnn_mnn_workspace_size": (SZ, [I, I, I, I]),
+        "rnn_mnn_workspace_size": (SZ, [I, I, I, I, I]),
         "rnn_mnn_exhaustive": (I, [P, I, I, P, I, I, I, I, P, I64, P, P, P, P, P, P, SZ, P]),
         "rnn_frm_num_seeds": (I64, [I, I, I]),
         "rnn_frm_max_pairs": (I64, [I, I, I, I, I]),
-        "rnn_frm_workspace_size": (SZ, [I, I, I, I, I, I]),
+        "rnn_frm_workspace_size": (SZ, [I, I, I, I, I, I, I]),
         "rnn_frm_match": (I, [P, I, I, P, I, I, I, I, I, I, P, I64, P, P, P, SZ, P]),
         "rnn_frm_match_batched": (I, [I, P, I64, P, I64, I, I, I, I, I, I, I, I, P, I64, P, P, P,
                                       SZ, P]),

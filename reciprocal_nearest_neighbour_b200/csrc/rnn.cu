@@ -138,6 +138,10 @@ static Geometry geometry(int d) {
   return g;
 }
 
+// Depth K of the tensor-core tiles for d channels (d rounded up to the
+// K-block layout the geometry picks).
+static int padded_depth(int d) { return geometry(d).kpad; }
+
 static uint32_t make_idesc(rnn_dtype dt, int block_n) {
   const uint32_t fmt = dt == RNN_BF16 ? 1u : 0u;
   uint32_t d = 0;
@@ -269,6 +273,29 @@ __global__ void zero_keys_kernel(unsigned long long* a, int64_t na, unsigned lon
     if (i < na) a[i] = 0ull; else b[i - na] = 0ull;
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
+}
+
+// Copy [nbatch][rows][d] descriptors (batch stride `bstride` elements) into
+// [nbatch][rows][kpad] rows padded with zeros.  The fused kernel's candidate
+// tiles are K = kpad wide; when d < kpad (d = 8, 24, 40, ...) a tensor map
+// over the caller's d-wide rows would zero-fill part of every box and fetch
+// rows that straddle L2 sectors, which costs the d = 24 sweep about a fifth
+// of its time.  The zeros add nothing to any dot product.
+__global__ void pad_rows_kernel(const uint16_t* src, int64_t bstride, int64_t rows, int nbatch,
+                                int d, uint16_t* dst, int kpad) {
+  const int cpr = kpad / 8, creal = d / 8;  // 16-byte chunks per padded / real row
+  const int64_t total = static_cast<int64_t>(nbatch) * rows * cpr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += stride) {
+    const int64_t rr = i / cpr;  // row over all batches
+    const int c = static_cast<int>(i - rr * cpr);
+    const int64_t b = rr / rows, r = rr - b * rows;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (c < creal)
+      v = __ldg(reinterpret_cast<const uint4*>(src + b * bstride + r * d) + c);
+    reinterpret_cast<uint4*>(dst)[i] = v;
+  }
 }
 
 // ------------------------------------------------------------------ locate
@@ -473,12 +500,15 @@ struct FrmState {
   int32_t* partner; // [B][N1] image-2 partner of a converged pixel
   const uint16_t* D1;  // descriptor maps (for the locate pass), pair b at D1 + b*bs1
   const uint16_t* D2;
+  uint16_t* P1;        // zero-padded copies [B][N][kpad] for the tensor maps, when d < kpad
+  uint16_t* P2;
   int64_t bs1, bs2;
   int B, k, N1, N2, nwords, d;
 };
 
 // Workspace layout of a batched FRM call; returns the bytes it needs.
-static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, FrmState* st) {
+static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int d,
+                         FrmState* st) {
   Carve c(ws);
   st->err = c.take<int>(64);
   st->count = c.take<int32_t>(B);
@@ -493,6 +523,9 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, FrmState* st) {
   const int64_t nwords = (N1 + 31) / 32;
   st->bitmap = c.take<uint32_t>(B * nwords);
   st->partner = c.take<int32_t>(B * N1);
+  const int kpad = padded_depth(d);
+  st->P1 = kpad != d ? c.take<uint16_t>(B * N1 * kpad) : nullptr;
+  st->P2 = kpad != d ? c.take<uint16_t>(B * N2 * kpad) : nullptr;
   st->B = B;
   st->k = static_cast<int>(k);
   st->N1 = static_cast<int>(N1);
@@ -500,9 +533,9 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, FrmState* st) {
   return c.off;
 }
 
-static size_t frm_bytes(int B, int64_t k, int64_t N1) {
+static size_t frm_bytes(int B, int64_t k, int64_t N1, int64_t N2, int d) {
   FrmState st;
-  return frm_layout(nullptr, B, k, N1, &st);
+  return frm_layout(nullptr, B, k, N1, N2, d, &st);
 }
 
 __global__ void frm_init_kernel(FrmState st, int W1, int S) {
@@ -688,13 +721,13 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   const int64_t k = num_seeds(H1, W1, S);
   const int64_t need = k < N2 ? k : N2;
   if (cap < need) return RNN_ECAPACITY;
-  if (!ws || !aligned256(ws) || ws_bytes < frm_bytes(B, k, N1)) return RNN_EWORKSPACE;
+  if (!ws || !aligned256(ws) || ws_bytes < frm_bytes(B, k, N1, N2, d)) return RNN_EWORKSPACE;
   DeviceInfo* di = nullptr;
   rnn_status r = device_info(&di);
   if (r != RNN_OK) return r;
 
   FrmState st;
-  frm_layout(ws, B, k, N1, &st);
+  frm_layout(ws, B, k, N1, N2, d, &st);
   st.D1 = static_cast<const uint16_t*>(D1);
   st.D2 = static_cast<const uint16_t*>(D2);
   st.bs1 = bs1;
@@ -709,8 +742,19 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     return RNN_OK;
   }
   CUtensorMap map1, map2;
-  if ((r = make_map(&map1, D1, d, N1, B, bs1, g)) != RNN_OK) return r;
-  if ((r = make_map(&map2, D2, d, N2, B, bs2, g)) != RNN_OK) return r;
+  if (st.P1) {
+    pad_rows_kernel<<<grid_for(B * N1 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
+        static_cast<const uint16_t*>(D1), bs1, N1, B, d, st.P1, g.kpad);
+    if ((r = launched()) != RNN_OK) return r;
+    pad_rows_kernel<<<grid_for(B * N2 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
+        static_cast<const uint16_t*>(D2), bs2, N2, B, d, st.P2, g.kpad);
+    if ((r = launched()) != RNN_OK) return r;
+    if ((r = make_map(&map1, st.P1, g.kpad, N1, B, N1 * g.kpad, g)) != RNN_OK) return r;
+    if ((r = make_map(&map2, st.P2, g.kpad, N2, B, N2 * g.kpad, g)) != RNN_OK) return r;
+  } else {
+    if ((r = make_map(&map1, D1, d, N1, B, bs1, g)) != RNN_OK) return r;
+    if ((r = make_map(&map2, D2, d, N2, B, bs2, g)) != RNN_OK) return r;
+  }
 
   frm_init_kernel<<<grid_for(B * k + B * st.nwords, di->sms), kSmallThreads, 0, s>>>(st, W1, S);
   const int lgrid = grid_for(static_cast<int64_t>(B) * k * 32, di->sms);
@@ -774,7 +818,7 @@ const char* rnn_status_string(rnn_status s) {
   return "unknown rnn_status";
 }
 
-int rnn_abi_version(void) { return 1; }
+int rnn_abi_version(void) { return 2; }
 
 uint64_t rnn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -859,15 +903,30 @@ rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, i
   return launched();
 }
 
-size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2) {
+// Workspace of the reciprocal set: error word, packed keys of both sweeps,
+// block counts, and (when d < kpad) zero-padded copies of both maps.
+static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, int** err,
+                         unsigned long long** rowk, unsigned long long** colk, int** counts,
+                         uint16_t** p1, uint16_t** p2) {
+  Carve c(ws);
+  *err = c.take<int>(64);
+  *rowk = c.take<unsigned long long>(n1 > 0 ? n1 : 1);
+  *colk = c.take<unsigned long long>(n2 > 0 ? n2 : 1);
+  *counts = c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
+  const int kpad = d > 0 ? padded_depth(d) : 0;
+  *p1 = kpad != d ? c.take<uint16_t>(n1 * kpad) : nullptr;
+  *p2 = kpad != d ? c.take<uint16_t>(n2 * kpad) : nullptr;
+  return c.off;
+}
+
+size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2, int d) {
   const int64_t n1 = static_cast<int64_t>(H1 > 0 ? H1 : 0) * (W1 > 0 ? W1 : 0);
   const int64_t n2 = static_cast<int64_t>(H2 > 0 ? H2 : 0) * (W2 > 0 ? W2 : 0);
-  Carve c(nullptr);
-  c.take<int>(64);
-  c.take<unsigned long long>(n1 > 0 ? n1 : 1);
-  c.take<unsigned long long>(n2 > 0 ? n2 : 1);
-  c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
-  return c.off;
+  int* e;
+  unsigned long long *a, *b;
+  int* cnt;
+  uint16_t *p1, *p2;
+  return mnn_layout(nullptr, n1, n2, d > 0 ? d : 0, &e, &a, &b, &cnt, &p1, &p2);
 }
 
 rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, int H2, int W2,
@@ -884,25 +943,41 @@ rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, in
   if (n1 > INT32_MAX || n2 > INT32_MAX) return RNN_EINVAL;
   if (!pairs_out || !count_out) return RNN_EINVAL;
   if (cap < (n1 < n2 ? n1 : n2)) return RNN_ECAPACITY;
-  if (!workspace || !aligned256(workspace) || ws_bytes < rnn_mnn_workspace_size(H1, W1, H2, W2))
+  if (!workspace || !aligned256(workspace) ||
+      ws_bytes < rnn_mnn_workspace_size(H1, W1, H2, W2, d))
     return RNN_EWORKSPACE;
   DeviceInfo* di = nullptr;
   if ((r = device_info(&di)) != RNN_OK) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  Carve c(workspace);
-  int* err = c.take<int>(64);
-  unsigned long long* rowk = c.take<unsigned long long>(n1);
-  unsigned long long* colk = c.take<unsigned long long>(n2);
+  int* err;
+  unsigned long long *rowk, *colk;
+  int* counts;
+  uint16_t *p1, *p2;
+  mnn_layout(workspace, n1, n2, d, &err, &rowk, &colk, &counts, &p1, &p2);
   const int nblk1 = static_cast<int>((n1 + kMnnChunk - 1) / kMnnChunk);
   const int nblk2 = static_cast<int>((n2 + kMnnChunk - 1) / kMnnChunk);
-  int* counts = c.take<int>(nblk1 + 1);
 
   const Geometry g = geometry(d);
+  // tensor maps over the padded copies when d < kpad, else over the inputs
+  const void* T1 = D1;
+  const void* T2 = D2;
+  int dm = d;
+  if (p1) {
+    pad_rows_kernel<<<grid_for(n1 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
+        static_cast<const uint16_t*>(D1), n1 * d, n1, 1, d, p1, g.kpad);
+    if ((r = launched()) != RNN_OK) return r;
+    pad_rows_kernel<<<grid_for(n2 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
+        static_cast<const uint16_t*>(D2), n2 * d, n2, 1, d, p2, g.kpad);
+    if ((r = launched()) != RNN_OK) return r;
+    T1 = p1;
+    T2 = p2;
+    dm = g.kpad;
+  }
   CUtensorMap m1, m2, q1, q2;
-  if ((r = make_map(&m1, D1, d, n1, 1, n1 * d, g)) != RNN_OK) return r;
-  if ((r = make_map(&m2, D2, d, n2, 1, n2 * d, g)) != RNN_OK) return r;
-  if ((r = make_map(&q1, D1, d, n1, 1, n1 * d, g, kBlockM)) != RNN_OK) return r;
-  if ((r = make_map(&q2, D2, d, n2, 1, n2 * d, g, kBlockM)) != RNN_OK) return r;
+  if ((r = make_map(&m1, T1, dm, n1, 1, n1 * dm, g)) != RNN_OK) return r;
+  if ((r = make_map(&m2, T2, dm, n2, 1, n2 * dm, g)) != RNN_OK) return r;
+  if ((r = make_map(&q1, T1, dm, n1, 1, n1 * dm, g, kBlockM)) != RNN_OK) return r;
+  if ((r = make_map(&q2, T2, dm, n2, 1, n2 * dm, g, kBlockM)) != RNN_OK) return r;
 
   zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(rowk, n1, colk, n2, err);
   if ((r = launched()) != RNN_OK) return r;
@@ -956,11 +1031,10 @@ int64_t rnn_frm_max_pairs(int H1, int W1, int H2, int W2, int seed_stride) {
   return k < n2 ? k : n2;
 }
 
-size_t rnn_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int seed_stride) {
-  (void)H2;
-  (void)W2;
-  if (B < 1 || H1 <= 0 || W1 <= 0 || seed_stride < 1) return 0;
-  return frm_bytes(B, num_seeds(H1, W1, seed_stride), static_cast<int64_t>(H1) * W1);
+size_t rnn_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int d, int seed_stride) {
+  if (B < 1 || H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || d <= 0 || seed_stride < 1) return 0;
+  return frm_bytes(B, num_seeds(H1, W1, seed_stride), static_cast<int64_t>(H1) * W1,
+                   static_cast<int64_t>(H2) * W2, d);
 }
 
 rnn_status rnn_frm_match(const void* D1, int H1, int W1, const void* D2, int H2, int W2, int d,

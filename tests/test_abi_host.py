@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rnn_abi_version() == 1
+    assert lib.rnn_abi_version() == 2
     for code, name in _lib.STATUS.items():
         assert lib.rnn_status_string(code).decode().startswith(name)
 
@@ -58,11 +58,15 @@ def test_seed_counts_match_oracle(lib, H, W, S):
 
 def test_workspace_sizes(lib):
     assert lib.rnn_nn_workspace_size(1000) >= 1000 * 8
-    assert lib.rnn_mnn_workspace_size(384, 512, 384, 512) >= 2 * 384 * 512 * 8
-    one = lib.rnn_frm_workspace_size(1, 384, 512, 384, 512, 8)
-    many = lib.rnn_frm_workspace_size(64, 288, 512, 288, 512, 8)
+    assert lib.rnn_mnn_workspace_size(384, 512, 384, 512, 32) >= 2 * 384 * 512 * 8
+    # d = 24 is padded to 32: the workspace also holds both maps at 64 bytes a row
+    assert (lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24)
+            >= lib.rnn_mnn_workspace_size(384, 512, 384, 512, 32) + 2 * 384 * 512 * 64)
+    one = lib.rnn_frm_workspace_size(1, 384, 512, 384, 512, 32, 8)
+    many = lib.rnn_frm_workspace_size(64, 288, 512, 288, 512, 32, 8)
     assert one > 0 and many > 64 * 2304 * 8
-    assert lib.rnn_frm_workspace_size(0, 384, 512, 384, 512, 8) == 0
+    assert lib.rnn_frm_workspace_size(0, 384, 512, 384, 512, 32, 8) == 0
+    assert lib.rnn_frm_workspace_size(1, 384, 512, 384, 512, 0, 8) == 0
     for v in (one, many):
         assert v % 256 == 0
 
@@ -88,7 +92,7 @@ def test_nn_argmax_argument_errors(lib):
 
 
 def test_mnn_argument_errors(lib):
-    ws = lib.rnn_mnn_workspace_size(4, 4, 4, 4)
+    ws = lib.rnn_mnn_workspace_size(4, 4, 4, 4, 16)
     f = lib.rnn_mnn_exhaustive
 
     def call(**kw):
@@ -108,7 +112,7 @@ def test_mnn_argument_errors(lib):
 
 
 def test_frm_argument_errors(lib):
-    ws = lib.rnn_frm_workspace_size(2, 8, 8, 8, 8, 2)
+    ws = lib.rnn_frm_workspace_size(2, 8, 8, 8, 8, 16, 2)
     f = lib.rnn_frm_match_batched
 
     def call(**kw):

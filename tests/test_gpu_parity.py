@@ -257,6 +257,38 @@ def test_frm_batched_matches_oracle_per_pair():
         assert np.array_equal(q, ref.seed_queries) and np.array_equal(c, ref.seed_converged)
 
 
+def test_frm_batched_strided_padded_maps():
+    """d = 24 (copied into zero-padded 32-wide rows) with batch strides wider
+    than H*W*d, through the C ABI; every pair against the oracle."""
+    B, H, W, d, S, it = 3, 24, 40, 24, 4, 10
+    gap = 8 * 5                                   # elements between consecutive maps
+    lib = rnn._lib.load()
+    maps = [synth.quantised_pair(400 + i, H, W, H, W, d) for i in range(B)]
+    n = H * W * d
+    a = torch.zeros(B * (n + gap), dtype=torch.float16)
+    b = torch.zeros(B * (n + gap), dtype=torch.float16)
+    for i, (m1, m2) in enumerate(maps):
+        a[i * (n + gap): i * (n + gap) + n] = synth.to_storage(m1, "f16").reshape(-1)
+        b[i * (n + gap): i * (n + gap) + n] = synth.to_storage(m2, "f16").reshape(-1)
+    a, b = dev(a), dev(b)
+    k = int(lib.rnn_frm_num_seeds(H, W, S))
+    cap = int(lib.rnn_frm_max_pairs(H, W, H, W, S))
+    pairs = torch.empty((B, cap, 2), dtype=torch.int32, device="cuda")
+    count = torch.zeros(B, dtype=torch.int32, device="cuda")
+    ws = torch.empty(lib.rnn_frm_workspace_size(B, H, W, H, W, d, S), dtype=torch.uint8,
+                     device="cuda")
+    rnn._lib.check(lib.rnn_frm_match_batched(
+        B, a.data_ptr(), n + gap, b.data_ptr(), n + gap, H, W, H, W, d, 0, S, it,
+        pairs.data_ptr(), cap, count.data_ptr(), None, ws.data_ptr(), ws.numel(),
+        torch.cuda.current_stream().cuda_stream), "rnn_frm_match_batched")
+    torch.cuda.synchronize()
+    assert k > 0
+    for i, (m1, m2) in enumerate(maps):
+        ref = oracle.frm(synth.to_storage(m1, "f16"), synth.to_storage(m2, "f16"), S, it)
+        got = pairs[i, : int(count[i])].cpu().numpy()
+        assert np.array_equal(got, ref.pairs.reshape(-1, 2)), i
+
+
 def test_frm_batched_workload_sampled_pairs():
     """The 64-pair 512x288 workload in one launch sequence; two pairs checked."""
     w = synth.WORKLOADS["frm_batched_64x512x288"]
@@ -281,7 +313,7 @@ def test_repeat_runs_are_identical():
 
 def test_workspace_status_ok_after_calls():
     a = dev(synth.to_storage(synth.quantised_pair(1, 16, 16, 16, 16, 16)[0], "f16"))
-    ws = torch.empty(rnn._lib.load().rnn_frm_workspace_size(1, 16, 16, 16, 16, 2),
+    ws = torch.empty(rnn._lib.load().rnn_frm_workspace_size(1, 16, 16, 16, 16, 16, 2),
                      dtype=torch.uint8, device="cuda")
     rnn.frm_match(a, a, 2, 10, workspace=ws)
     rnn.workspace_status(ws)
