@@ -21,6 +21,10 @@ What each function computes, with its source:
   ``fast_reciprocal_NNs`` runs it (staskaer.github.io blog on DUSt3R/MASt3R,
   MASt3R matching section): grid seeds, two half-steps with their tests,
   ``max_iter`` cap, unique sorted output.
+* ``frm_ex``: the same function's other options: given start pixels (made
+  unique and sorted), the ``pixel_tol`` convergence rule that returns the
+  start pixel, the basin output, and the Euclidean-distance metric of its
+  brute-force matcher (``metric="l2"``; also for ``nn`` and ``mnn``).
 """
 from __future__ import annotations
 
@@ -72,6 +76,13 @@ def _load():
     lib.oracle_frm.argtypes = [P, i32, i32, P, i32, i32, i32, i32, i32, P, P, P, P, P, P, P,
                                P, i32]
     lib.oracle_frm.restype = ctypes.c_int64
+    lib.oracle_nn_metric.argtypes = [P, i64, P, i64, i32, i32, P, P, P, i32]
+    lib.oracle_nn_metric.restype = None
+    lib.oracle_mnn_metric.argtypes = [P, i64, P, i64, i32, i32, P, P, P, P, P, P, P, i32]
+    lib.oracle_mnn_metric.restype = ctypes.c_int64
+    lib.oracle_frm_ex.argtypes = [P, i32, i32, P, i32, i32, i32, P, i64, i32, i32,
+                                  ctypes.c_double, i32, i32, P, i64, P, P, P, P, P, P, i32]
+    lib.oracle_frm_ex.restype = ctypes.c_int64
     _lib = lib
     return lib
 
@@ -112,8 +123,13 @@ class NNResult:
         return self.best - self.second
 
 
-def nn(Q, X, threads: int = 0) -> NNResult:
-    """Nearest neighbour (largest dot product, lowest index) of each row of Q in X."""
+METRICS = {"dot": 0, "l2": 1}
+
+
+def nn(Q, X, threads: int = 0, metric: str = "dot") -> NNResult:
+    """Nearest neighbour of each row of Q in X, lowest index on ties: the
+    largest dot product, or with ``metric="l2"`` the smallest Euclidean
+    distance (``best``/``second`` are then negated squared distances)."""
     q, x = _rows(Q), _rows(X)
     assert q.shape[1] == x.shape[1]
     nq, nx, d = q.shape[0], x.shape[0], q.shape[1]
@@ -121,8 +137,8 @@ def nn(Q, X, threads: int = 0) -> NNResult:
     best = np.empty(nq, np.float64)
     second = np.empty(nq, np.float64)
     if nq:
-        _load().oracle_nn(_ptr(q), nq, _ptr(x), nx, d, _ptr(arg), _ptr(best), _ptr(second),
-                          threads)
+        _load().oracle_nn_metric(_ptr(q), nq, _ptr(x), nx, d, METRICS[metric], _ptr(arg),
+                                 _ptr(best), _ptr(second), threads)
     return NNResult(arg, best, second)
 
 
@@ -145,7 +161,7 @@ class MNNResult:
     col: NNResult        # NN1 of every D2 pixel
 
 
-def mnn(D1, D2, threads: int = 0) -> MNNResult:
+def mnn(D1, D2, threads: int = 0, metric: str = "dot") -> MNNResult:
     """The reciprocal nearest-neighbour set between two descriptor maps."""
     a, b = _rows(D1), _rows(D2)
     n1, n2, d = a.shape[0], b.shape[0], a.shape[1]
@@ -153,8 +169,9 @@ def mnn(D1, D2, threads: int = 0) -> MNNResult:
     ra, ca = np.empty(n1, np.int32), np.empty(n2, np.int32)
     rb, rs = np.empty(n1), np.empty(n1)
     cb, cs = np.empty(n2), np.empty(n2)
-    m = _load().oracle_mnn(_ptr(a), n1, _ptr(b), n2, d, _ptr(pairs), _ptr(ra), _ptr(ca),
-                           _ptr(rb), _ptr(rs), _ptr(cb), _ptr(cs), threads)
+    m = _load().oracle_mnn_metric(_ptr(a), n1, _ptr(b), n2, d, METRICS[metric], _ptr(pairs),
+                                  _ptr(ra), _ptr(ca), _ptr(rb), _ptr(rs), _ptr(cb), _ptr(cs),
+                                  threads)
     return MNNResult(pairs[:m].copy(), NNResult(ra, rb, rs), NNResult(ca, cb, cs))
 
 
@@ -200,3 +217,56 @@ def frm(D1, D2, seed_stride: int = 8, max_iter: int = 10, threads: int = 0) -> F
                            _ptr(pairs), _ptr(su), _ptr(sv), _ptr(sq), _ptr(sc), _ptr(sg),
                            _ptr(traj), _ptr(aph), threads)
     return FRMResult(pairs[:n].copy(), seeds, su, sv, sq, sc.astype(bool), sg, traj, aph)
+
+
+@dataclass
+class FRMExResult:
+    pairs: np.ndarray           # int32 [n][2], unique, sorted
+    seeds: np.ndarray           # int32 [k] start pixels, ascending
+    seed_u: np.ndarray          # int32 [k] final U
+    seed_v: np.ndarray          # int32 [k] final V
+    seed_queries: np.ndarray    # int32 [k]
+    seed_converged: np.ndarray  # bool  [k]
+    basin: np.ndarray           # int32 [H1*W1 + 1] or None
+
+
+def frm_ex(D1, D2, seed_stride: int = 8, max_iter: int = 10, init=None,
+           pixel_tol: float = 0.0, basin: bool = False, metric: str = "dot",
+           threads: int = 0) -> FRMExResult:
+    """Fast Reciprocal Matching with the quoted function's options: start
+    pixels ``init`` (linear indices; None = the grid), ``pixel_tol``, basin
+    mode, metric."""
+    a, b = as_f64(D1), as_f64(D2)
+    H1, W1, d = a.shape
+    H2, W2, d2 = b.shape
+    assert d == d2
+    a, b = a.reshape(-1, d), b.reshape(-1, d)
+    if init is not None:
+        init = np.ascontiguousarray(np.asarray(init, dtype=np.int32).reshape(-1))
+        seeds = np.unique(init)
+    else:
+        seeds = frm_seeds(H1, W1, seed_stride)
+    k = len(seeds)
+    pairs = np.empty((max(k, 1), 2), np.int32)
+    su, sv, sq = (np.empty(max(k, 1), np.int32) for _ in range(3))
+    sc = np.empty(max(k, 1), np.uint8)
+    bas = np.empty(H1 * W1 + 1, np.int32) if basin else None
+    ns = ctypes.c_int64(0)
+    n = _load().oracle_frm_ex(_ptr(a), H1, W1, _ptr(b), H2, W2, d,
+                              _ptr(init) if init is not None else None,
+                              len(init) if init is not None else 0, seed_stride, max_iter,
+                              float(pixel_tol), int(bool(basin)), METRICS[metric], _ptr(pairs),
+                              len(pairs), _ptr(su), _ptr(sv), _ptr(sq), _ptr(sc),
+                              _ptr(bas) if bas is not None else None, ctypes.byref(ns),
+                              threads)
+    assert ns.value == k
+    return FRMExResult(pairs[:n].copy(), seeds, su[:k], sv[:k], sq[:k], sc[:k].astype(bool),
+                       bas)
+
+
+def frm_refine(D1, D2, init, pixel_tol: float = 0.0, metric: str = "dot",
+               threads: int = 0) -> FRMExResult:
+    """The quoted function called with start pixels: one iteration
+    (``max_iter`` = 1), the ``pixel_tol`` rule, (start, match) pairs."""
+    return frm_ex(D1, D2, init=init, max_iter=1, pixel_tol=pixel_tol, metric=metric,
+                  threads=threads)

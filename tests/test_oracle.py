@@ -262,3 +262,152 @@ def test_workloads_have_stated_shapes():
     assert len(oracle.frm_seeds(w.H, w.W, w.seed_stride)) == 3072
     b = synth.WORKLOADS["frm_batched_64x512x288"]
     assert (b.pairs, b.H, b.W, b.occlusion) == (64, 288, 512, 0.30)
+
+
+# ------------------------------------------------- metric, start pixels, basin
+# Pins for the quoted function's other options (see oracle.frm_ex): the
+# Euclidean metric of its brute-force matcher, FRM from given start pixels
+# with the pixel tolerance, and the basin output.
+
+def _ints(D):
+    """Integer numerators k of a quantised map (values k/64)."""
+    return np.rint(np.asarray(D, dtype=np.float64).reshape(-1, np.asarray(D).shape[-1]) * 64
+                   ).astype(np.int64)
+
+
+def _nn_int(A, B, metric):
+    """Exact NN of each row of A among the rows of B (integers), first index on ties."""
+    if metric == "dot":
+        return (A @ B.T).argmax(axis=1)
+    d2 = ((A[:, None, :] - B[None, :, :]) ** 2).sum(axis=2)
+    return d2.argmin(axis=1)
+
+
+def test_golden_nn_l2_ties(golden_dir):
+    g = _load(golden_dir, "nn_l2_ties.json")
+    X, Q = np.array(g["X"], float), np.array(g["Q"], float)
+    assert oracle.nn(Q, X, metric="l2").arg.tolist() == g["l2_arg"]
+    assert oracle.nn(Q, X, metric="dot").arg.tolist() == g["dot_arg"]
+
+
+@pytest.mark.parametrize("shape", [((7, 9), (8, 6), 16), ((5, 13), (11, 3), 24),
+                                   ((16, 16), (16, 16), 8)])
+def test_l2_nn_and_mnn_match_integer_bruteforce(shape):
+    (H1, W1), (H2, W2), d = shape
+    rng = np.random.default_rng(31 + d)
+    D1 = synth.quantised_map(rng, H1, W1, d)
+    D2 = synth.quantised_map(rng, H2, W2, d)
+    A, B = _ints(D1), _ints(D2)
+    ra, ca = _nn_int(A, B, "l2"), _nn_int(B, A, "l2")
+    r = oracle.mnn(D1, D2, metric="l2")
+    assert np.array_equal(r.row.arg, ra) and np.array_equal(r.col.arg, ca)
+    mutual = [(i, int(ra[i])) for i in range(len(ra)) if ca[ra[i]] == i]
+    assert [tuple(p) for p in r.pairs.tolist()] == mutual
+    # best = -min squared distance, exact (multiples of 1/4096)
+    d2 = ((A[:, None, :] - B[None, :, :]) ** 2).sum(axis=2)
+    assert np.array_equal(-r.row.best * 4096, d2.min(axis=1).astype(np.float64))
+
+
+def test_l2_equals_dot_on_unit_vectors():
+    """For unit vectors |a-b|^2 = 2 - 2 a.b, so both metrics pick the same NN."""
+    rng = np.random.default_rng(5)
+    A = rng.standard_normal((200, 16))
+    B = rng.standard_normal((300, 16))
+    A /= np.linalg.norm(A, axis=1, keepdims=True)
+    B /= np.linalg.norm(B, axis=1, keepdims=True)
+    dot, l2 = oracle.nn(A, B), oracle.nn(A, B, metric="l2")
+    sep = dot.gap > 1e-9
+    assert sep.mean() > 0.99
+    assert np.array_equal(dot.arg[sep], l2.arg[sep])
+
+
+@pytest.mark.parametrize("case", range(5))
+def test_golden_refine(golden_dir, case):
+    g = _load(golden_dir, "frm_refine_1x3_1x2.json")
+    c = g["cases"][case]
+    D1 = np.array(g["D1"], float).reshape(g["H1"], g["W1"], g["d"])
+    D2 = np.array(g["D2"], float).reshape(g["H2"], g["W2"], g["d"])
+    r = oracle.frm_refine(D1, D2, g["init"], pixel_tol=c["pixel_tol"], metric=c["metric"])
+    assert r.seeds.tolist() == [0, 1, 2]
+    assert r.pairs.tolist() == c["pairs"]
+    assert r.seed_queries.tolist() == [2, 2, 2]
+
+
+def _refine_numpy(A, B, H1, W1, init, tol, metric):
+    """The pixel-tolerance round trip from each unique start, written out."""
+    pairs = set()
+    for u in np.unique(init):
+        v = int(_nn_int(A[u:u + 1], B, metric)[0])
+        u2 = int(_nn_int(B[v:v + 1], A, metric)[0])
+        if tol > 0:
+            conv = math.hypot(u // W1 - u2 // W1, u % W1 - u2 % W1) < tol
+        else:
+            conv = u2 == u
+        if conv:
+            pairs.add((int(u), v))
+    return sorted(pairs)
+
+
+@pytest.mark.parametrize("metric", ["dot", "l2"])
+@pytest.mark.parametrize("tol", [0.0, 1.0, 1.5, 2.3])
+def test_refine_matches_numpy_roundtrip(metric, tol):
+    rng = np.random.default_rng(77)
+    H1, W1, H2, W2, d = 9, 11, 8, 10, 16
+    D1 = synth.quantised_map(rng, H1, W1, d)
+    D2 = synth.quantised_map(rng, H2, W2, d)
+    init = rng.integers(0, H1 * W1, size=60).astype(np.int32)
+    init[5] = init[0]                                # a duplicate
+    r = oracle.frm_refine(D1, D2, init, pixel_tol=tol, metric=metric)
+    ref = _refine_numpy(_ints(D1), _ints(D2), H1, W1, init, tol, metric)
+    assert [tuple(p) for p in r.pairs.tolist()] == ref
+    assert np.array_equal(r.seeds, np.unique(init))
+
+
+@pytest.mark.parametrize("case", range(5))
+def test_golden_basin(golden_dir, case):
+    g = _load(golden_dir, "frm_basin_chain_2x2_1x4.json")
+    c = g["cases"][case]
+    D1, D2 = _chain_maps(g)
+    r = oracle.frm_ex(D1, D2, c["stride"], c["max_iter"], basin=True)
+    assert r.pairs.tolist() == c["pairs"]
+    assert r.basin.tolist() == c["basin"]
+    if "seed_queries" in c:
+        assert r.seed_queries.tolist() == c["seed_queries"]
+
+
+def _basin_numpy(A, B, seeds, max_iter):
+    """Replay of the basin-mode loop with exact integer NN queries."""
+    n1 = A.shape[0]
+    U = seeds.astype(np.int64).copy()
+    V = np.full_like(U, -1)
+    Uold = U.copy()
+    active = np.ones(len(U), bool)
+    basin = np.full(n1 + 1, -1, np.int64)
+    t = 0
+    while active.any():
+        idx = np.nonzero(active)[0]
+        V[idx] = _nn_int(A[U[idx]], B, "dot")
+        U[idx] = _nn_int(B[V[idx]], A, "dot")
+        basin[Uold[idx]] = U[idx]
+        active[idx] = U[idx] != Uold[idx]
+        t += 1
+        if t >= max_iter:
+            break
+        Uold = U.copy()
+    conv = ~active
+    pairs = sorted({(int(U[s]), int(V[s])) for s in range(len(U)) if conv[s]})
+    return pairs, basin
+
+
+@pytest.mark.parametrize("S,max_iter", [(2, 10), (3, 2), (1, 10)])
+def test_basin_matches_numpy_replay_and_plain_frm(S, max_iter):
+    rng = np.random.default_rng(90 + S)
+    H, W, d = 10, 12, 16
+    D1 = synth.quantised_map(rng, H, W, d)
+    D2 = synth.quantised_map(rng, H, W, d)
+    r = oracle.frm_ex(D1, D2, S, max_iter, basin=True)
+    pairs, basin = _basin_numpy(_ints(D1), _ints(D2), oracle.frm_seeds(H, W, S), max_iter)
+    assert [tuple(p) for p in r.pairs.tolist()] == pairs
+    assert np.array_equal(r.basin, basin)
+    # skipping the first half-step's test changes no output pair
+    assert np.array_equal(r.pairs, oracle.frm(D1, D2, S, max_iter).pairs)
