@@ -59,6 +59,20 @@ typedef enum rnn_status {
 
 typedef enum rnn_dtype { RNN_F16 = 0, RNN_BF16 = 1 } rnn_dtype;
 
+/*
+ * Meaning of "nearest" (the *_ex entry points; the others use RNN_DOT):
+ *   RNN_DOT  the largest dot product s(i, j) = sum_c D1[i][c] * D2[j][c];
+ *            for unit descriptors, as the matching head emits, this is the
+ *            nearest neighbour in Euclidean distance (cv-learn.com "MASt3R"
+ *            note, section "Method and architecture").
+ *   RNN_L2   the smallest Euclidean distance |D1_i - D2_j|, which is what the
+ *            brute-force matcher of the quoted fast_reciprocal_NNs computes
+ *            ("every distance, then the minimum"; staskaer.github.io
+ *            DUSt3R/MASt3R blog, MASt3R matching section).
+ * Ties go to the lowest index under either metric.
+ */
+typedef enum rnn_metric { RNN_DOT = 0, RNN_L2 = 1 } rnn_metric;
+
 /* Largest batch of the batched FRM entry point. */
 #define RNN_MAX_BATCH 1024
 
@@ -163,6 +177,70 @@ rnn_status rnn_frm_match_batched(int B, const void *D1, int64_t d1_batch_stride,
                                  int32_t *pairs_out, int64_t cap, int32_t *count_out,
                                  int32_t *seed_state_out, void *workspace, size_t ws_bytes,
                                  rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The same operations with every option of the quoted fast_reciprocal_NNs
+ * (staskaer.github.io DUSt3R/MASt3R blog, MASt3R matching section) and the
+ * metric.  The entry points above are these with RNN_DOT, the grid seeds,
+ * no pixel tolerance and no basin.
+ *
+ * rnn_nn_argmax_ex / rnn_mnn_exhaustive_ex: as rnn_nn_argmax /
+ * rnn_mnn_exhaustive.  With RNN_L2 the scores written (score_out, rowmax_out,
+ * colmax_out) are squared distances |q - x|^2 of the chosen neighbours.
+ * Their workspace sizes depend on the metric (the Euclidean metric keeps
+ * augmented copies of the maps in it: rows [x, -|x|^2/2 in three 16-bit
+ * parts] and [q, 1, 1, 1], whose dot product q.x - |x|^2/2 the tensor cores
+ * maximise).
+ *
+ * rnn_frm_match_ex: FRM over B pairs (as rnn_frm_match_batched) with
+ *   init_xy1     NULL: seeds on the grid of stride seed_stride (>= 1).
+ *                Else device int32 [B][n_init] start pixels y*W1 + x of each
+ *                pair; they are made unique and ascending (starts outside
+ *                the image are dropped), and seed_stride is not used.  The
+ *                quoted function runs given starts for one iteration
+ *                (max_iter = 1); any max_iter >= 1 is accepted.
+ *   pixel_tol    0: a seed is output when it is no longer active, as (U, V).
+ *                > 0 (only with init_xy1, else RNN_EINVAL): a seed is output
+ *                when its last move, from U_old to U, is shorter than
+ *                pixel_tol pixels (Euclidean distance of the row/column
+ *                positions), as (U_old, V): with one iteration, the start
+ *                pixel and its match.
+ *   basin_out    NULL, or device int32 [B][H1*W1 + 1]: basin mode.  The first
+ *                half-step then deactivates no seed, and after the second,
+ *                basin[U_old] = U for every seed it served; entries never
+ *                written are -1 (the last entry always).  The output pairs
+ *                are the same as without basin mode.
+ *   pairs_out    [B][cap][2], cap >= min(k, H2*W2), or cap >= k with a pixel
+ *                tolerance; k = n_init with given starts, else the grid size.
+ *   seed_state_out  (may be NULL) [B][k][4] per seed slot: final U, final V,
+ *                queries made, 1 if output; slots past a pair's unique starts
+ *                hold -1, -1, 0, 0.
+ * rnn_frm_workspace_size_ex takes n_init = the starts per pair, or -1 for the
+ * grid of stride seed_stride.
+ * 2 + 6*max_iter kernel launches, plus 2 (padded copies, dot metric with
+ * d = 8, 24, 40, ...) or 4 (Euclidean metric) for the row copies, plus 2 with
+ * given starts.
+ */
+size_t rnn_nn_workspace_size_ex(int64_t nq, int64_t nx, int d, rnn_metric metric);
+rnn_status rnn_nn_argmax_ex(const void *Q, int64_t nq, const void *X, int64_t nx, int d,
+                            rnn_dtype dtype, rnn_metric metric, int32_t *idx_out,
+                            float *score_out, void *workspace, size_t ws_bytes,
+                            rnn_stream_t stream);
+size_t rnn_mnn_workspace_size_ex(int H1, int W1, int H2, int W2, int d, rnn_metric metric);
+rnn_status rnn_mnn_exhaustive_ex(const void *D1, int H1, int W1, const void *D2, int H2, int W2,
+                                 int d, rnn_dtype dtype, rnn_metric metric, int32_t *pairs_out,
+                                 int64_t cap, int32_t *count_out, int32_t *rowarg_out,
+                                 float *rowmax_out, int32_t *colarg_out, float *colmax_out,
+                                 void *workspace, size_t ws_bytes, rnn_stream_t stream);
+size_t rnn_frm_workspace_size_ex(int B, int H1, int W1, int H2, int W2, int d,
+                                 rnn_metric metric, int seed_stride, int64_t n_init);
+rnn_status rnn_frm_match_ex(int B, const void *D1, int64_t d1_batch_stride, const void *D2,
+                            int64_t d2_batch_stride, int H1, int W1, int H2, int W2, int d,
+                            rnn_dtype dtype, rnn_metric metric, const int32_t *init_xy1,
+                            int64_t n_init, int seed_stride, int max_iter, float pixel_tol,
+                            int32_t *pairs_out, int64_t cap, int32_t *count_out,
+                            int32_t *seed_state_out, int32_t *basin_out, void *workspace,
+                            size_t ws_bytes, rnn_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Nearest neighbours without any allocation.  (The matching method itself

@@ -16,6 +16,11 @@ contiguous fp16/bf16 CUDA tensors; pixel index ``p = y*W + x``.
 * ``frm_match`` / ``frm_match_batched``: Fast Reciprocal Matching from grid
   seeds, with the loop of the quoted ``fast_reciprocal_NNs``
   (staskaer.github.io DUSt3R/MASt3R blog, MASt3R matching section).
+* ``frm_match_ex`` / ``frm_refine``: the same function's other options: given
+  start pixels, the pixel tolerance, the basin output.
+* ``metric="l2"`` (``nn_argmax``, ``mnn_exhaustive``, ``frm_match_ex``,
+  ``frm_refine``): the smallest Euclidean distance instead of the largest dot
+  product; scores are then squared distances.
 
 Results stay on the device; pair lists come back as ``(pairs, count)`` with
 ``pairs`` a ``[cap, 2]`` int32 buffer and ``count`` a device int32 tensor;
@@ -34,7 +39,7 @@ from ._lib import RNNError, RNNLibraryError  # noqa: F401
 __all__ = [
     "nn_argmax", "mnn_exhaustive", "frm_match", "frm_match_batched", "frm_num_seeds",
     "frm_max_pairs", "workspace_status", "trim", "MNNResult", "FRMResult", "RNNError",
-    "RNNLibraryError", "FRMPlan",
+    "RNNLibraryError", "FRMPlan", "frm_match_ex", "frm_refine",
 ]
 
 _DT = {torch.float16: _lib.RNN_F16, torch.bfloat16: _lib.RNN_BF16}
@@ -80,12 +85,19 @@ def trim(pairs: torch.Tensor, count: torch.Tensor) -> torch.Tensor:
     return pairs[: int(count.reshape(-1)[0].item())]
 
 
+def _metric(metric: str) -> int:
+    if metric not in _lib.METRICS:
+        raise ValueError(f"metric must be one of {sorted(_lib.METRICS)}, got {metric!r}")
+    return _lib.METRICS[metric]
+
+
 def nn_argmax(Q: torch.Tensor, X: torch.Tensor, *, workspace: Optional[torch.Tensor] = None,
               idx_out: Optional[torch.Tensor] = None, score_out: Optional[torch.Tensor] = None,
-              with_scores: bool = True):
+              with_scores: bool = True, metric: str = "dot"):
     """NN of each row of ``Q [nq, d]`` among the rows of ``X [nx, d]``.
 
-    Returns ``(idx int32 [nq], score float32 [nq] or None)``.
+    Returns ``(idx int32 [nq], score float32 [nq] or None)``; with
+    ``metric="l2"`` the score is the squared distance.
     """
     _check_map(Q, "Q", 2)
     _check_map(X, "X", 2)
@@ -99,12 +111,13 @@ def nn_argmax(Q: torch.Tensor, X: torch.Tensor, *, workspace: Optional[torch.Ten
         idx_out = torch.empty(nq, dtype=torch.int32, device=dev)
     if score_out is None and with_scores:
         score_out = torch.empty(nq, dtype=torch.float32, device=dev)
-    need = lib.rnn_nn_workspace_size(nq)
+    m = _metric(metric)
+    need = lib.rnn_nn_workspace_size_ex(nq, nx, d, m)
     if workspace is None:
         workspace = _workspace(need, dev)
-    _lib.check(lib.rnn_nn_argmax(Q.data_ptr(), nq, X.data_ptr(), nx, d, _dtype_code(Q),
-                                 idx_out.data_ptr(), _ptr(score_out), workspace.data_ptr(),
-                                 workspace.numel(), _stream(Q)), "rnn_nn_argmax")
+    _lib.check(lib.rnn_nn_argmax_ex(Q.data_ptr(), nq, X.data_ptr(), nx, d, _dtype_code(Q), m,
+                                    idx_out.data_ptr(), _ptr(score_out), workspace.data_ptr(),
+                                    workspace.numel(), _stream(Q)), "rnn_nn_argmax_ex")
     return idx_out, score_out
 
 
@@ -123,7 +136,7 @@ class MNNResult:
 
 def mnn_exhaustive(D1: torch.Tensor, D2: torch.Tensor, *, with_nn: bool = False,
                    workspace: Optional[torch.Tensor] = None,
-                   out: Optional[MNNResult] = None) -> MNNResult:
+                   out: Optional[MNNResult] = None, metric: str = "dot") -> MNNResult:
     """Exhaustive reciprocal NN set between ``D1 [H1, W1, d]`` and ``D2 [H2, W2, d]``."""
     _check_map(D1, "D1", 3)
     _check_map(D2, "D2", 3)
@@ -142,14 +155,15 @@ def mnn_exhaustive(D1: torch.Tensor, D2: torch.Tensor, *, with_nn: bool = False,
             out.rowmax = torch.empty(n1, dtype=torch.float32, device=dev)
             out.colarg = torch.empty(n2, dtype=torch.int32, device=dev)
             out.colmax = torch.empty(n2, dtype=torch.float32, device=dev)
-    need = lib.rnn_mnn_workspace_size(H1, W1, H2, W2, d)
+    m = _metric(metric)
+    need = lib.rnn_mnn_workspace_size_ex(H1, W1, H2, W2, d, m)
     if workspace is None:
         workspace = _workspace(need, dev)
-    _lib.check(lib.rnn_mnn_exhaustive(
-        D1.data_ptr(), H1, W1, D2.data_ptr(), H2, W2, d, _dtype_code(D1), out.pairs.data_ptr(),
-        out.pairs.shape[0], out.count.data_ptr(), _ptr(out.rowarg), _ptr(out.rowmax),
-        _ptr(out.colarg), _ptr(out.colmax), workspace.data_ptr(), workspace.numel(),
-        _stream(D1)), "rnn_mnn_exhaustive")
+    _lib.check(lib.rnn_mnn_exhaustive_ex(
+        D1.data_ptr(), H1, W1, D2.data_ptr(), H2, W2, d, _dtype_code(D1), m,
+        out.pairs.data_ptr(), out.pairs.shape[0], out.count.data_ptr(), _ptr(out.rowarg),
+        _ptr(out.rowmax), _ptr(out.colarg), _ptr(out.colmax), workspace.data_ptr(),
+        workspace.numel(), _stream(D1)), "rnn_mnn_exhaustive_ex")
     return out
 
 
@@ -166,6 +180,7 @@ class FRMResult:
     pairs: torch.Tensor                      # [B, cap, 2] int32 (B = 1 for frm_match)
     count: torch.Tensor                      # [B] int32 on the device
     seed_state: Optional[torch.Tensor] = None  # [B, k, 4]: U, V, queries, converged
+    basin: Optional[torch.Tensor] = None       # [B, H1*W1 + 1] (basin mode)
 
     def trimmed(self, b: int = 0) -> torch.Tensor:
         return self.pairs[b, : int(self.count[b].item())]
@@ -258,3 +273,68 @@ def frm_match_batched(D1: torch.Tensor, D2: torch.Tensor, seed_stride: int = 8,
     plan = FRMPlan(B, H1, W1, H2, W2, d, D1.dtype, seed_stride, max_iter, D1.device,
                    with_seed_state)
     return plan.run(D1, D2)
+
+
+def frm_match_ex(D1: torch.Tensor, D2: torch.Tensor, *, seed_stride: int = 8,
+                 max_iter: int = 10, metric: str = "dot", init: Optional[torch.Tensor] = None,
+                 pixel_tol: float = 0.0, with_basin: bool = False,
+                 with_seed_state: bool = False,
+                 workspace: Optional[torch.Tensor] = None) -> FRMResult:
+    """FRM with every option of the quoted ``fast_reciprocal_NNs``.
+
+    ``D1``/``D2`` are ``[H, W, d]`` or ``[B, H, W, d]``.  ``init`` (CUDA int32,
+    ``[n]`` or ``[B, n]``) gives the start pixels ``y*W1 + x`` instead of the
+    grid; ``pixel_tol > 0`` (only with ``init``) outputs ``(start, match)``
+    for the starts whose round trip lands closer than ``pixel_tol`` pixels;
+    ``with_basin`` returns ``basin [B, H1*W1 + 1]`` (basin[p] = the pixel a
+    round trip from p returned to, -1 if never visited).
+    """
+    batched = D1.dim() == 4
+    _check_map(D1, "D1", 4 if batched else 3)
+    _check_map(D2, "D2", 4 if batched else 3)
+    if D1.dtype != D2.dtype or D1.shape[-1] != D2.shape[-1]:
+        raise ValueError("D1 and D2 must share dtype and d")
+    if batched and D1.shape[0] != D2.shape[0]:
+        raise ValueError("D1 and D2 must share B")
+    B = D1.shape[0] if batched else 1
+    H1, W1, d = D1.shape[-3:]
+    H2, W2, _ = D2.shape[-3:]
+    lib = _lib.load()
+    m = _metric(metric)
+    dev = D1.device
+    n_init = -1
+    if init is not None:
+        if not isinstance(init, torch.Tensor) or not init.is_cuda or init.dtype != torch.int32:
+            raise ValueError("init must be a CUDA int32 tensor")
+        init = init.reshape(B, -1).contiguous()
+        n_init = init.shape[1]
+        k = n_init
+    else:
+        k = int(lib.rnn_frm_num_seeds(H1, W1, seed_stride)) if seed_stride >= 1 else 0
+    n2 = H2 * W2
+    cap = max(1, k if pixel_tol > 0 else min(k, n2))
+    out = FRMResult(torch.empty((B, cap, 2), dtype=torch.int32, device=dev),
+                    torch.zeros(B, dtype=torch.int32, device=dev),
+                    torch.empty((B, max(k, 1), 4), dtype=torch.int32, device=dev)
+                    if with_seed_state else None,
+                    torch.empty((B, H1 * W1 + 1), dtype=torch.int32, device=dev)
+                    if with_basin else None)
+    if workspace is None:
+        workspace = _workspace(lib.rnn_frm_workspace_size_ex(B, H1, W1, H2, W2, d, m,
+                                                             seed_stride, n_init), dev)
+    _lib.check(lib.rnn_frm_match_ex(
+        B, D1.data_ptr(), H1 * W1 * d, D2.data_ptr(), H2 * W2 * d, H1, W1, H2, W2, d,
+        _dtype_code(D1), m, _ptr(init), max(n_init, 0), seed_stride, max_iter,
+        float(pixel_tol), out.pairs.data_ptr(), cap, out.count.data_ptr(),
+        _ptr(out.seed_state), _ptr(out.basin), workspace.data_ptr(), workspace.numel(),
+        _stream(D1)), "rnn_frm_match_ex")
+    return out
+
+
+def frm_refine(D1: torch.Tensor, D2: torch.Tensor, init: torch.Tensor, pixel_tol: float = 0.0,
+               *, metric: str = "dot", with_seed_state: bool = False) -> FRMResult:
+    """The quoted function called with start pixels: one round trip from each
+    unique start, ``(start, match)`` pairs for the starts that come back
+    (exactly, or within ``pixel_tol`` pixels)."""
+    return frm_match_ex(D1, D2, max_iter=1, metric=metric, init=init, pixel_tol=pixel_tol,
+                        with_seed_state=with_seed_state)

@@ -28,6 +28,12 @@ EXPORTS = (
     "rnn_launch_count",
     "rnn_set_kernel_timer",
     "rnn_nn_argmax_noalloc",
+    "rnn_nn_workspace_size_ex",
+    "rnn_nn_argmax_ex",
+    "rnn_mnn_workspace_size_ex",
+    "rnn_mnn_exhaustive_ex",
+    "rnn_frm_workspace_size_ex",
+    "rnn_frm_match_ex",
 )
 
 STATUS = {
@@ -35,6 +41,8 @@ STATUS = {
     5: "RNN_ETIMEOUT", 6: "RNN_EUNSUPPORTED", 7: "RNN_EWORKSPACE",
 }
 RNN_F16, RNN_BF16 = 0, 1
+RNN_DOT, RNN_L2 = 0, 1
+METRICS = {"dot": RNN_DOT, "l2": RNN_L2}
 RNN_MAX_BATCH = 1024
 RNN_NN_NOALLOC_MAX_QUERIES = 65536
 
@@ -84,6 +92,14 @@ def load():
         "rnn_launch_count": (ctypes.c_uint64, []),
         "rnn_set_kernel_timer": (None, [P, P, I, P]),
         "rnn_nn_argmax_noalloc": (I, [P, I64, P, I64, I, I, P, P, P]),
+        "rnn_nn_workspace_size_ex": (SZ, [I64, I64, I, I]),
+        "rnn_nn_argmax_ex": (I, [P, I64, P, I64, I, I, I, P, P, P, SZ, P]),
+        "rnn_mnn_workspace_size_ex": (SZ, [I, I, I, I, I, I]),
+        "rnn_mnn_exhaustive_ex": (I, [P, I, I, P, I, I, I, I, I, P, I64, P, P, P, P, P, P, SZ,
+                                      P]),
+        "rnn_frm_workspace_size_ex": (SZ, [I, I, I, I, I, I, I, I, I64]),
+        "rnn_frm_match_ex": (I, [I, P, I64, P, I64, I, I, I, I, I, I, I, P, I64, I, I,
+                                 ctypes.c_float, P, I64, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

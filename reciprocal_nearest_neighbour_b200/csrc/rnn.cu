@@ -263,6 +263,7 @@ static rnn_status check_desc(const void* p, int d) {
 }
 
 static bool valid_dtype(rnn_dtype dt) { return dt == RNN_F16 || dt == RNN_BF16; }
+static bool valid_metric(rnn_metric m) { return m == RNN_DOT || m == RNN_L2; }
 
 // -------------------------------------------------------------- small kernels
 __global__ void zero_keys_kernel(unsigned long long* a, int64_t na, unsigned long long* b,
@@ -275,26 +276,70 @@ __global__ void zero_keys_kernel(unsigned long long* a, int64_t na, unsigned lon
   if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
 }
 
-// Copy [nbatch][rows][d] descriptors (batch stride `bstride` elements) into
-// [nbatch][rows][kpad] rows padded with zeros.  The fused kernel's candidate
-// tiles are K = kpad wide; when d < kpad (d = 8, 24, 40, ...) a tensor map
-// over the caller's d-wide rows would zero-fill part of every box and fetch
-// rows that straddle L2 sectors, which costs the d = 24 sweep about a fifth
-// of its time.  The zeros add nothing to any dot product.
-__global__ void pad_rows_kernel(const uint16_t* src, int64_t bstride, int64_t rows, int nbatch,
-                                int d, uint16_t* dst, int kpad) {
-  const int cpr = kpad / 8, creal = d / 8;  // 16-byte chunks per padded / real row
-  const int64_t total = static_cast<int64_t>(nbatch) * rows * cpr;
+// Row forms the fused kernel reads (all [nbatch][rows][kpad], zero beyond
+// the written columns):
+//   kFormPad    the d channels (d < kpad happens for d = 8, 24, 40, ...: over
+//               the caller's d-wide rows every box would zero-fill part of
+//               itself and fetch rows straddling L2 sectors, which costs the
+//               d = 24 sweep about a fifth of its time);
+//   kFormQuery  the channels, then 1, 1, 1 (Euclidean metric, query side);
+//   kFormCand   the channels, then c1, c2, c3 with c1 + c2 + c3 = -|x|^2/2
+//               (Euclidean metric, candidate side).
+// With both augmented forms the tensor cores compute q.x - |x|^2/2 =
+// (|q|^2 - |q - x|^2)/2, whose largest value over x is the nearest x.
+// |x|^2 is summed in fp32 from exact products and split into three 16-bit
+// parts; on k/64 inputs every part and every partial sum is a multiple of
+// 2^-13 well inside fp32's range, so the augmented score stays exact.
+constexpr int kFormPad = 0, kFormQuery = 1, kFormCand = 2;
+constexpr int kAugCols = 3;  // extra columns of the Euclidean forms
+
+__device__ __forceinline__ float bits_to_f(uint16_t h, bool bf16) {
+  return bf16 ? __bfloat162float(__ushort_as_bfloat16(h)) : __half2float(__ushort_as_half(h));
+}
+__device__ __forceinline__ uint16_t f_to_bits(float x, bool bf16) {
+  return bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(x))
+              : __half_as_ushort(__float2half_rn(x));
+}
+
+template <bool kBf16>
+__global__ void prep_rows_kernel(const uint16_t* src, int64_t bstride, int64_t rows, int nbatch,
+                                 int d, uint16_t* dst, int kpad, int form) {
+  const int64_t total = static_cast<int64_t>(nbatch) * rows;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += stride) {
-    const int64_t rr = i / cpr;  // row over all batches
-    const int c = static_cast<int>(i - rr * cpr);
+  for (int64_t rr = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; rr < total;
+       rr += stride) {
     const int64_t b = rr / rows, r = rr - b * rows;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (c < creal)
-      v = __ldg(reinterpret_cast<const uint4*>(src + b * bstride + r * d) + c);
-    reinterpret_cast<uint4*>(dst)[i] = v;
+    const uint4* in = reinterpret_cast<const uint4*>(src + b * bstride + r * d);
+    uint4* out = reinterpret_cast<uint4*>(dst + rr * kpad);
+    float n2 = 0.f;
+    for (int c = 0; c < d / 8; ++c) {
+      const uint4 v = __ldg(in + c);
+      out[c] = v;
+      if (form == kFormCand) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float lo = bits_to_f(static_cast<uint16_t>(w[e] & 0xFFFFu), kBf16);
+          const float hi = bits_to_f(static_cast<uint16_t>(w[e] >> 16), kBf16);
+          n2 = fmaf(lo, lo, n2);
+          n2 = fmaf(hi, hi, n2);
+        }
+      }
+    }
+    // columns d .. kpad-1: the augmentation (if any), then zeros
+    uint16_t aug[kAugCols] = {0, 0, 0};
+    if (form == kFormQuery) {
+      aug[0] = aug[1] = aug[2] = f_to_bits(1.0f, kBf16);
+    } else if (form == kFormCand) {
+      float v = -0.5f * n2;
+#pragma unroll
+      for (int e = 0; e < kAugCols; ++e) {
+        aug[e] = f_to_bits(v, kBf16);
+        v -= bits_to_f(aug[e], kBf16);
+      }
+    }
+    uint16_t* tail = dst + rr * kpad + d;
+    for (int c = 0; c < kpad - d; ++c) tail[c] = c < kAugCols && form != kFormPad ? aug[c] : 0;
   }
 }
 
@@ -332,40 +377,62 @@ __device__ __forceinline__ float dot_rows(const uint16_t* a, const uint16_t* b, 
 
 template <bool kBf16>
 __device__ __forceinline__ int locate_chunk(const uint16_t* q, const uint16_t* X, int n_cand,
-                                            int d, int c0) {
+                                            int ld, int c0, float* best = nullptr) {
   const int lane = threadIdx.x & 31;
   const int j = c0 + lane;
   float sc = -__int_as_float(0x7f800000);
-  if (j < n_cand) sc = dot_rows<kBf16>(q, X + static_cast<int64_t>(j) * d, d);
+  if (j < n_cand) sc = dot_rows<kBf16>(q, X + static_cast<int64_t>(j) * ld, ld);
   float m = sc;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   const unsigned hit = __ballot_sync(0xffffffffu, sc == m);
+  if (best) *best = m;
   return c0 + __ffs(hit) - 1;
 }
 
+// |q|^2 over the first d channels of a row, in fp32 (exact products).
+template <bool kBf16>
+__device__ __forceinline__ float sqnorm_row(const uint16_t* q, int d) {
+  return dot_rows<kBf16>(q, q, d);
+}
+
+// Score a caller sees: the dot product, or with the Euclidean forms the
+// squared distance |q|^2 - 2 (q.x - |x|^2/2) of the located candidate.
+template <bool kBf16>
+__device__ __forceinline__ float reported_score(const uint16_t* q, int d, bool l2, float key_s,
+                                                float located_s) {
+  return l2 ? sqnorm_row<kBf16>(q, d) - 2.f * located_s : key_s;
+}
+
 // nn_argmax results: locate every query's index, write index and score.
+// Q and X rows are ld elements apart (the caller's rows, or their forms).
 template <bool kBf16>
 __global__ void locate_unpack_kernel(const unsigned long long* keys, int64_t n, const uint16_t* Q,
-                                     const uint16_t* X, int nx, int d, int32_t* idx,
-                                     float* score) {
+                                     const uint16_t* X, int nx, int ld, int d, int l2,
+                                     int32_t* idx, float* score) {
   const int64_t w0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t i = w0; i < n; i += nw) {
     const unsigned long long k = keys[i];
-    const int j = locate_chunk<kBf16>(Q + i * d, X, nx, d, key_index(k));
+    const uint16_t* q = Q + i * ld;
+    float m;
+    const int j = locate_chunk<kBf16>(q, X, nx, ld, key_index(k), &m);
+    const float sc = reported_score<kBf16>(q, d, l2 != 0, key_score(k), m);
     if ((threadIdx.x & 31) == 0) {
       idx[i] = j;
-      if (score) score[i] = key_score(k);
+      if (score) score[i] = sc;
     }
   }
 }
 
 // Both sweeps of the reciprocal set: rewrite each packed key with its exact
-// index (rows of D1 against D2, then rows of D2 against D1).
+// index and the reported score (rows of image 1, Q1, against the candidates
+// of image 2, X2; then rows of image 2, Q2, against X1).
 template <bool kBf16>
 __global__ void locate_mnn_kernel(unsigned long long* rowk, int64_t n1, unsigned long long* colk,
-                                  int64_t n2, const uint16_t* D1, const uint16_t* D2, int d) {
+                                  int64_t n2, const uint16_t* Q1, const uint16_t* X1,
+                                  const uint16_t* Q2, const uint16_t* X2, int ld, int d,
+                                  int l2) {
   const int64_t w0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   for (int64_t i = w0; i < n1 + n2; i += nw) {
@@ -373,9 +440,12 @@ __global__ void locate_mnn_kernel(unsigned long long* rowk, int64_t n1, unsigned
     const int64_t r = row ? i : i - n1;
     unsigned long long* kp = row ? rowk + r : colk + r;
     const unsigned long long k = *kp;
-    const int j = row ? locate_chunk<kBf16>(D1 + r * d, D2, static_cast<int>(n2), d, key_index(k))
-                      : locate_chunk<kBf16>(D2 + r * d, D1, static_cast<int>(n1), d, key_index(k));
-    if ((threadIdx.x & 31) == 0) *kp = pack_key(key_score(k), j);
+    const uint16_t* q = (row ? Q1 : Q2) + r * ld;
+    float m;
+    const int j = row ? locate_chunk<kBf16>(q, X2, static_cast<int>(n2), ld, key_index(k), &m)
+                      : locate_chunk<kBf16>(q, X1, static_cast<int>(n1), ld, key_index(k), &m);
+    const float sc = reported_score<kBf16>(q, d, l2 != 0, key_score(k), m);
+    if ((threadIdx.x & 31) == 0) *kp = pack_key(sc, j);
   }
 }
 
@@ -485,9 +555,14 @@ __global__ void mnn_write_kernel(const unsigned long long* rowk, int64_t n1,
 }
 
 // ------------------------------------------------------------------- FRM
+// Options of the quoted fast_reciprocal_NNs (staskaer.github.io DUSt3R/MASt3R
+// blog, MASt3R matching section) besides the grid stride: given start pixels
+// (made unique and ascending), the pixel tolerance rule, the basin output;
+// and the metric of its brute-force matcher.
 struct FrmState {
   int* err;
   int32_t* count;   // [B] active seeds
+  int32_t* nseeds;  // [B] seeds of each pair: the grid size, or its unique starts
   int32_t* U;       // [B][k]
   int32_t* V;
   int32_t* Uold;
@@ -496,81 +571,192 @@ struct FrmState {
   int32_t* nq;      // [B][k] queries made per seed
   uint8_t* act;     // [B][k] 1 while active
   unsigned long long* keys;  // [B][k] NN result per list position
-  uint32_t* bitmap; // [B][nwords] converged image-1 pixels
-  int32_t* partner; // [B][N1] image-2 partner of a converged pixel
-  const uint16_t* D1;  // descriptor maps (for the locate pass), pair b at D1 + b*bs1
-  const uint16_t* D2;
-  uint16_t* P1;        // zero-padded copies [B][N][kpad] for the tensor maps, when d < kpad
-  uint16_t* P2;
-  int64_t bs1, bs2;
-  int B, k, N1, N2, nwords, d;
+  uint32_t* bitmap; // [B][nwords]: the start set, then the output pixels
+  int32_t* partner; // [B][N1] image-2 partner of an output pixel
+  int32_t* basin;   // [B][N1 + 1] or null (basin mode)
+  // row forms (see prep_rows_kernel) read by the query gather and the locate
+  // pass: Q* query side, X* candidate side; pair b at base + b*s1 (image 1)
+  // or b*s2 (image 2), rows of ld elements
+  const uint16_t* Q1;
+  const uint16_t* Q2;
+  const uint16_t* X1;
+  const uint16_t* X2;
+  int64_t s1, s2;
+  int ld;
+  float pixel_tol;  // > 0: converged when the move from U_old is below it
+  int starts;       // 1: the seeds were given (output U_old with pixel_tol)
+  int B, k, N1, N2, nwords;
+};
+
+// Row-form copies a call needs: none, one padded copy per map (dot metric,
+// d short of the K-block layout), or a query and a candidate form per map
+// (Euclidean metric).
+enum { kCopiesNone = 0, kCopiesPad = 1, kCopiesEuclid = 2 };
+
+static int copies_for(int d, rnn_metric metric) {
+  if (metric == RNN_L2) return kCopiesEuclid;
+  return padded_depth(d) != d ? kCopiesPad : kCopiesNone;
+}
+
+// K of the tensor-core tiles: the channels, plus the Euclidean augmentation.
+static int tile_depth(int d, rnn_metric metric) {
+  return padded_depth(d + (metric == RNN_L2 ? kAugCols : 0));
+}
+
+struct FrmCopies {
+  uint16_t *q1, *x1, *q2, *x2;  // null when not needed (x* alias q* with kCopiesPad)
 };
 
 // Workspace layout of a batched FRM call; returns the bytes it needs.
 static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int d,
-                         FrmState* st) {
+                         rnn_metric metric, FrmState* st, FrmCopies* cp) {
   Carve c(ws);
   st->err = c.take<int>(64);
   st->count = c.take<int32_t>(B);
-  st->U = c.take<int32_t>(B * k);
-  st->V = c.take<int32_t>(B * k);
-  st->Uold = c.take<int32_t>(B * k);
-  st->Vold = c.take<int32_t>(B * k);
-  st->list = c.take<int32_t>(B * k);
-  st->nq = c.take<int32_t>(B * k);
-  st->act = c.take<uint8_t>(B * k);
-  st->keys = c.take<unsigned long long>(B * k);
+  st->nseeds = c.take<int32_t>(B);
+  const int64_t kk = k > 0 ? k : 1;
+  st->U = c.take<int32_t>(B * kk);
+  st->V = c.take<int32_t>(B * kk);
+  st->Uold = c.take<int32_t>(B * kk);
+  st->Vold = c.take<int32_t>(B * kk);
+  st->list = c.take<int32_t>(B * kk);
+  st->nq = c.take<int32_t>(B * kk);
+  st->act = c.take<uint8_t>(B * kk);
+  st->keys = c.take<unsigned long long>(B * kk);
   const int64_t nwords = (N1 + 31) / 32;
   st->bitmap = c.take<uint32_t>(B * nwords);
   st->partner = c.take<int32_t>(B * N1);
-  const int kpad = padded_depth(d);
-  st->P1 = kpad != d ? c.take<uint16_t>(B * N1 * kpad) : nullptr;
-  st->P2 = kpad != d ? c.take<uint16_t>(B * N2 * kpad) : nullptr;
+  const int mode = copies_for(d, metric);
+  const int kpad = tile_depth(d, metric);
+  cp->q1 = cp->x1 = cp->q2 = cp->x2 = nullptr;
+  if (mode != kCopiesNone) {
+    cp->q1 = c.take<uint16_t>(B * N1 * kpad);
+    cp->q2 = c.take<uint16_t>(B * N2 * kpad);
+    cp->x1 = cp->q1;
+    cp->x2 = cp->q2;
+    if (mode == kCopiesEuclid) {
+      cp->x1 = c.take<uint16_t>(B * N1 * kpad);
+      cp->x2 = c.take<uint16_t>(B * N2 * kpad);
+    }
+  }
   st->B = B;
   st->k = static_cast<int>(k);
   st->N1 = static_cast<int>(N1);
+  st->N2 = static_cast<int>(N2);
   st->nwords = static_cast<int>(nwords);
+  st->basin = nullptr;
   return c.off;
 }
 
-static size_t frm_bytes(int B, int64_t k, int64_t N1, int64_t N2, int d) {
+static size_t frm_bytes(int B, int64_t k, int64_t N1, int64_t N2, int d, rnn_metric metric) {
   FrmState st;
-  return frm_layout(nullptr, B, k, N1, N2, d, &st);
+  FrmCopies cp;
+  return frm_layout(nullptr, B, k, N1, N2, d, metric, &st, &cp);
 }
 
+// Per-seed state of slot s holding pixel u (u < 0: an unused slot).
+__device__ __forceinline__ void frm_seed_init(const FrmState& st, int64_t t, int s, int32_t u) {
+  st.U[t] = u;
+  st.Uold[t] = u;
+  st.V[t] = -1;
+  st.Vold[t] = -1;
+  st.list[t] = s;
+  st.nq[t] = 0;
+  st.act[t] = u >= 0 ? 1 : 0;
+  st.keys[t] = 0ull;
+}
+
+// Grid seeds (stride S), the converged-pixel bitmap, the basin array.
 __global__ void frm_init_kernel(FrmState st, int W1, int S) {
   const int x0 = S / 2;
   const int nx = W1 > x0 ? (W1 - x0 + S - 1) / S : 0;
   const int64_t nseed = static_cast<int64_t>(st.B) * st.k;
   const int64_t nbits = static_cast<int64_t>(st.B) * st.nwords;
+  const int64_t nbasin = st.basin ? static_cast<int64_t>(st.B) * (st.N1 + 1) : 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-       t < nseed + nbits; t += stride) {
+       t < nseed + nbits + nbasin; t += stride) {
     if (t < nseed) {
       const int s = static_cast<int>(t % st.k);
       const int iy = s / nx, ix = s - (s / nx) * nx;
-      const int32_t u = (x0 + iy * S) * W1 + (x0 + ix * S);
-      st.U[t] = u;
-      st.Uold[t] = u;
-      st.V[t] = -1;
-      st.Vold[t] = -1;
-      st.list[t] = s;
-      st.nq[t] = 0;
-      st.act[t] = 1;
-      st.keys[t] = 0ull;
-    } else {
+      frm_seed_init(st, t, s, (x0 + iy * S) * W1 + (x0 + ix * S));
+    } else if (t < nseed + nbits) {
       st.bitmap[t - nseed] = 0u;
+    } else {
+      st.basin[t - nseed - nbits] = -1;
     }
   }
   if (blockIdx.x == 0) {
-    for (int b = threadIdx.x; b < st.B; b += blockDim.x) st.count[b] = st.k;
+    for (int b = threadIdx.x; b < st.B; b += blockDim.x) {
+      st.count[b] = st.k;
+      st.nseeds[b] = st.k;
+    }
     if (threadIdx.x == 0) *st.err = 0;
   }
 }
 
+// Given start pixels, step 1: clear the bitmaps and the basin array.
+__global__ void frm_starts_clear_kernel(FrmState st) {
+  const int64_t nbits = static_cast<int64_t>(st.B) * st.nwords;
+  const int64_t nbasin = st.basin ? static_cast<int64_t>(st.B) * (st.N1 + 1) : 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+       t < nbits + nbasin; t += stride) {
+    if (t < nbits) st.bitmap[t] = 0u;
+    else st.basin[t - nbits] = -1;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *st.err = 0;
+}
+
+// Step 2: mark every start in its pair's bitmap (starts outside the image
+// are ignored), which makes them unique.
+__global__ void frm_starts_mark_kernel(FrmState st, const int32_t* init, int64_t n_init) {
+  const int64_t n = static_cast<int64_t>(st.B) * n_init;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < n;
+       t += stride) {
+    const int64_t b = t / n_init;
+    const int32_t u = init[t];
+    if (u >= 0 && u < st.N1)
+      atomicOr(st.bitmap + b * st.nwords + (u >> 5), 1u << (u & 31));
+  }
+}
+
+// Step 3 (one CTA per pair): the marked pixels in increasing order become
+// the seeds; the bitmap is cleared again for the merge.
+__global__ void frm_starts_compact_kernel(FrmState st) {
+  const int b = blockIdx.x;
+  uint32_t* bm = st.bitmap + static_cast<int64_t>(b) * st.nwords;
+  const int per = (st.nwords + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * per;
+  const int w1 = min(st.nwords, w0 + per);
+  int c = 0;
+  for (int w = w0; w < w1; ++w) c += __popc(bm[w]);
+  int tot;
+  int pos = block_exclusive_scan(c, &tot);
+  const int64_t base = static_cast<int64_t>(b) * st.k;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = bm[w];
+    bm[w] = 0u;
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      frm_seed_init(st, base + pos, pos, w * 32 + bit);
+      ++pos;
+    }
+  }
+  // unused slots (duplicated or out-of-image starts)
+  for (int s = tot + threadIdx.x; s < st.k; s += blockDim.x) frm_seed_init(st, base + s, s, -1);
+  if (threadIdx.x == 0) {
+    st.count[b] = tot;
+    st.nseeds[b] = tot;
+  }
+}
+
 // Exact index inside each kept chunk for every active seed of every pair
-// (one warp per seed): NN2 queries are rows U of D1 against D2, NN1 queries
-// rows V of D2 against D1.
+// (one warp per seed): NN2 queries are rows U of image 1 against image 2,
+// NN1 queries rows V of image 2 against image 1, in the row forms the
+// tensor cores read.
 template <bool kBf16>
 __global__ void frm_locate_kernel(FrmState st, int nn2_half) {
   const int64_t w0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -582,24 +768,27 @@ __global__ void frm_locate_kernel(FrmState st, int nn2_half) {
     const int i = static_cast<int>(x - static_cast<int64_t>(b) * st.k);
     if (i >= st.count[b]) continue;
     const int64_t base = static_cast<int64_t>(b) * st.k;
-    const uint16_t* Dq = nn2_half ? st.D1 + b * st.bs1 : st.D2 + b * st.bs2;
-    const uint16_t* Dx = nn2_half ? st.D2 + b * st.bs2 : st.D1 + b * st.bs1;
+    const uint16_t* Dq = nn2_half ? st.Q1 + b * st.s1 : st.Q2 + b * st.s2;
+    const uint16_t* Dx = nn2_half ? st.X2 + b * st.s2 : st.X1 + b * st.s1;
     const int sl = st.list[base + i];
     const unsigned long long k = st.keys[base + i];
     const int64_t qr = rows[base + sl];
-    const int j = locate_chunk<kBf16>(Dq + qr * st.d, Dx, n_cand, st.d, key_index(k));
+    const int j = locate_chunk<kBf16>(Dq + qr * st.ld, Dx, n_cand, st.ld, key_index(k));
     if ((threadIdx.x & 31) == 0) st.keys[base + i] = pack_key(key_score(k), j);
   }
 }
 
 // Result of one half-step for pair blockIdx.x: store the NN found for every
 // active seed, apply the convergence test, refresh the old copies at the end
-// of an iteration, and compact the list of seeds that stay active.
+// of an iteration, and compact the list of seeds that stay active.  In basin
+// mode the NN2 half-step deactivates no one and the NN1 half-step records
+// basin[U_old] = U for every seed it served.
 __global__ void frm_update_kernel(FrmState st, int nn2_half, int last_iter) {
   __shared__ int s_out;
   const int b = blockIdx.x;
   const int64_t base = static_cast<int64_t>(b) * st.k;
   const int n = st.count[b];
+  int32_t* basin = st.basin ? st.basin + static_cast<int64_t>(b) * (st.N1 + 1) : nullptr;
   if (threadIdx.x == 0) s_out = 0;
   __syncthreads();
   for (int i0 = 0; i0 < n; i0 += blockDim.x) {
@@ -613,9 +802,10 @@ __global__ void frm_update_kernel(FrmState st, int nn2_half, int last_iter) {
       st.nq[base + s] += 1;
       if (nn2_half) {
         st.V[base + s] = j;
-        still = j != st.Vold[base + s];
+        still = basin ? 1 : j != st.Vold[base + s];
       } else {
         st.U[base + s] = j;
+        if (basin) basin[st.Uold[base + s]] = j;
         still = j != st.Uold[base + s];
         if (still && !last_iter) {
           st.Uold[base + s] = j;
@@ -634,25 +824,46 @@ __global__ void frm_update_kernel(FrmState st, int nn2_half, int last_iter) {
   if (threadIdx.x == 0) st.count[b] = s_out;
 }
 
-// Unique converged pairs of pair blockIdx.x, sorted by the image-1 pixel.
-__global__ void frm_merge_kernel(FrmState st, int32_t* pairs, int64_t cap, int32_t* count_out,
-                                 int32_t* seed_state) {
+// Unique output pairs of pair blockIdx.x, sorted by the image-1 pixel.  A
+// seed is in the output when it is no longer active, or, with a pixel
+// tolerance, when its last move (U_old -> U) is shorter than the tolerance;
+// the pair is (U, V), or (U_old, V) with a tolerance and given starts.  An
+// output pixel determines its partner (a mutual pair, or a start's match),
+// so a bitmap over image 1 de-duplicates and sorts.
+__global__ void frm_merge_kernel(FrmState st, int W1, int32_t* pairs, int64_t cap,
+                                 int32_t* count_out, int32_t* seed_state) {
   const int b = blockIdx.x;
   const int64_t base = static_cast<int64_t>(b) * st.k;
+  const int ns = st.nseeds[b];
   uint32_t* bm = st.bitmap + static_cast<int64_t>(b) * st.nwords;
   int32_t* partner = st.partner + static_cast<int64_t>(b) * st.N1;
   for (int s = threadIdx.x; s < st.k; s += blockDim.x) {
-    const int conv = st.act[base + s] == 0;
-    const int32_t u = st.U[base + s], v = st.V[base + s];
-    if (conv) {
-      atomicOr(bm + (u >> 5), 1u << (u & 31));
-      partner[u] = v;
+    int conv = 0;
+    int32_t u = -1, v = -1;
+    if (s < ns) {
+      u = st.U[base + s];
+      v = st.V[base + s];
+      int32_t uo = u;
+      if (st.pixel_tol > 0.f) {
+        const int32_t u0 = st.Uold[base + s];
+        // in double, as the distance is written down
+        const double dy = static_cast<double>(u0 / W1 - u / W1);
+        const double dx = static_cast<double>(u0 % W1 - u % W1);
+        conv = sqrt(dy * dy + dx * dx) < static_cast<double>(st.pixel_tol);
+        if (st.starts) uo = u0;
+      } else {
+        conv = st.act[base + s] == 0;
+      }
+      if (conv) {
+        atomicOr(bm + (uo >> 5), 1u << (uo & 31));
+        partner[uo] = v;
+      }
     }
     if (seed_state) {
       int32_t* o = seed_state + (base + s) * 4;
       o[0] = u;
       o[1] = v;
-      o[2] = st.nq[base + s];
+      o[2] = s < ns ? st.nq[base + s] : 0;
       o[3] = conv;
     }
   }
@@ -702,68 +913,119 @@ static int64_t num_seeds(int H, int W, int S) {
   return ny * nx;
 }
 
+// One launch of the row-form preparation over [nbatch][rows][d] maps.
+static rnn_status prep_rows(const void* src, int64_t bstride, int64_t rows, int nbatch, int d,
+                            uint16_t* dst, int kpad, int form, rnn_dtype dt, DeviceInfo* di,
+                            cudaStream_t s) {
+  const int grid = grid_for(static_cast<int64_t>(nbatch) * rows, di->sms);
+  const uint16_t* in = static_cast<const uint16_t*>(src);
+  if (dt == RNN_BF16)
+    prep_rows_kernel<true><<<grid, kSmallThreads, 0, s>>>(in, bstride, rows, nbatch, d, dst,
+                                                         kpad, form);
+  else
+    prep_rows_kernel<false><<<grid, kSmallThreads, 0, s>>>(in, bstride, rows, nbatch, d, dst,
+                                                          kpad, form);
+  return launched();
+}
+
+// The FRM loop over B pairs with every option; frm entry points call it.
 static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, int64_t bs2, int H1,
-                          int W1, int H2, int W2, int d, rnn_dtype dt, int S, int max_iter,
-                          int32_t* pairs, int64_t cap, int32_t* count_out, int32_t* seed_state,
-                          void* ws, size_t ws_bytes, cudaStream_t s) {
+                          int W1, int H2, int W2, int d, rnn_dtype dt, rnn_metric metric,
+                          const int32_t* init, int64_t n_init, int S, int max_iter,
+                          float pixel_tol, int32_t* pairs, int64_t cap, int32_t* count_out,
+                          int32_t* seed_state, int32_t* basin, void* ws, size_t ws_bytes,
+                          cudaStream_t s) {
   if (B < 1) return RNN_EINVAL;
   if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
-  if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || S < 1 || max_iter < 1) return RNN_EINVAL;
-  if (!valid_dtype(dt)) return RNN_EINVAL;
+  if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || max_iter < 1) return RNN_EINVAL;
+  if (!valid_dtype(dt) || !valid_metric(metric)) return RNN_EINVAL;
+  if (init ? n_init < 0 : S < 1) return RNN_EINVAL;
+  if (!(pixel_tol >= 0.f) || (pixel_tol > 0.f && !init)) return RNN_EINVAL;
   rnn_status st0 = check_desc(D1, d);
   if (st0 != RNN_OK) return st0;
   st0 = check_desc(D2, d);
   if (st0 != RNN_OK) return st0;
   const int64_t N1 = static_cast<int64_t>(H1) * W1, N2 = static_cast<int64_t>(H2) * W2;
-  if (N1 > INT32_MAX || N2 > INT32_MAX) return RNN_EINVAL;
+  if (N1 >= INT32_MAX || N2 > INT32_MAX) return RNN_EINVAL;
   if (bs1 < N1 * d || bs2 < N2 * d || bs1 % 8 != 0 || bs2 % 8 != 0) return RNN_EINVAL;
   if (!pairs || !count_out) return RNN_EINVAL;
-  const int64_t k = num_seeds(H1, W1, S);
-  const int64_t need = k < N2 ? k : N2;
+  const int64_t k = init ? n_init : num_seeds(H1, W1, S);
+  if (k > INT32_MAX) return RNN_EINVAL;
+  // outputs are mutual pairs (distinct V), except (start, match) pairs under
+  // a pixel tolerance, where only the starts are distinct
+  const int64_t need = pixel_tol > 0.f ? k : (k < N2 ? k : N2);
   if (cap < need) return RNN_ECAPACITY;
-  if (!ws || !aligned256(ws) || ws_bytes < frm_bytes(B, k, N1, N2, d)) return RNN_EWORKSPACE;
+  if (!ws || !aligned256(ws) || ws_bytes < frm_bytes(B, k, N1, N2, d, metric))
+    return RNN_EWORKSPACE;
   DeviceInfo* di = nullptr;
   rnn_status r = device_info(&di);
   if (r != RNN_OK) return r;
 
   FrmState st;
-  frm_layout(ws, B, k, N1, N2, d, &st);
-  st.D1 = static_cast<const uint16_t*>(D1);
-  st.D2 = static_cast<const uint16_t*>(D2);
-  st.bs1 = bs1;
-  st.bs2 = bs2;
-  st.N2 = static_cast<int>(N2);
-  st.d = d;
-  const Geometry g = geometry(d);
+  FrmCopies cp;
+  frm_layout(ws, B, k, N1, N2, d, metric, &st, &cp);
+  st.basin = basin;
+  st.pixel_tol = pixel_tol;
+  st.starts = init ? 1 : 0;
+  const Geometry g = geometry(d + (metric == RNN_L2 ? kAugCols : 0));
+  const int mode = copies_for(d, metric);
   if (k == 0) {
-    // no seeds: every count is zero
+    // no seeds: every count is zero (the basin, if asked for, untouched pixels)
     if (cudaMemsetAsync(count_out, 0, sizeof(int32_t) * B, s) != cudaSuccess) return RNN_ECUDA;
     if (cudaMemsetAsync(st.err, 0, sizeof(int), s) != cudaSuccess) return RNN_ECUDA;
+    if (basin && cudaMemsetAsync(basin, 0xFF, sizeof(int32_t) * B * (N1 + 1), s) != cudaSuccess)
+      return RNN_ECUDA;
     return RNN_OK;
   }
-  CUtensorMap map1, map2;
-  if (st.P1) {
-    pad_rows_kernel<<<grid_for(B * N1 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
-        static_cast<const uint16_t*>(D1), bs1, N1, B, d, st.P1, g.kpad);
-    if ((r = launched()) != RNN_OK) return r;
-    pad_rows_kernel<<<grid_for(B * N2 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
-        static_cast<const uint16_t*>(D2), bs2, N2, B, d, st.P2, g.kpad);
-    if ((r = launched()) != RNN_OK) return r;
-    if ((r = make_map(&map1, st.P1, g.kpad, N1, B, N1 * g.kpad, g)) != RNN_OK) return r;
-    if ((r = make_map(&map2, st.P2, g.kpad, N2, B, N2 * g.kpad, g)) != RNN_OK) return r;
+  if (mode == kCopiesNone) {
+    st.Q1 = st.X1 = static_cast<const uint16_t*>(D1);
+    st.Q2 = st.X2 = static_cast<const uint16_t*>(D2);
+    st.s1 = bs1;
+    st.s2 = bs2;
+    st.ld = d;
   } else {
-    if ((r = make_map(&map1, D1, d, N1, B, bs1, g)) != RNN_OK) return r;
-    if ((r = make_map(&map2, D2, d, N2, B, bs2, g)) != RNN_OK) return r;
+    const int qform = mode == kCopiesEuclid ? kFormQuery : kFormPad;
+    if ((r = prep_rows(D1, bs1, N1, B, d, cp.q1, g.kpad, qform, dt, di, s)) != RNN_OK) return r;
+    if ((r = prep_rows(D2, bs2, N2, B, d, cp.q2, g.kpad, qform, dt, di, s)) != RNN_OK) return r;
+    if (mode == kCopiesEuclid) {
+      if ((r = prep_rows(D1, bs1, N1, B, d, cp.x1, g.kpad, kFormCand, dt, di, s)) != RNN_OK)
+        return r;
+      if ((r = prep_rows(D2, bs2, N2, B, d, cp.x2, g.kpad, kFormCand, dt, di, s)) != RNN_OK)
+        return r;
+    }
+    st.Q1 = cp.q1;
+    st.Q2 = cp.q2;
+    st.X1 = cp.x1;
+    st.X2 = cp.x2;
+    st.s1 = N1 * g.kpad;
+    st.s2 = N2 * g.kpad;
+    st.ld = g.kpad;
   }
+  CUtensorMap map1, map2;
+  if ((r = make_map(&map1, st.X1, st.ld, N1, B, st.s1, g)) != RNN_OK) return r;
+  if ((r = make_map(&map2, st.X2, st.ld, N2, B, st.s2, g)) != RNN_OK) return r;
 
-  frm_init_kernel<<<grid_for(B * k + B * st.nwords, di->sms), kSmallThreads, 0, s>>>(st, W1, S);
-  const int lgrid = grid_for(static_cast<int64_t>(B) * k * 32, di->sms);
+  if (init) {
+    frm_starts_clear_kernel<<<grid_for(B * st.nwords + (basin ? B * (N1 + 1) : 0), di->sms),
+                              kSmallThreads, 0, s>>>(st);
+    if ((r = launched()) != RNN_OK) return r;
+    if (n_init > 0) {
+      frm_starts_mark_kernel<<<grid_for(B * n_init, di->sms), kSmallThreads, 0, s>>>(st, init,
+                                                                                    n_init);
+      if ((r = launched()) != RNN_OK) return r;
+    }
+    frm_starts_compact_kernel<<<B, kSmallThreads, 0, s>>>(st);
+  } else {
+    frm_init_kernel<<<grid_for(B * k + B * st.nwords + (basin ? B * (N1 + 1) : 0), di->sms),
+                      kSmallThreads, 0, s>>>(st, W1, S);
+  }
   if ((r = launched()) != RNN_OK) return r;
+  const int lgrid = grid_for(static_cast<int64_t>(B) * k * 32, di->sms);
 
   NNParams p;
   std::memset(&p, 0, sizeof(p));
   p.nfam = 1;
-  p.d = d;
+  p.d = st.ld;  // the gather copies whole rows of the forms
   p.idesc = make_idesc(dt, g.block_n);
   p.err = st.err;
   NNFamily& F = p.fam[0];
@@ -775,8 +1037,8 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   F.key_bstride = k;
   for (int it = 1; it <= max_iter; ++it) {
     // half-step 1: V = NN2(U)
-    F.q_base = static_cast<const uint16_t*>(D1);
-    F.q_bstride = bs1;
+    F.q_base = st.Q1;
+    F.q_bstride = st.s1;
     F.q_index = st.U;
     F.n_cand = static_cast<int32_t>(N2);
     if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s)) != RNN_OK) return r;
@@ -784,8 +1046,8 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 1, 0);
     if ((r = launched()) != RNN_OK) return r;
     // half-step 2: U = NN1(V)
-    F.q_base = static_cast<const uint16_t*>(D2);
-    F.q_bstride = bs2;
+    F.q_base = st.Q2;
+    F.q_bstride = st.s2;
     F.q_index = st.V;
     F.n_cand = static_cast<int32_t>(N1);
     if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s)) != RNN_OK) return r;
@@ -793,7 +1055,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 0, it == max_iter ? 1 : 0);
     if ((r = launched()) != RNN_OK) return r;
   }
-  frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, pairs, cap, count_out, seed_state);
+  frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, W1, pairs, cap, count_out, seed_state);
   return launched();
 }
 
@@ -842,47 +1104,81 @@ rnn_status rnn_workspace_status(const void* workspace, rnn_stream_t stream) {
   return err ? RNN_ETIMEOUT : RNN_OK;
 }
 
-size_t rnn_nn_workspace_size(int64_t nq) {
-  Carve c(nullptr);
-  c.take<int>(64);
-  c.take<unsigned long long>(nq > 0 ? nq : 1);
+// Workspace of the nearest-neighbour call: error word, packed keys, and with
+// the Euclidean metric the query and candidate forms.
+static size_t nn_layout(void* ws, int64_t nq, int64_t nx, int d, rnn_metric metric, int** err,
+                        unsigned long long** keys, uint16_t** qf, uint16_t** xf) {
+  Carve c(ws);
+  *err = c.take<int>(64);
+  *keys = c.take<unsigned long long>(nq > 0 ? nq : 1);
+  *qf = *xf = nullptr;
+  if (metric == RNN_L2 && d > 0) {
+    const int kpad = tile_depth(d, metric);
+    *qf = c.take<uint16_t>((nq > 0 ? nq : 1) * kpad);
+    *xf = c.take<uint16_t>((nx > 0 ? nx : 1) * kpad);
+  }
   return c.off;
 }
 
-rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, int d,
-                         rnn_dtype dtype, int32_t* idx_out, float* score_out, void* workspace,
-                         size_t ws_bytes, rnn_stream_t stream) {
+size_t rnn_nn_workspace_size_ex(int64_t nq, int64_t nx, int d, rnn_metric metric) {
+  int* e;
+  unsigned long long* k;
+  uint16_t *a, *b;
+  return nn_layout(nullptr, nq > 0 ? nq : 0, nx > 0 ? nx : 0, d, metric, &e, &k, &a, &b);
+}
+
+size_t rnn_nn_workspace_size(int64_t nq) { return rnn_nn_workspace_size_ex(nq, 0, 0, RNN_DOT); }
+
+rnn_status rnn_nn_argmax_ex(const void* Q, int64_t nq, const void* X, int64_t nx, int d,
+                            rnn_dtype dtype, rnn_metric metric, int32_t* idx_out,
+                            float* score_out, void* workspace, size_t ws_bytes,
+                            rnn_stream_t stream) {
   if (nq < 0 || nx < 1 || nq > INT32_MAX || nx > INT32_MAX) return RNN_EINVAL;
-  if (!valid_dtype(dtype)) return RNN_EINVAL;
+  if (!valid_dtype(dtype) || !valid_metric(metric)) return RNN_EINVAL;
   rnn_status r = check_desc(X, d);
   if (r != RNN_OK) return r;
   if (nq > 0) {  // with no queries, Q and idx_out may be null
     if ((r = check_desc(Q, d)) != RNN_OK) return r;
     if (!idx_out) return RNN_EINVAL;
   }
-  if (!workspace || !aligned256(workspace) || ws_bytes < rnn_nn_workspace_size(nq))
+  if (!workspace || !aligned256(workspace) ||
+      ws_bytes < rnn_nn_workspace_size_ex(nq, nx, d, metric))
     return RNN_EWORKSPACE;
   DeviceInfo* di = nullptr;
   if ((r = device_info(&di)) != RNN_OK) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  Carve c(workspace);
-  int* err = c.take<int>(64);
-  unsigned long long* keys = c.take<unsigned long long>(nq > 0 ? nq : 1);
+  int* err;
+  unsigned long long* keys;
+  uint16_t *qf, *xf;
+  nn_layout(workspace, nq, nx, d, metric, &err, &keys, &qf, &xf);
   zero_keys_kernel<<<grid_for(nq, di->sms), kSmallThreads, 0, s>>>(keys, nq, nullptr, 0, err);
   if ((r = launched()) != RNN_OK) return r;
   if (nq == 0) return RNN_OK;
-  const Geometry g = geometry(d);
+  const bool l2 = metric == RNN_L2;
+  const Geometry g = geometry(d + (l2 ? kAugCols : 0));
+  const uint16_t* q16 = static_cast<const uint16_t*>(Q);
+  const uint16_t* x16 = static_cast<const uint16_t*>(X);
+  int ld = d;
+  if (l2) {
+    if ((r = prep_rows(Q, nq * d, nq, 1, d, qf, g.kpad, kFormQuery, dtype, di, s)) != RNN_OK)
+      return r;
+    if ((r = prep_rows(X, nx * d, nx, 1, d, xf, g.kpad, kFormCand, dtype, di, s)) != RNN_OK)
+      return r;
+    q16 = qf;
+    x16 = xf;
+    ld = g.kpad;
+  }
   CUtensorMap mx, mq;
-  if ((r = make_map(&mx, X, d, nx, 1, nx * d, g)) != RNN_OK) return r;
-  if ((r = make_map(&mq, Q, d, nq, 1, nq * d, g, kBlockM)) != RNN_OK) return r;
+  if ((r = make_map(&mx, x16, ld, nx, 1, nx * ld, g)) != RNN_OK) return r;
+  if ((r = make_map(&mq, q16, ld, nq, 1, nq * ld, g, kBlockM)) != RNN_OK) return r;
   NNParams p;
   std::memset(&p, 0, sizeof(p));
   p.nfam = 1;
-  p.d = d;
+  p.d = ld;
   p.idesc = make_idesc(dtype, g.block_n);
   p.err = err;
   NNFamily& F = p.fam[0];
-  F.q_base = static_cast<const uint16_t*>(Q);
+  F.q_base = q16;
   F.q_count = static_cast<int32_t>(nq);
   F.n_cand = static_cast<int32_t>(nx);
   F.nbatch = 1;
@@ -890,52 +1186,73 @@ rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, i
   F.q_tma = 1;
   if ((r = launch_nn(p, mx, mx, mq, mq, g, di, s)) != RNN_OK) return r;
   const int lg = grid_for(nq * 32, di->sms);
-  const uint16_t* q16 = static_cast<const uint16_t*>(Q);
-  const uint16_t* x16 = static_cast<const uint16_t*>(X);
   if (dtype == RNN_BF16)
-    locate_unpack_kernel<true><<<lg, kSmallThreads, 0, s>>>(keys, nq, q16, x16,
-                                                           static_cast<int>(nx), d, idx_out,
-                                                           score_out);
+    locate_unpack_kernel<true><<<lg, kSmallThreads, 0, s>>>(
+        keys, nq, q16, x16, static_cast<int>(nx), ld, d, l2, idx_out, score_out);
   else
-    locate_unpack_kernel<false><<<lg, kSmallThreads, 0, s>>>(keys, nq, q16, x16,
-                                                            static_cast<int>(nx), d, idx_out,
-                                                            score_out);
+    locate_unpack_kernel<false><<<lg, kSmallThreads, 0, s>>>(
+        keys, nq, q16, x16, static_cast<int>(nx), ld, d, l2, idx_out, score_out);
   return launched();
 }
 
+rnn_status rnn_nn_argmax(const void* Q, int64_t nq, const void* X, int64_t nx, int d,
+                         rnn_dtype dtype, int32_t* idx_out, float* score_out, void* workspace,
+                         size_t ws_bytes, rnn_stream_t stream) {
+  return rnn_nn_argmax_ex(Q, nq, X, nx, d, dtype, RNN_DOT, idx_out, score_out, workspace,
+                          ws_bytes, stream);
+}
+
 // Workspace of the reciprocal set: error word, packed keys of both sweeps,
-// block counts, and (when d < kpad) zero-padded copies of both maps.
-static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, int** err,
-                         unsigned long long** rowk, unsigned long long** colk, int** counts,
-                         uint16_t** p1, uint16_t** p2) {
+// block counts, and the row forms: a zero-padded copy of each map (dot
+// metric, d = 8, 24, 40, ...), or a query and a candidate form of each map
+// (Euclidean metric).
+struct MnnWs {
+  int* err;
+  unsigned long long *rowk, *colk;
+  int* counts;
+  uint16_t *q1, *x1, *q2, *x2;
+};
+
+static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, rnn_metric metric, MnnWs* w) {
   Carve c(ws);
-  *err = c.take<int>(64);
-  *rowk = c.take<unsigned long long>(n1 > 0 ? n1 : 1);
-  *colk = c.take<unsigned long long>(n2 > 0 ? n2 : 1);
-  *counts = c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
-  const int kpad = d > 0 ? padded_depth(d) : 0;
-  *p1 = kpad != d ? c.take<uint16_t>(n1 * kpad) : nullptr;
-  *p2 = kpad != d ? c.take<uint16_t>(n2 * kpad) : nullptr;
+  w->err = c.take<int>(64);
+  w->rowk = c.take<unsigned long long>(n1 > 0 ? n1 : 1);
+  w->colk = c.take<unsigned long long>(n2 > 0 ? n2 : 1);
+  w->counts = c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
+  w->q1 = w->x1 = w->q2 = w->x2 = nullptr;
+  const int mode = d > 0 ? copies_for(d, metric) : kCopiesNone;
+  if (mode != kCopiesNone) {
+    const int kpad = tile_depth(d, metric);
+    w->q1 = c.take<uint16_t>(n1 * kpad);
+    w->q2 = c.take<uint16_t>(n2 * kpad);
+    w->x1 = w->q1;
+    w->x2 = w->q2;
+    if (mode == kCopiesEuclid) {
+      w->x1 = c.take<uint16_t>(n1 * kpad);
+      w->x2 = c.take<uint16_t>(n2 * kpad);
+    }
+  }
   return c.off;
 }
 
-size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2, int d) {
+size_t rnn_mnn_workspace_size_ex(int H1, int W1, int H2, int W2, int d, rnn_metric metric) {
   const int64_t n1 = static_cast<int64_t>(H1 > 0 ? H1 : 0) * (W1 > 0 ? W1 : 0);
   const int64_t n2 = static_cast<int64_t>(H2 > 0 ? H2 : 0) * (W2 > 0 ? W2 : 0);
-  int* e;
-  unsigned long long *a, *b;
-  int* cnt;
-  uint16_t *p1, *p2;
-  return mnn_layout(nullptr, n1, n2, d > 0 ? d : 0, &e, &a, &b, &cnt, &p1, &p2);
+  MnnWs w;
+  return mnn_layout(nullptr, n1, n2, d > 0 ? d : 0, metric, &w);
 }
 
-rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, int H2, int W2,
-                              int d, rnn_dtype dtype, int32_t* pairs_out, int64_t cap,
-                              int32_t* count_out, int32_t* rowarg_out, float* rowmax_out,
-                              int32_t* colarg_out, float* colmax_out, void* workspace,
-                              size_t ws_bytes, rnn_stream_t stream) {
+size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2, int d) {
+  return rnn_mnn_workspace_size_ex(H1, W1, H2, W2, d, RNN_DOT);
+}
+
+rnn_status rnn_mnn_exhaustive_ex(const void* D1, int H1, int W1, const void* D2, int H2, int W2,
+                                 int d, rnn_dtype dtype, rnn_metric metric, int32_t* pairs_out,
+                                 int64_t cap, int32_t* count_out, int32_t* rowarg_out,
+                                 float* rowmax_out, int32_t* colarg_out, float* colmax_out,
+                                 void* workspace, size_t ws_bytes, rnn_stream_t stream) {
   if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0) return RNN_EINVAL;
-  if (!valid_dtype(dtype)) return RNN_EINVAL;
+  if (!valid_dtype(dtype) || !valid_metric(metric)) return RNN_EINVAL;
   rnn_status r = check_desc(D1, d);
   if (r != RNN_OK) return r;
   if ((r = check_desc(D2, d)) != RNN_OK) return r;
@@ -944,80 +1261,99 @@ rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, in
   if (!pairs_out || !count_out) return RNN_EINVAL;
   if (cap < (n1 < n2 ? n1 : n2)) return RNN_ECAPACITY;
   if (!workspace || !aligned256(workspace) ||
-      ws_bytes < rnn_mnn_workspace_size(H1, W1, H2, W2, d))
+      ws_bytes < rnn_mnn_workspace_size_ex(H1, W1, H2, W2, d, metric))
     return RNN_EWORKSPACE;
   DeviceInfo* di = nullptr;
   if ((r = device_info(&di)) != RNN_OK) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int* err;
-  unsigned long long *rowk, *colk;
-  int* counts;
-  uint16_t *p1, *p2;
-  mnn_layout(workspace, n1, n2, d, &err, &rowk, &colk, &counts, &p1, &p2);
+  MnnWs w;
+  mnn_layout(workspace, n1, n2, d, metric, &w);
   const int nblk1 = static_cast<int>((n1 + kMnnChunk - 1) / kMnnChunk);
   const int nblk2 = static_cast<int>((n2 + kMnnChunk - 1) / kMnnChunk);
 
-  const Geometry g = geometry(d);
-  // tensor maps over the padded copies when d < kpad, else over the inputs
-  const void* T1 = D1;
-  const void* T2 = D2;
-  int dm = d;
-  if (p1) {
-    pad_rows_kernel<<<grid_for(n1 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
-        static_cast<const uint16_t*>(D1), n1 * d, n1, 1, d, p1, g.kpad);
-    if ((r = launched()) != RNN_OK) return r;
-    pad_rows_kernel<<<grid_for(n2 * (g.kpad / 8), di->sms), kSmallThreads, 0, s>>>(
-        static_cast<const uint16_t*>(D2), n2 * d, n2, 1, d, p2, g.kpad);
-    if ((r = launched()) != RNN_OK) return r;
-    T1 = p1;
-    T2 = p2;
-    dm = g.kpad;
+  const bool l2 = metric == RNN_L2;
+  const Geometry g = geometry(d + (l2 ? kAugCols : 0));
+  // tensor maps and locate rows over the row forms, or over the inputs
+  const uint16_t* Q1 = static_cast<const uint16_t*>(D1);
+  const uint16_t* Q2 = static_cast<const uint16_t*>(D2);
+  const uint16_t* X1 = Q1;
+  const uint16_t* X2 = Q2;
+  int ld = d;
+  const int mode = copies_for(d, metric);
+  if (mode != kCopiesNone) {
+    const int qform = l2 ? kFormQuery : kFormPad;
+    if ((r = prep_rows(D1, n1 * d, n1, 1, d, w.q1, g.kpad, qform, dtype, di, s)) != RNN_OK)
+      return r;
+    if ((r = prep_rows(D2, n2 * d, n2, 1, d, w.q2, g.kpad, qform, dtype, di, s)) != RNN_OK)
+      return r;
+    if (l2) {
+      if ((r = prep_rows(D1, n1 * d, n1, 1, d, w.x1, g.kpad, kFormCand, dtype, di, s)) != RNN_OK)
+        return r;
+      if ((r = prep_rows(D2, n2 * d, n2, 1, d, w.x2, g.kpad, kFormCand, dtype, di, s)) != RNN_OK)
+        return r;
+    }
+    Q1 = w.q1;
+    Q2 = w.q2;
+    X1 = w.x1;
+    X2 = w.x2;
+    ld = g.kpad;
   }
   CUtensorMap m1, m2, q1, q2;
-  if ((r = make_map(&m1, T1, dm, n1, 1, n1 * dm, g)) != RNN_OK) return r;
-  if ((r = make_map(&m2, T2, dm, n2, 1, n2 * dm, g)) != RNN_OK) return r;
-  if ((r = make_map(&q1, T1, dm, n1, 1, n1 * dm, g, kBlockM)) != RNN_OK) return r;
-  if ((r = make_map(&q2, T2, dm, n2, 1, n2 * dm, g, kBlockM)) != RNN_OK) return r;
+  if ((r = make_map(&m1, X1, ld, n1, 1, n1 * ld, g)) != RNN_OK) return r;
+  if ((r = make_map(&m2, X2, ld, n2, 1, n2 * ld, g)) != RNN_OK) return r;
+  if ((r = make_map(&q1, Q1, ld, n1, 1, n1 * ld, g, kBlockM)) != RNN_OK) return r;
+  if ((r = make_map(&q2, Q2, ld, n2, 1, n2 * ld, g, kBlockM)) != RNN_OK) return r;
 
-  zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(rowk, n1, colk, n2, err);
+  zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2,
+                                                                        w.err);
   if ((r = launched()) != RNN_OK) return r;
   NNParams p;
   std::memset(&p, 0, sizeof(p));
   p.nfam = 2;
-  p.d = d;
+  p.d = ld;
   p.idesc = make_idesc(dtype, g.block_n);
-  p.err = err;
+  p.err = w.err;
   // sweep 1: rows of D1 against D2 -> NN2; sweep 2: rows of D2 against D1 -> NN1
-  p.fam[0].q_base = static_cast<const uint16_t*>(D1);
+  p.fam[0].q_base = Q1;
   p.fam[0].q_count = static_cast<int32_t>(n1);
   p.fam[0].n_cand = static_cast<int32_t>(n2);
   p.fam[0].nbatch = 1;
-  p.fam[0].keys = rowk;
-  p.fam[1].q_base = static_cast<const uint16_t*>(D2);
+  p.fam[0].keys = w.rowk;
+  p.fam[1].q_base = Q2;
   p.fam[1].q_count = static_cast<int32_t>(n2);
   p.fam[1].n_cand = static_cast<int32_t>(n1);
   p.fam[1].nbatch = 1;
-  p.fam[1].keys = colk;
+  p.fam[1].keys = w.colk;
   p.fam[0].q_tma = 1;
   p.fam[1].q_tma = 1;
   if ((r = launch_nn(p, m2, m1, q1, q2, g, di, s)) != RNN_OK) return r;
-  const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
   {
     const int lg = grid_for((n1 + n2) * 32, di->sms);
-    const uint16_t* a16 = static_cast<const uint16_t*>(D1);
-    const uint16_t* b16 = static_cast<const uint16_t*>(D2);
     if (dtype == RNN_BF16)
-      locate_mnn_kernel<true><<<lg, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, a16, b16, d);
+      locate_mnn_kernel<true><<<lg, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2, Q1, X1, Q2,
+                                                           X2, ld, d, l2);
     else
-      locate_mnn_kernel<false><<<lg, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, a16, b16, d);
+      locate_mnn_kernel<false><<<lg, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2, Q1, X1, Q2,
+                                                            X2, ld, d, l2);
     if ((r = launched()) != RNN_OK) return r;
   }
-  mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(rowk, n1, colk, n2, counts, nblk1, rowarg_out,
-                                                rowmax_out, colarg_out, colmax_out);
+  const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
+  mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2, w.counts, nblk1,
+                                                rowarg_out, rowmax_out, colarg_out, colmax_out);
   if ((r = launched()) != RNN_OK) return r;
-  mnn_write_kernel<<<nblk1, kSmallThreads, 0, s>>>(rowk, n1, colk, counts, nblk1, pairs_out,
-                                                   count_out);
+  mnn_write_kernel<<<nblk1, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, w.counts, nblk1,
+                                                   pairs_out, count_out);
   return launched();
+}
+
+rnn_status rnn_mnn_exhaustive(const void* D1, int H1, int W1, const void* D2, int H2, int W2,
+                              int d, rnn_dtype dtype, int32_t* pairs_out, int64_t cap,
+                              int32_t* count_out, int32_t* rowarg_out, float* rowmax_out,
+                              int32_t* colarg_out, float* colmax_out, void* workspace,
+                              size_t ws_bytes, rnn_stream_t stream) {
+  return rnn_mnn_exhaustive_ex(D1, H1, W1, D2, H2, W2, d, dtype, RNN_DOT, pairs_out, cap,
+                               count_out, rowarg_out, rowmax_out, colarg_out, colmax_out,
+                               workspace, ws_bytes, stream);
 }
 
 int64_t rnn_frm_num_seeds(int H1, int W1, int seed_stride) {
@@ -1031,10 +1367,17 @@ int64_t rnn_frm_max_pairs(int H1, int W1, int H2, int W2, int seed_stride) {
   return k < n2 ? k : n2;
 }
 
+size_t rnn_frm_workspace_size_ex(int B, int H1, int W1, int H2, int W2, int d,
+                                 rnn_metric metric, int seed_stride, int64_t n_init) {
+  if (B < 1 || H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || d <= 0) return 0;
+  if (!valid_metric(metric) || (n_init < 0 && seed_stride < 1)) return 0;
+  const int64_t k = n_init >= 0 ? n_init : num_seeds(H1, W1, seed_stride);
+  return frm_bytes(B, k, static_cast<int64_t>(H1) * W1, static_cast<int64_t>(H2) * W2, d,
+                   metric);
+}
+
 size_t rnn_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int d, int seed_stride) {
-  if (B < 1 || H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || d <= 0 || seed_stride < 1) return 0;
-  return frm_bytes(B, num_seeds(H1, W1, seed_stride), static_cast<int64_t>(H1) * W1,
-                   static_cast<int64_t>(H2) * W2, d);
+  return rnn_frm_workspace_size_ex(B, H1, W1, H2, W2, d, RNN_DOT, seed_stride, -1);
 }
 
 rnn_status rnn_frm_match(const void* D1, int H1, int W1, const void* D2, int H2, int W2, int d,
@@ -1042,9 +1385,9 @@ rnn_status rnn_frm_match(const void* D1, int H1, int W1, const void* D2, int H2,
                          int64_t cap, int32_t* count_out, int32_t* seed_state_out,
                          void* workspace, size_t ws_bytes, rnn_stream_t stream) {
   const int64_t n1 = static_cast<int64_t>(H1) * W1, n2 = static_cast<int64_t>(H2) * W2;
-  return frm_run(1, D1, n1 * d, D2, n2 * d, H1, W1, H2, W2, d, dtype, seed_stride, max_iter,
-                 pairs_out, cap, count_out, seed_state_out, workspace, ws_bytes,
-                 reinterpret_cast<cudaStream_t>(stream));
+  return frm_run(1, D1, n1 * d, D2, n2 * d, H1, W1, H2, W2, d, dtype, RNN_DOT, nullptr, 0,
+                 seed_stride, max_iter, 0.f, pairs_out, cap, count_out, seed_state_out, nullptr,
+                 workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 rnn_status rnn_frm_match_batched(int B, const void* D1, int64_t d1_batch_stride, const void* D2,
@@ -1053,9 +1396,23 @@ rnn_status rnn_frm_match_batched(int B, const void* D1, int64_t d1_batch_stride,
                                  int32_t* pairs_out, int64_t cap, int32_t* count_out,
                                  int32_t* seed_state_out, void* workspace, size_t ws_bytes,
                                  rnn_stream_t stream) {
-  return frm_run(B, D1, d1_batch_stride, D2, d2_batch_stride, H1, W1, H2, W2, d, dtype,
-                 seed_stride, max_iter, pairs_out, cap, count_out, seed_state_out, workspace,
-                 ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return frm_run(B, D1, d1_batch_stride, D2, d2_batch_stride, H1, W1, H2, W2, d, dtype, RNN_DOT,
+                 nullptr, 0, seed_stride, max_iter, 0.f, pairs_out, cap, count_out,
+                 seed_state_out, nullptr, workspace, ws_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+rnn_status rnn_frm_match_ex(int B, const void* D1, int64_t d1_batch_stride, const void* D2,
+                            int64_t d2_batch_stride, int H1, int W1, int H2, int W2, int d,
+                            rnn_dtype dtype, rnn_metric metric, const int32_t* init_xy1,
+                            int64_t n_init, int seed_stride, int max_iter, float pixel_tol,
+                            int32_t* pairs_out, int64_t cap, int32_t* count_out,
+                            int32_t* seed_state_out, int32_t* basin_out, void* workspace,
+                            size_t ws_bytes, rnn_stream_t stream) {
+  return frm_run(B, D1, d1_batch_stride, D2, d2_batch_stride, H1, W1, H2, W2, d, dtype, metric,
+                 init_xy1, n_init, seed_stride, max_iter, pixel_tol, pairs_out, cap, count_out,
+                 seed_state_out, basin_out, workspace, ws_bytes,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -135,3 +135,53 @@ def test_frm_argument_errors(lib):
     single = lib.rnn_frm_match
     assert single(FAKE, 8, 8, FAKE, 8, 8, 16, 0, 2, 0, FAKE, 16, FAKE, None, FAKE, ws,
                   None) == EINVAL
+
+
+def test_ex_workspace_sizes(lib):
+    dot = lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, _lib.RNN_DOT)
+    assert dot == lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24)
+    # the Euclidean metric keeps a query and a candidate form of each map
+    l2 = lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, _lib.RNN_L2)
+    assert l2 >= dot + 2 * 384 * 512 * 32 * 2
+    assert lib.rnn_nn_workspace_size_ex(100, 5000, 24, _lib.RNN_DOT) == \
+        lib.rnn_nn_workspace_size(100)
+    assert lib.rnn_nn_workspace_size_ex(100, 5000, 24, _lib.RNN_L2) >= \
+        lib.rnn_nn_workspace_size(100) + (100 + 5000) * 32 * 2
+    grid = lib.rnn_frm_workspace_size_ex(2, 64, 64, 64, 64, 16, _lib.RNN_DOT, 8, -1)
+    assert grid == lib.rnn_frm_workspace_size(2, 64, 64, 64, 64, 16, 8)
+    # given starts: sized by their count, whatever the stride
+    assert lib.rnn_frm_workspace_size_ex(2, 64, 64, 64, 64, 16, _lib.RNN_DOT, 0, 1000) > \
+        lib.rnn_frm_workspace_size_ex(2, 64, 64, 64, 64, 16, _lib.RNN_DOT, 0, 10)
+    assert lib.rnn_frm_workspace_size_ex(2, 64, 64, 64, 64, 16, 7, 8, -1) == 0
+
+
+def test_frm_ex_argument_errors(lib):
+    n_init = 20
+    ws = lib.rnn_frm_workspace_size_ex(2, 8, 8, 8, 8, 16, _lib.RNN_DOT, 2, n_init)
+    f = lib.rnn_frm_match_ex
+
+    def call(**kw):
+        a = dict(B=2, D1=FAKE, s1=8 * 8 * 16, D2=FAKE, s2=8 * 8 * 16, H1=8, W1=8, H2=8, W2=8,
+                 d=16, dt=0, metric=0, init=FAKE, n=n_init, S=2, it=1, tol=0.0, pairs=FAKE,
+                 cap=20, count=FAKE, basin=None, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return f(a["B"], a["D1"], a["s1"], a["D2"], a["s2"], a["H1"], a["W1"], a["H2"], a["W2"],
+                 a["d"], a["dt"], a["metric"], a["init"], a["n"], a["S"], a["it"], a["tol"],
+                 a["pairs"], a["cap"], a["count"], None, a["basin"], a["ws"], a["wsb"], None)
+
+    assert call(metric=2) == EINVAL
+    assert call(tol=-1.0) == EINVAL
+    assert call(tol=float("nan")) == EINVAL
+    assert call(init=None, tol=1.5) == EINVAL       # a tolerance needs given starts
+    assert call(n=-1) == EINVAL
+    assert call(init=None, S=0) == EINVAL
+    assert call(it=0) == EINVAL
+    # with a tolerance the (start, match) pairs are bounded by the starts only
+    assert call(tol=1.5, cap=19) == ECAP
+    assert call(wsb=ws - 1) == EWS
+    assert call(d=4) == EALIGN
+    nn = lib.rnn_nn_argmax_ex
+    assert nn(FAKE, 10, FAKE, 10, 16, 0, 5, FAKE, None, FAKE, 1 << 20, None) == EINVAL
+    mnn = lib.rnn_mnn_exhaustive_ex
+    assert mnn(FAKE, 4, 4, FAKE, 4, 4, 16, 0, 9, FAKE, 16, FAKE, None, None, None, None, FAKE,
+               1 << 20, None) == EINVAL
