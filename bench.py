@@ -28,6 +28,26 @@ import statistics
 import sys
 import time
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
+# the fused kernel in the bench step, from one ncu capture of the step's
+# first FRM call (20 launches averaged).  It belongs to the kernel sources it
+# was taken on: with any other sources the bench reports traffic as null.
+TRAFFIC = {"sources_sha256": "bc38bcce7e358f6b8e111af581462b336795c3a8ef7103877e8ad4560c70ded4",
+           "frm_nn_bytes_per_launch": 37.33e6}
+
+
+def _kernel_sources_sha256() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "reciprocal_nearest_neighbour_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -288,8 +308,10 @@ def run_native(args):
     nn_time_s = sum(nn_ms) * 1e-3
     achieved_tf = flops / nn_time_s / 1e12
     peak_tf = peaks["bf16_tflops_sustained"]
+    traffic = (TRAFFIC["frm_nn_bytes_per_launch"]
+               if _kernel_sources_sha256() == TRAFFIC["sources_sha256"] else None)
     roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": achieved_tf / peak_tf, "traffic": None,
+                "frac": achieved_tf / peak_tf, "traffic": traffic,
                 "kernel": "nn_argmax_kernel (FRM half-steps)",
                 "launches": nrec, "avg_launch_us": 1e3 * sum(nn_ms) / max(nrec, 1),
                 "flops_per_launch": flops / max(nrec, 1),
@@ -332,12 +354,15 @@ def run_native(args):
         mnn = {}
         props = torch.cuda.get_device_properties(dev)
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        for mode, wl in (("quantised", "mnn_512x384_q"), ("fp16", "mnn_512x384_f")):
+        for mode, wl, metric in (("quantised", "mnn_512x384_q", "dot"),
+                                 ("fp16", "mnn_512x384_f", "dot"),
+                                 ("fp16_euclidean", "mnn_512x384_f", "l2")):
             ww = synth.WORKLOADS[wl]
             a, b = synth.make_workload_storage(ww, "f16", pairs=[0])
             a, b = a[0].to(dev), b[0].to(dev)
-            out = rnn.mnn_exhaustive(a, b)
-            ws = torch.empty(lib.rnn_mnn_workspace_size(ww.H, ww.W, ww.H, ww.W, ww.d),
+            out = rnn.mnn_exhaustive(a, b, metric=metric)
+            ws = torch.empty(lib.rnn_mnn_workspace_size_ex(ww.H, ww.W, ww.H, ww.W, ww.d,
+                                                           _lib.METRICS[metric]),
                              dtype=torch.uint8, device=dev)
             reps = args.mnn_reps
             ka = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
@@ -351,12 +376,12 @@ def run_native(args):
             hb = (ctypes.c_void_p * reps)(*[e.cuda_event for e in kb])
             r2 = ctypes.c_int(0)
             for _ in range(2):
-                rnn.mnn_exhaustive(a, b, workspace=ws, out=out)
+                rnn.mnn_exhaustive(a, b, workspace=ws, out=out, metric=metric)
             lib.rnn_set_kernel_timer(ha, hb, reps, ctypes.byref(r2))
             for i in range(reps):
                 flush.fill_(i & 0xFF)                   # evict the maps from L2
                 ca[i].record()
-                rnn.mnn_exhaustive(a, b, workspace=ws, out=out)
+                rnn.mnn_exhaustive(a, b, workspace=ws, out=out, metric=metric)
                 cb[i].record()
             torch.cuda.synchronize()
             lib.rnn_set_kernel_timer(None, None, 0, None)
@@ -368,7 +393,8 @@ def run_native(args):
             peak_cmp = props.multi_processor_count * 128 * peaks["sm_max_mhz"] * 1e6
             achieved_cmp = compares / (kern_ms * 1e-3)
             mnn[mode] = {
-                "metric": "exhaustive MNN pair-scores/s at 512x384, d=24",
+                "metric": ("exhaustive MNN pair-scores/s at 512x384, d=24" if metric == "dot"
+                           else "exhaustive Euclidean MNN pair-scores/s at 512x384, d=24"),
                 "value": scores / (call_ms * 1e-3), "unit": "pair-scores/s",
                 "ms_per_call": call_ms, "pairs": int(out.count.item()),
                 "roofline": {"bound": "alu", "achieved": achieved_cmp / 1e12,
@@ -380,6 +406,36 @@ def run_native(args):
                                            f"{peaks['sm_max_mhz']:.0f} MHz"},
                 "l2": "256 MB flush before every call"}
         del flush
+
+    # ---------------- FRM options on the step's pairs: given starts, basin mode
+    options = None
+    if not args.skip_mnn:
+        options = {}
+        # starts one pixel right of and below each grid seed (3072 a pair)
+        seeds = torch.arange(w.H * w.W, device=dev, dtype=torch.int32).reshape(w.H, w.W)
+        off = w.seed_stride // 2 + 1
+        starts = seeds[off::w.seed_stride, off::w.seed_stride].reshape(1, -1).repeat(P, 1)
+        cases = (("refine", dict(max_iter=1, init=starts, pixel_tol=1.5), starts.shape[1] * P,
+                  "refined starts/s (one round trip, pixel_tol 1.5)"),
+                 ("basin", dict(seed_stride=w.seed_stride, max_iter=w.max_iter, with_basin=True),
+                  P, "FRM pairs/s with the basin output"))
+        for name, kw, units, what in cases:
+            for _ in range(2):
+                r = rnn.frm_match_ex(A, B, **kw)
+            reps = 10
+            oa = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            ob = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            for i in range(reps):
+                oa[i].record()
+                r = rnn.frm_match_ex(A, B, **kw)
+                ob[i].record()
+            torch.cuda.synchronize()
+            ms = statistics.median(_event_ms(oa, ob, reps))
+            options[name] = {"metric": what, "value": units / (ms * 1e-3),
+                             "unit": "starts/s" if name == "refine" else "pairs/s",
+                             "ms_per_call": ms, "pairs_per_call": P,
+                             "outputs": int(r.count.sum().item()),
+                             "note": "includes the binding's output and workspace allocation"}
 
     # ----------------------------------------------------------- CPU baseline
     cpu = None
@@ -399,7 +455,8 @@ def run_native(args):
                        "d": w.d, "seed_stride": w.seed_stride, "max_iter": w.max_iter,
                        "global_batch": world * P, "parallelism": f"replicas x{world}",
                        "l2": f"step inputs {2 * A_h.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
-            "e2e": e2e, "roofline": roofline, "mnn": mnn, "cpu_baseline": cpu,
+            "e2e": e2e, "roofline": roofline, "mnn": mnn, "frm_options": options,
+            "cpu_baseline": cpu,
             "clocks": clocks, "gpu_launches": int(launches),
         }
         print(json.dumps(line), flush=True)
