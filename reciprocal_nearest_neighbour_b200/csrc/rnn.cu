@@ -301,45 +301,53 @@ __device__ __forceinline__ uint16_t f_to_bits(float x, bool bf16) {
               : __half_as_ushort(__float2half_rn(x));
 }
 
+// One thread per 16-byte chunk of the output, so that reads and writes are
+// coalesced.  d is a multiple of 8, so a chunk lies wholly among the channels
+// or wholly past them; the first chunk past them holds the augmentation (its
+// thread reads the whole row for |x|^2), the rest are zero.
 template <bool kBf16>
 __global__ void prep_rows_kernel(const uint16_t* src, int64_t bstride, int64_t rows, int nbatch,
                                  int d, uint16_t* dst, int kpad, int form) {
-  const int64_t total = static_cast<int64_t>(nbatch) * rows;
+  const int cpr = kpad / 8, creal = d / 8;  // chunks per output row / per input row
+  const int64_t total = static_cast<int64_t>(nbatch) * rows * cpr;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t rr = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; rr < total;
-       rr += stride) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += stride) {
+    const int64_t rr = i / cpr;  // row over all batches
+    const int c = static_cast<int>(i - rr * cpr);
     const int64_t b = rr / rows, r = rr - b * rows;
     const uint4* in = reinterpret_cast<const uint4*>(src + b * bstride + r * d);
-    uint4* out = reinterpret_cast<uint4*>(dst + rr * kpad);
-    float n2 = 0.f;
-    for (int c = 0; c < d / 8; ++c) {
-      const uint4 v = __ldg(in + c);
-      out[c] = v;
-      if (form == kFormCand) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (c < creal) {
+      v = __ldg(in + c);
+    } else if (c == creal && form != kFormPad) {
+      uint16_t aug[kAugCols];
+      if (form == kFormQuery) {
+        aug[0] = aug[1] = aug[2] = f_to_bits(1.0f, kBf16);
+      } else {
+        float n2 = 0.f;
+        for (int cc = 0; cc < creal; ++cc) {
+          const uint4 x = __ldg(in + cc);
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float lo = bits_to_f(static_cast<uint16_t>(w[e] & 0xFFFFu), kBf16);
-          const float hi = bits_to_f(static_cast<uint16_t>(w[e] >> 16), kBf16);
-          n2 = fmaf(lo, lo, n2);
-          n2 = fmaf(hi, hi, n2);
+          for (int e = 0; e < 4; ++e) {
+            const float lo = bits_to_f(static_cast<uint16_t>(w[e] & 0xFFFFu), kBf16);
+            const float hi = bits_to_f(static_cast<uint16_t>(w[e] >> 16), kBf16);
+            n2 = fmaf(lo, lo, n2);
+            n2 = fmaf(hi, hi, n2);
+          }
+        }
+        float rest = -0.5f * n2;
+#pragma unroll
+        for (int e = 0; e < kAugCols; ++e) {
+          aug[e] = f_to_bits(rest, kBf16);
+          rest -= bits_to_f(aug[e], kBf16);
         }
       }
+      v.x = static_cast<uint32_t>(aug[0]) | (static_cast<uint32_t>(aug[1]) << 16);
+      v.y = static_cast<uint32_t>(aug[2]);
     }
-    // columns d .. kpad-1: the augmentation (if any), then zeros
-    uint16_t aug[kAugCols] = {0, 0, 0};
-    if (form == kFormQuery) {
-      aug[0] = aug[1] = aug[2] = f_to_bits(1.0f, kBf16);
-    } else if (form == kFormCand) {
-      float v = -0.5f * n2;
-#pragma unroll
-      for (int e = 0; e < kAugCols; ++e) {
-        aug[e] = f_to_bits(v, kBf16);
-        v -= bits_to_f(aug[e], kBf16);
-      }
-    }
-    uint16_t* tail = dst + rr * kpad + d;
-    for (int c = 0; c < kpad - d; ++c) tail[c] = c < kAugCols && form != kFormPad ? aug[c] : 0;
+    reinterpret_cast<uint4*>(dst)[i] = v;
   }
 }
 
@@ -917,7 +925,7 @@ static int64_t num_seeds(int H, int W, int S) {
 static rnn_status prep_rows(const void* src, int64_t bstride, int64_t rows, int nbatch, int d,
                             uint16_t* dst, int kpad, int form, rnn_dtype dt, DeviceInfo* di,
                             cudaStream_t s) {
-  const int grid = grid_for(static_cast<int64_t>(nbatch) * rows, di->sms);
+  const int grid = grid_for(static_cast<int64_t>(nbatch) * rows * (kpad / 8), di->sms);
   const uint16_t* in = static_cast<const uint16_t*>(src);
   if (dt == RNN_BF16)
     prep_rows_kernel<true><<<grid, kSmallThreads, 0, s>>>(in, bstride, rows, nbatch, d, dst,
