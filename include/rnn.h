@@ -145,7 +145,7 @@ rnn_status rnn_mnn_exhaustive(const void *D1, int H1, int W1, const void *D2, in
  *   output the (U, V) of the seeds that are no longer active, unique, sorted
  *          by U.  Every output pair is in M.
  *
- * The whole loop runs on the device: 6*max_iter + 2 kernel launches (2 more
+ * The whole loop runs on the device: 4*max_iter + 2 kernel launches (2 more
  * when d needs padded copies), no host synchronisation.
  *
  *   seed_stride >= 1, max_iter >= 1 (RNN_EINVAL otherwise).
@@ -217,7 +217,7 @@ rnn_status rnn_frm_match_batched(int B, const void *D1, int64_t d1_batch_stride,
  *                hold -1, -1, 0, 0.
  * rnn_frm_workspace_size_ex takes n_init = the starts per pair, or -1 for the
  * grid of stride seed_stride.
- * 2 + 6*max_iter kernel launches, plus 2 (padded copies, dot metric with
+ * 2 + 4*max_iter kernel launches, plus 2 (padded copies, dot metric with
  * d = 8, 24, 40, ...) or 4 (Euclidean metric) for the row copies, plus 2 with
  * given starts.
  */

@@ -569,13 +569,17 @@ __global__ void mnn_write_kernel(const unsigned long long* rowk, int64_t n1,
 // and the metric of its brute-force matcher.
 struct FrmState {
   int* err;
-  int32_t* count;   // [B] active seeds
+  // Active seeds of half-step h: list[h % 2] (slots, [B][k], in no particular
+  // order) and cnt[h % 3] ([B]).  The kernel of half-step h appends the
+  // seeds that stay active to list[(h+1) % 2], counting in cnt[(h+1) % 3],
+  // and clears cnt[(h+2) % 3] for the half-step after.
+  int32_t* cnt[3];
   int32_t* nseeds;  // [B] seeds of each pair: the grid size, or its unique starts
   int32_t* U;       // [B][k]
   int32_t* V;
   int32_t* Uold;
   int32_t* Vold;
-  int32_t* list;    // [B][k] active slots, compacted
+  int32_t* list[2];
   int32_t* nq;      // [B][k] queries made per seed
   uint8_t* act;     // [B][k] 1 while active
   unsigned long long* keys;  // [B][k] NN result per list position
@@ -620,14 +624,14 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int
                          rnn_metric metric, FrmState* st, FrmCopies* cp) {
   Carve c(ws);
   st->err = c.take<int>(64);
-  st->count = c.take<int32_t>(B);
+  for (int i = 0; i < 3; ++i) st->cnt[i] = c.take<int32_t>(B);
   st->nseeds = c.take<int32_t>(B);
   const int64_t kk = k > 0 ? k : 1;
   st->U = c.take<int32_t>(B * kk);
   st->V = c.take<int32_t>(B * kk);
   st->Uold = c.take<int32_t>(B * kk);
   st->Vold = c.take<int32_t>(B * kk);
-  st->list = c.take<int32_t>(B * kk);
+  for (int i = 0; i < 2; ++i) st->list[i] = c.take<int32_t>(B * kk);
   st->nq = c.take<int32_t>(B * kk);
   st->act = c.take<uint8_t>(B * kk);
   st->keys = c.take<unsigned long long>(B * kk);
@@ -668,7 +672,7 @@ __device__ __forceinline__ void frm_seed_init(const FrmState& st, int64_t t, int
   st.Uold[t] = u;
   st.V[t] = -1;
   st.Vold[t] = -1;
-  st.list[t] = s;
+  st.list[0][t] = s;
   st.nq[t] = 0;
   st.act[t] = u >= 0 ? 1 : 0;
   st.keys[t] = 0ull;
@@ -696,7 +700,8 @@ __global__ void frm_init_kernel(FrmState st, int W1, int S) {
   }
   if (blockIdx.x == 0) {
     for (int b = threadIdx.x; b < st.B; b += blockDim.x) {
-      st.count[b] = st.k;
+      st.cnt[0][b] = st.k;
+      st.cnt[1][b] = 0;
       st.nseeds[b] = st.k;
     }
     if (threadIdx.x == 0) *st.err = 0;
@@ -756,17 +761,32 @@ __global__ void frm_starts_compact_kernel(FrmState st) {
   // unused slots (duplicated or out-of-image starts)
   for (int s = tot + threadIdx.x; s < st.k; s += blockDim.x) frm_seed_init(st, base + s, s, -1);
   if (threadIdx.x == 0) {
-    st.count[b] = tot;
+    st.cnt[0][b] = tot;
+    st.cnt[1][b] = 0;
     st.nseeds[b] = tot;
   }
 }
 
-// Exact index inside each kept chunk for every active seed of every pair
-// (one warp per seed): NN2 queries are rows U of image 1 against image 2,
-// NN1 queries rows V of image 2 against image 1, in the row forms the
-// tensor cores read.
+// Result of half-step h for every active seed of every pair (one warp per
+// seed).  The warp first resolves the exact index inside the kept chunk
+// (NN2 queries are rows U of image 1 against image 2, NN1 queries rows V of
+// image 2 against image 1, in the row forms the tensor cores read); lane 0
+// then stores the NN found, applies the convergence test, refreshes the old
+// copies at the end of an iteration, and appends the seed to the next list
+// if it stays active.  In basin mode the NN2 half-step deactivates no one and
+// the NN1 half-step records basin[U_old] = U for every seed it served.  A
+// seed's result does not depend on its place in the list, so the order in
+// which the appends land changes nothing.
 template <bool kBf16>
-__global__ void frm_locate_kernel(FrmState st, int nn2_half) {
+__global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter) {
+  const int32_t* cnt_in = st.cnt[h % 3];
+  int32_t* cnt_out = st.cnt[(h + 1) % 3];
+  const int32_t* list_in = st.list[h % 2];
+  int32_t* list_out = st.list[(h + 1) % 2];
+  if (blockIdx.x == 0) {
+    int32_t* cnt_next = st.cnt[(h + 2) % 3];
+    for (int b = threadIdx.x; b < st.B; b += blockDim.x) cnt_next[b] = 0;
+  }
   const int64_t w0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int n_cand = nn2_half ? st.N2 : st.N1;
@@ -774,62 +794,34 @@ __global__ void frm_locate_kernel(FrmState st, int nn2_half) {
   for (int64_t x = w0; x < static_cast<int64_t>(st.B) * st.k; x += nw) {
     const int b = static_cast<int>(x / st.k);
     const int i = static_cast<int>(x - static_cast<int64_t>(b) * st.k);
-    if (i >= st.count[b]) continue;
+    if (i >= cnt_in[b]) continue;
     const int64_t base = static_cast<int64_t>(b) * st.k;
     const uint16_t* Dq = nn2_half ? st.Q1 + b * st.s1 : st.Q2 + b * st.s2;
     const uint16_t* Dx = nn2_half ? st.X2 + b * st.s2 : st.X1 + b * st.s1;
-    const int sl = st.list[base + i];
-    const unsigned long long k = st.keys[base + i];
-    const int64_t qr = rows[base + sl];
-    const int j = locate_chunk<kBf16>(Dq + qr * st.ld, Dx, n_cand, st.ld, key_index(k));
-    if ((threadIdx.x & 31) == 0) st.keys[base + i] = pack_key(key_score(k), j);
-  }
-}
-
-// Result of one half-step for pair blockIdx.x: store the NN found for every
-// active seed, apply the convergence test, refresh the old copies at the end
-// of an iteration, and compact the list of seeds that stay active.  In basin
-// mode the NN2 half-step deactivates no one and the NN1 half-step records
-// basin[U_old] = U for every seed it served.
-__global__ void frm_update_kernel(FrmState st, int nn2_half, int last_iter) {
-  __shared__ int s_out;
-  const int b = blockIdx.x;
-  const int64_t base = static_cast<int64_t>(b) * st.k;
-  const int n = st.count[b];
-  int32_t* basin = st.basin ? st.basin + static_cast<int64_t>(b) * (st.N1 + 1) : nullptr;
-  if (threadIdx.x == 0) s_out = 0;
-  __syncthreads();
-  for (int i0 = 0; i0 < n; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    int s = -1, still = 0;
-    if (i < n) {
-      s = st.list[base + i];
-      const unsigned long long key = st.keys[base + i];
+    const int s = list_in[base + i];
+    const unsigned long long key = st.keys[base + i];
+    const int64_t qr = rows[base + s];
+    const int j = locate_chunk<kBf16>(Dq + qr * st.ld, Dx, n_cand, st.ld, key_index(key));
+    if ((threadIdx.x & 31) == 0) {
       st.keys[base + i] = 0ull;
-      const int j = key_index(key);
       st.nq[base + s] += 1;
+      int still;
       if (nn2_half) {
         st.V[base + s] = j;
-        still = basin ? 1 : j != st.Vold[base + s];
+        still = st.basin ? 1 : j != st.Vold[base + s];
       } else {
         st.U[base + s] = j;
-        if (basin) basin[st.Uold[base + s]] = j;
+        if (st.basin) st.basin[static_cast<int64_t>(b) * (st.N1 + 1) + st.Uold[base + s]] = j;
         still = j != st.Uold[base + s];
         if (still && !last_iter) {
           st.Uold[base + s] = j;
           st.Vold[base + s] = st.V[base + s];
         }
       }
-      if (!still) st.act[base + s] = 0;
+      if (still) list_out[base + atomicAdd(cnt_out + b, 1)] = s;
+      else st.act[base + s] = 0;
     }
-    int tot;
-    const int pos = block_exclusive_scan(still, &tot);  // also orders reads before writes
-    if (still) st.list[base + s_out + pos] = s;
-    __syncthreads();
-    if (threadIdx.x == 0) s_out += tot;
-    __syncthreads();
   }
-  if (threadIdx.x == 0) st.count[b] = s_out;
 }
 
 // Unique output pairs of pair blockIdx.x, sorted by the image-1 pixel.  A
@@ -905,12 +897,12 @@ static int grid_for(int64_t n, int sms) {
   return static_cast<int>(g);
 }
 
-static rnn_status frm_locate(const FrmState& st, int nn2_half, rnn_dtype dt, int grid,
-                             cudaStream_t s) {
+static rnn_status frm_step(const FrmState& st, int h, int nn2_half, int last_iter,
+                           rnn_dtype dt, int grid, cudaStream_t s) {
   if (dt == RNN_BF16)
-    frm_locate_kernel<true><<<grid, kSmallThreads, 0, s>>>(st, nn2_half);
+    frm_step_kernel<true><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter);
   else
-    frm_locate_kernel<false><<<grid, kSmallThreads, 0, s>>>(st, nn2_half);
+    frm_step_kernel<false><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter);
   return launched();
 }
 
@@ -1038,30 +1030,30 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   p.err = st.err;
   NNFamily& F = p.fam[0];
   F.slot_bstride = k;
-  F.q_list = st.list;
-  F.q_count_dev = st.count;
+
   F.nbatch = B;
   F.keys = st.keys;
   F.key_bstride = k;
   for (int it = 1; it <= max_iter; ++it) {
+    const int h = 2 * (it - 1);
     // half-step 1: V = NN2(U)
+    F.q_list = st.list[h % 2];
+    F.q_count_dev = st.cnt[h % 3];
     F.q_base = st.Q1;
     F.q_bstride = st.s1;
     F.q_index = st.U;
     F.n_cand = static_cast<int32_t>(N2);
     if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s)) != RNN_OK) return r;
-    if ((r = frm_locate(st, 1, dt, lgrid, s)) != RNN_OK) return r;
-    frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 1, 0);
-    if ((r = launched()) != RNN_OK) return r;
+    if ((r = frm_step(st, h, 1, 0, dt, lgrid, s)) != RNN_OK) return r;
     // half-step 2: U = NN1(V)
+    F.q_list = st.list[(h + 1) % 2];
+    F.q_count_dev = st.cnt[(h + 1) % 3];
     F.q_base = st.Q2;
     F.q_bstride = st.s2;
     F.q_index = st.V;
     F.n_cand = static_cast<int32_t>(N1);
     if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s)) != RNN_OK) return r;
-    if ((r = frm_locate(st, 0, dt, lgrid, s)) != RNN_OK) return r;
-    frm_update_kernel<<<B, kSmallThreads, 0, s>>>(st, 0, it == max_iter ? 1 : 0);
-    if ((r = launched()) != RNN_OK) return r;
+    if ((r = frm_step(st, h + 1, 0, it == max_iter ? 1 : 0, dt, lgrid, s)) != RNN_OK) return r;
   }
   frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, W1, pairs, cap, count_out, seed_state);
   return launched();
