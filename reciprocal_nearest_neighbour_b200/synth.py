@@ -18,6 +18,13 @@ weights here, so these maps stand in for them:
   the image centre, with fresh random vectors where the source falls outside
   the first image, optionally an occluded rectangle and a share of outlier
   pixels.
+* ``pointmap_pair``: the 3-D inputs, two point maps ``[H][W][3]`` of one
+  smooth surface in the first camera's frame (MASt3R regresses both point
+  maps in that frame): a smooth random depth map back-projected through a
+  pinhole camera, and the same surface sampled at pixel positions moved by a
+  random similarity, plus noise; optionally rounded to multiples of 1/64.
+* ``quantised_points``: ``n`` points with coordinates ``k/64`` in [-16, 16]
+  drawn in clusters, with repeated points (ties).
 
 Arrays are float64 ``[H][W][d]`` (channel-last, row-major, pixel index
 ``y*W + x``) holding values that are exactly representable in the requested
@@ -37,6 +44,8 @@ __all__ = [
     "quantised_map",
     "quantised_pair",
     "smooth_pair",
+    "pointmap_pair",
+    "quantised_points",
     "to_storage",
     "Workload",
     "WORKLOADS",
@@ -137,6 +146,67 @@ def smooth_pair(seed: int, H: int, W: int, d: int, *, sigma: float = 2.0,
 
     d2 = _unit(d2).reshape(H, W, d)
     return d1, d2
+
+
+def pointmap_pair(seed: int, H: int, W: int, *, depth=(2.0, 5.0), sigma: float = 6.0,
+                  noise: float = 0.002, max_rot_deg: float = 10.0,
+                  scale_range=(0.9, 1.1), quantised: bool = False):
+    """Point maps ``P1, P2 [H][W][3]`` (float64) of one smooth surface.
+
+    Depth ``z = depth[0] + (depth[1]-depth[0]) * (field + 2.5)/5`` clipped to
+    the range (``field`` a unit-variance smooth random field), back-projected
+    with focal length ``W`` about the image centre.  P2 samples the same depth
+    at pixel positions moved by a random similarity about the centre (pixels
+    sampled outside the image take the nearest border depth), then adds
+    ``noise`` to every coordinate of both maps.  ``quantised`` rounds every
+    coordinate to a multiple of 1/64 (then all squared distances are exact in
+    fp32; the coordinates stay inside [-16, 16] for the default depths).
+
+    Draw order from ``default_rng(seed)``: field (H*W normals), rotation,
+    log-scale, P1 noise, P2 noise.
+    """
+    rng = np.random.default_rng(seed)
+    field = _smooth_field(rng, H, W, 1, sigma)[..., 0]
+    z = depth[0] + (depth[1] - depth[0]) * np.clip((field + 2.5) / 5.0, 0.0, 1.0)
+    theta = math.radians(rng.uniform(-max_rot_deg, max_rot_deg))
+    scale = math.exp(rng.uniform(math.log(scale_range[0]), math.log(scale_range[1])))
+    f = float(W)
+    cx, cy = (W - 1) / 2.0, (H - 1) / 2.0
+    ys, xs = np.mgrid[0:H, 0:W].astype(np.float64)
+
+    def backproject(u, v, zz):
+        return np.stack([(u - cx) * zz / f, (v - cy) * zz / f, zz], axis=-1)
+
+    p1 = backproject(xs, ys, z)
+    c, s = math.cos(theta), math.sin(theta)
+    px, py = xs - cx, ys - cy
+    sx = np.clip(cx + scale * (c * px - s * py), 0, W - 1)
+    sy = np.clip(cy + scale * (s * px + c * py), 0, H - 1)
+    z2 = _bilinear(z[..., None], sx.reshape(-1), sy.reshape(-1)).reshape(H, W)
+    p2 = backproject(sx, sy, z2)
+    p1 = p1 + noise * rng.standard_normal(p1.shape)
+    p2 = p2 + noise * rng.standard_normal(p2.shape)
+    if quantised:
+        p1 = np.clip(_round_half_away(p1 * 64.0), -1024, 1024) / 64.0
+        p2 = np.clip(_round_half_away(p2 * 64.0), -1024, 1024) / 64.0
+    return p1, p2
+
+
+def quantised_points(rng: np.random.Generator, n: int, clusters: int = 8,
+                     spread: float = 1.5, repeat: float = 0.05) -> np.ndarray:
+    """``[n][3]`` points ``k/64`` in [-16, 16]: Gaussian clusters (centres
+    uniform in [-12, 12]^3, standard deviation ``spread``), then a share
+    ``repeat`` of the points replaced by copies of earlier ones."""
+    centres = rng.uniform(-12.0, 12.0, size=(clusters, 3))
+    which = rng.integers(0, clusters, size=n)
+    p = centres[which] + spread * rng.standard_normal((n, 3))
+    p = np.clip(_round_half_away(p * 64.0), -1024, 1024) / 64.0
+    nrep = int(round(repeat * n))
+    if nrep and n > 1:
+        dst = rng.integers(1, n, size=nrep)
+        src = (rng.random(nrep) * dst).astype(np.int64)
+        p[dst] = p[src]
+    return p
 
 
 def to_storage(a: np.ndarray, dtype: str):

@@ -411,3 +411,98 @@ def test_basin_matches_numpy_replay_and_plain_frm(S, max_iter):
     assert np.array_equal(r.basin, basin)
     # skipping the first half-step's test changes no output pair
     assert np.array_equal(r.pairs, oracle.frm(D1, D2, S, max_iter).pairs)
+
+
+# ------------------------------------------------------------------ 3-D points
+# MASt3R's NN function on 3-D points is a K-d tree query (scipy's cKDTree
+# here): the oracle's Euclidean metric at d = 3 must give its answers.
+
+def test_points_nn_matches_kdtree():
+    from scipy.spatial import cKDTree
+
+    rng = np.random.default_rng(123)
+    X = rng.standard_normal((3000, 3)) * np.array([3.0, 2.0, 1.0])
+    Q = rng.standard_normal((1000, 3)) * 4.0            # some queries far outside
+    r = oracle.nn(Q, X, metric="l2")
+    dist, idx = cKDTree(X).query(Q)
+    assert np.array_equal(r.arg, idx)
+    assert np.allclose(-r.best, dist ** 2, rtol=1e-12, atol=0.0)
+
+
+def test_points_nn_ties_lowest_index_via_ball_query():
+    """Repeated points and equal distances: the distance is the tree's, and
+    the index is the lowest of all points at that distance (a ball query
+    collects them; their squared distances are compared as integers)."""
+    from scipy.spatial import cKDTree
+
+    rng = np.random.default_rng(124)
+    X = synth.quantised_points(rng, 2000, repeat=0.2)
+    Q = synth.quantised_points(rng, 400)
+    Q[:50] = X[rng.integers(0, len(X), 50)]               # queries on data points
+    r = oracle.nn(Q, X, metric="l2")
+    tree = cKDTree(X)
+    dist, _ = tree.query(Q)
+    assert np.allclose(-r.best, dist ** 2, rtol=1e-12, atol=0.0)
+    Xi, Qi = np.rint(X * 64).astype(np.int64), np.rint(Q * 64).astype(np.int64)
+    for t in range(len(Q)):
+        near = np.array(tree.query_ball_point(Q[t], dist[t] * (1 + 1e-9) + 1e-12))
+        d2 = ((Xi[near] - Qi[t]) ** 2).sum(axis=1)
+        low = near[d2 == d2.min()].min()
+        assert r.arg[t] == low, t
+        assert -r.best[t] * 4096 == d2.min()
+
+
+def _frm_kdtree(P1, P2, seeds, max_iter):
+    """The FRM loop on point maps with K-d tree queries as the NN function,
+    written out (grid seeds, V = NN2(U), U = NN1(V), the two convergence
+    tests, max_iter), as the quoted function runs it on the CPU."""
+    from scipy.spatial import cKDTree
+
+    A, B = P1.reshape(-1, 3), P2.reshape(-1, 3)
+    t1, t2 = cKDTree(A), cKDTree(B)
+    U = seeds.astype(np.int64).copy()
+    V = np.full_like(U, -1)
+    Uold, Vold = U.copy(), V.copy()
+    active = np.ones(len(U), bool)
+    for it in range(max_iter):
+        idx = np.nonzero(active)[0]
+        if len(idx) == 0:
+            break
+        V[idx] = t2.query(A[U[idx]])[1]
+        active[idx] = V[idx] != Vold[idx]
+        idx = np.nonzero(active)[0]
+        U[idx] = t1.query(B[V[idx]])[1]
+        active[idx] = U[idx] != Uold[idx]
+        Uold, Vold = U.copy(), V.copy()
+    return sorted({(int(U[s]), int(V[s])) for s in range(len(U)) if not active[s]})
+
+
+@pytest.mark.parametrize("S,max_iter", [(4, 10), (2, 3), (1, 10)])
+def test_points_frm_matches_kdtree_replay(S, max_iter):
+    P1, P2 = synth.pointmap_pair(51 + S, 24, 32, noise=0.01)
+    r = oracle.frm_ex(P1, P2, S, max_iter, metric="l2")
+    ref = _frm_kdtree(P1, P2, oracle.frm_seeds(24, 32, S), max_iter)
+    assert [tuple(p) for p in r.pairs.tolist()] == ref
+    assert len(ref) > 0
+
+
+def test_points_mnn_matches_kdtree():
+    from scipy.spatial import cKDTree
+
+    P1, P2 = synth.pointmap_pair(60, 20, 28, noise=0.01)
+    A, B = P1.reshape(-1, 3), P2.reshape(-1, 3)
+    r = oracle.mnn(P1, P2, metric="l2")
+    ra, ca = cKDTree(B).query(A)[1], cKDTree(A).query(B)[1]
+    assert np.array_equal(r.row.arg, ra) and np.array_equal(r.col.arg, ca)
+    mutual = [(i, int(ra[i])) for i in range(len(ra)) if ca[ra[i]] == i]
+    assert [tuple(p) for p in r.pairs.tolist()] == mutual
+
+
+def test_pointmap_generator_ranges():
+    P1, P2 = synth.pointmap_pair(3, 48, 64, quantised=True)
+    for P in (P1, P2):
+        assert P.shape == (48, 64, 3)
+        assert np.abs(P).max() <= 16.0
+        assert np.array_equal(P * 64, np.rint(P * 64))
+    Q = synth.quantised_points(np.random.default_rng(1), 1000)
+    assert np.abs(Q).max() <= 16.0 and np.array_equal(Q * 64, np.rint(Q * 64))
