@@ -243,6 +243,60 @@ rnn_status rnn_frm_match_ex(int B, const void *D1, int64_t d1_batch_stride, cons
                             size_t ws_bytes, rnn_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * 3-D points.  MASt3R picks the NN function of reciprocal matching by the
+ * dimension of its input, and matches 3-D points (its point maps) with K-d
+ * trees (MASt3R paper text quoted in the staskaer.github.io DUSt3R/MASt3R
+ * blog, MASt3R matching section).  These entry points compute the same
+ * thing: the exact nearest point in Euclidean distance, lowest index on
+ * ties, and with it the reciprocal set and FRM on point maps.
+ *
+ *   points     fp32 [n][3] (x, y, z), 4-byte aligned DEVICE pointers (RNN_EALIGN
+ *              otherwise); point maps [H][W][3], pixel p = y*W + x.
+ *   distances  squared Euclidean distances, computed in fp32 as
+ *              fma(dz, dz, fma(dy, dy, dx*dx)) with d = q - x; the NN is the
+ *              lowest index with the smallest such value.  On coordinates that
+ *              are multiples of 2^-6 within [-16, 16] every such value is
+ *              exact (each partial result is a multiple of 2^-12 below 2^12).
+ *   sizes      at most 2^28 points per set (RNN_EUNSUPPORTED above).
+ *   inputs     finite; NaN or Inf gives undefined matches (but valid indices
+ *              and no out-of-bounds access).
+ *   time       a uniform grid over each set's bounding box (cells of about
+ *              two point spacings on a surface through the box): a query
+ *              visits a few cells on point maps of surfaces; a query far from
+ *              the set, or a set with most points in a few cells, costs up to
+ *              a pass over every point.
+ *
+ * rnn_pts_nn: NN of each of the nq query points among the nx >= 1 points of
+ *   X.  idx_out [nq] int32, dist2_out [nq] float (may be NULL).  nq may be 0.
+ *   7 kernel launches (6 when nq = 0).
+ * rnn_pts_mnn: the reciprocal set between two point maps; outputs as
+ *   rnn_mnn_exhaustive, with squared distances in rowd2_out / cold2_out.
+ *   9 kernel launches.
+ * rnn_pts_frm_match: FRM over B pairs of point maps with every option of
+ *   rnn_frm_match_ex (batch strides in floats, at least 3*H*W; init_xy1,
+ *   n_init, pixel_tol, basin_out, cap and seed_state_out as there).
+ *   rnn_pts_frm_workspace_size takes n_init = starts per pair, or -1 for the
+ *   grid of stride seed_stride.  8 + 2*max_iter kernel launches (2 more with
+ *   given starts).
+ */
+size_t rnn_pts_nn_workspace_size(int64_t nq, int64_t nx);
+rnn_status rnn_pts_nn(const float *Q, int64_t nq, const float *X, int64_t nx, int32_t *idx_out,
+                      float *dist2_out, void *workspace, size_t ws_bytes, rnn_stream_t stream);
+size_t rnn_pts_mnn_workspace_size(int H1, int W1, int H2, int W2);
+rnn_status rnn_pts_mnn(const float *P1, int H1, int W1, const float *P2, int H2, int W2,
+                       int32_t *pairs_out, int64_t cap, int32_t *count_out, int32_t *rowarg_out,
+                       float *rowd2_out, int32_t *colarg_out, float *cold2_out, void *workspace,
+                       size_t ws_bytes, rnn_stream_t stream);
+size_t rnn_pts_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int seed_stride,
+                                  int64_t n_init);
+rnn_status rnn_pts_frm_match(int B, const float *P1, int64_t p1_batch_stride, const float *P2,
+                             int64_t p2_batch_stride, int H1, int W1, int H2, int W2,
+                             const int32_t *init_xy1, int64_t n_init, int seed_stride,
+                             int max_iter, float pixel_tol, int32_t *pairs_out, int64_t cap,
+                             int32_t *count_out, int32_t *seed_state_out, int32_t *basin_out,
+                             void *workspace, size_t ws_bytes, rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Nearest neighbours without any allocation.  (The matching method itself
  * has no counterpart of this: it exists for callers, not for the algorithm.)
  *

@@ -21,6 +21,9 @@ contiguous fp16/bf16 CUDA tensors; pixel index ``p = y*W + x``.
 * ``metric="l2"`` (``nn_argmax``, ``mnn_exhaustive``, ``frm_match_ex``,
   ``frm_refine``): the smallest Euclidean distance instead of the largest dot
   product; scores are then squared distances.
+* ``pts_nn`` / ``pts_mnn`` / ``pts_frm_match``: the same operations on 3-D
+  points (fp32 ``[..., 3]``), where MASt3R's NN function is the exact nearest
+  point in Euclidean distance (a K-d tree query in its reference code).
 
 Results stay on the device; pair lists come back as ``(pairs, count)`` with
 ``pairs`` a ``[cap, 2]`` int32 buffer and ``count`` a device int32 tensor;
@@ -39,7 +42,8 @@ from ._lib import RNNError, RNNLibraryError  # noqa: F401
 __all__ = [
     "nn_argmax", "mnn_exhaustive", "frm_match", "frm_match_batched", "frm_num_seeds",
     "frm_max_pairs", "workspace_status", "trim", "MNNResult", "FRMResult", "RNNError",
-    "RNNLibraryError", "FRMPlan", "frm_match_ex", "frm_refine",
+    "RNNLibraryError", "FRMPlan", "frm_match_ex", "frm_refine", "pts_nn", "pts_mnn",
+    "pts_frm_match",
 ]
 
 _DT = {torch.float16: _lib.RNN_F16, torch.bfloat16: _lib.RNN_BF16}
@@ -338,3 +342,99 @@ def frm_refine(D1: torch.Tensor, D2: torch.Tensor, init: torch.Tensor, pixel_tol
     (exactly, or within ``pixel_tol`` pixels)."""
     return frm_match_ex(D1, D2, max_iter=1, metric=metric, init=init, pixel_tol=pixel_tol,
                         with_seed_state=with_seed_state)
+
+
+# ------------------------------------------------------------------ 3-D points
+
+def _check_points(t: torch.Tensor, name: str, ndim: int) -> None:
+    _check_map(t, name, ndim)
+    if t.dtype != torch.float32 or t.shape[-1] != 3:
+        raise ValueError(f"{name} must be float32 [..., 3], got {t.dtype} {tuple(t.shape)}")
+
+
+def pts_nn(Q: torch.Tensor, X: torch.Tensor, *, workspace: Optional[torch.Tensor] = None):
+    """Nearest point of ``X [nx, 3]`` to each of ``Q [nq, 3]`` (Euclidean,
+    lowest index on ties).  Returns ``(idx int32 [nq], squared distance
+    float32 [nq])``."""
+    _check_points(Q, "Q", 2)
+    _check_points(X, "X", 2)
+    lib = _lib.load()
+    nq, nx = Q.shape[0], X.shape[0]
+    idx = torch.empty(nq, dtype=torch.int32, device=Q.device)
+    d2 = torch.empty(nq, dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(lib.rnn_pts_nn_workspace_size(nq, nx), Q.device)
+    _lib.check(lib.rnn_pts_nn(Q.data_ptr(), nq, X.data_ptr(), nx, idx.data_ptr(), d2.data_ptr(),
+                              workspace.data_ptr(), workspace.numel(), _stream(Q)), "rnn_pts_nn")
+    return idx, d2
+
+
+def pts_mnn(P1: torch.Tensor, P2: torch.Tensor, *, with_nn: bool = False,
+            workspace: Optional[torch.Tensor] = None) -> MNNResult:
+    """Reciprocal set between point maps ``P1 [H1, W1, 3]`` and ``P2 [H2, W2, 3]``;
+    ``rowmax``/``colmax`` hold squared distances."""
+    _check_points(P1, "P1", 3)
+    _check_points(P2, "P2", 3)
+    lib = _lib.load()
+    H1, W1, _ = P1.shape
+    H2, W2, _ = P2.shape
+    n1, n2 = H1 * W1, H2 * W2
+    dev = P1.device
+    out = MNNResult(torch.empty((min(n1, n2), 2), dtype=torch.int32, device=dev),
+                    torch.zeros(1, dtype=torch.int32, device=dev))
+    if with_nn:
+        out.rowarg = torch.empty(n1, dtype=torch.int32, device=dev)
+        out.rowmax = torch.empty(n1, dtype=torch.float32, device=dev)
+        out.colarg = torch.empty(n2, dtype=torch.int32, device=dev)
+        out.colmax = torch.empty(n2, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _workspace(lib.rnn_pts_mnn_workspace_size(H1, W1, H2, W2), dev)
+    _lib.check(lib.rnn_pts_mnn(
+        P1.data_ptr(), H1, W1, P2.data_ptr(), H2, W2, out.pairs.data_ptr(), out.pairs.shape[0],
+        out.count.data_ptr(), _ptr(out.rowarg), _ptr(out.rowmax), _ptr(out.colarg),
+        _ptr(out.colmax), workspace.data_ptr(), workspace.numel(), _stream(P1)), "rnn_pts_mnn")
+    return out
+
+
+def pts_frm_match(P1: torch.Tensor, P2: torch.Tensor, *, seed_stride: int = 8,
+                  max_iter: int = 10, init: Optional[torch.Tensor] = None,
+                  pixel_tol: float = 0.0, with_basin: bool = False,
+                  with_seed_state: bool = False,
+                  workspace: Optional[torch.Tensor] = None) -> FRMResult:
+    """FRM on point maps ``[H, W, 3]`` or ``[B, H, W, 3]`` (fp32), with the
+    options of ``frm_match_ex``."""
+    batched = P1.dim() == 4
+    _check_points(P1, "P1", 4 if batched else 3)
+    _check_points(P2, "P2", 4 if batched else 3)
+    if batched and P1.shape[0] != P2.shape[0]:
+        raise ValueError("P1 and P2 must share B")
+    B = P1.shape[0] if batched else 1
+    H1, W1, _ = P1.shape[-3:]
+    H2, W2, _ = P2.shape[-3:]
+    lib = _lib.load()
+    dev = P1.device
+    n_init = -1
+    if init is not None:
+        if not isinstance(init, torch.Tensor) or not init.is_cuda or init.dtype != torch.int32:
+            raise ValueError("init must be a CUDA int32 tensor")
+        init = init.reshape(B, -1).contiguous()
+        n_init = init.shape[1]
+        k = n_init
+    else:
+        k = int(lib.rnn_frm_num_seeds(H1, W1, seed_stride)) if seed_stride >= 1 else 0
+    cap = max(1, k if pixel_tol > 0 else min(k, H2 * W2))
+    out = FRMResult(torch.empty((B, cap, 2), dtype=torch.int32, device=dev),
+                    torch.zeros(B, dtype=torch.int32, device=dev),
+                    torch.empty((B, max(k, 1), 4), dtype=torch.int32, device=dev)
+                    if with_seed_state else None,
+                    torch.empty((B, H1 * W1 + 1), dtype=torch.int32, device=dev)
+                    if with_basin else None)
+    if workspace is None:
+        workspace = _workspace(lib.rnn_pts_frm_workspace_size(B, H1, W1, H2, W2, seed_stride,
+                                                              n_init), dev)
+    _lib.check(lib.rnn_pts_frm_match(
+        B, P1.data_ptr(), H1 * W1 * 3, P2.data_ptr(), H2 * W2 * 3, H1, W1, H2, W2, _ptr(init),
+        max(n_init, 0), seed_stride, max_iter, float(pixel_tol), out.pairs.data_ptr(), cap,
+        out.count.data_ptr(), _ptr(out.seed_state), _ptr(out.basin), workspace.data_ptr(),
+        workspace.numel(), _stream(P1)), "rnn_pts_frm_match")
+    return out

@@ -34,6 +34,12 @@ EXPORTS = (
     "rnn_mnn_exhaustive_ex",
     "rnn_frm_workspace_size_ex",
     "rnn_frm_match_ex",
+    "rnn_pts_nn_workspace_size",
+    "rnn_pts_nn",
+    "rnn_pts_mnn_workspace_size",
+    "rnn_pts_mnn",
+    "rnn_pts_frm_workspace_size",
+    "rnn_pts_frm_match",
 )
 
 STATUS = {
@@ -100,6 +106,13 @@ def load():
         "rnn_frm_workspace_size_ex": (SZ, [I, I, I, I, I, I, I, I, I64]),
         "rnn_frm_match_ex": (I, [I, P, I64, P, I64, I, I, I, I, I, I, I, P, I64, I, I,
                                  ctypes.c_float, P, I64, P, P, P, P, SZ, P]),
+        "rnn_pts_nn_workspace_size": (SZ, [I64, I64]),
+        "rnn_pts_nn": (I, [P, I64, P, I64, P, P, P, SZ, P]),
+        "rnn_pts_mnn_workspace_size": (SZ, [I, I, I, I]),
+        "rnn_pts_mnn": (I, [P, I, I, P, I, I, P, I64, P, P, P, P, P, P, SZ, P]),
+        "rnn_pts_frm_workspace_size": (SZ, [I, I, I, I, I, I, I64]),
+        "rnn_pts_frm_match": (I, [I, P, I64, P, I64, I, I, I, I, P, I64, I, I, ctypes.c_float,
+                                  P, I64, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

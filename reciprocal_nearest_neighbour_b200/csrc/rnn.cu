@@ -638,10 +638,10 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int
   const int64_t nwords = (N1 + 31) / 32;
   st->bitmap = c.take<uint32_t>(B * nwords);
   st->partner = c.take<int32_t>(B * N1);
-  const int mode = copies_for(d, metric);
-  const int kpad = tile_depth(d, metric);
+  const int mode = d > 0 ? copies_for(d, metric) : kCopiesNone;  // d = 0: point maps
   cp->q1 = cp->x1 = cp->q2 = cp->x2 = nullptr;
   if (mode != kCopiesNone) {
+    const int kpad = tile_depth(d, metric);
     cp->q1 = c.take<uint16_t>(B * N1 * kpad);
     cp->q2 = c.take<uint16_t>(B * N2 * kpad);
     cp->x1 = cp->q1;
@@ -767,16 +767,39 @@ __global__ void frm_starts_compact_kernel(FrmState st) {
   }
 }
 
+// Result j of a half-step for seed slot s of pair b: store the NN found,
+// apply the convergence test, refresh the old copies at the end of an
+// iteration, and append the seed to the next list if it stays active.  In
+// basin mode the NN2 half-step deactivates no one and the NN1 half-step
+// records basin[U_old] = U for every seed it served.  A seed's result does not
+// depend on its place in the list, so the order in which the appends land
+// changes nothing.
+__device__ __forceinline__ void frm_apply(const FrmState& st, int b, int64_t base, int s, int j,
+                                          int nn2_half, int last_iter, int32_t* list_out,
+                                          int32_t* cnt_out) {
+  st.nq[base + s] += 1;
+  int still;
+  if (nn2_half) {
+    st.V[base + s] = j;
+    still = st.basin ? 1 : j != st.Vold[base + s];
+  } else {
+    st.U[base + s] = j;
+    if (st.basin) st.basin[static_cast<int64_t>(b) * (st.N1 + 1) + st.Uold[base + s]] = j;
+    still = j != st.Uold[base + s];
+    if (still && !last_iter) {
+      st.Uold[base + s] = j;
+      st.Vold[base + s] = st.V[base + s];
+    }
+  }
+  if (still) list_out[base + atomicAdd(cnt_out + b, 1)] = s;
+  else st.act[base + s] = 0;
+}
+
 // Result of half-step h for every active seed of every pair (one warp per
-// seed).  The warp first resolves the exact index inside the kept chunk
-// (NN2 queries are rows U of image 1 against image 2, NN1 queries rows V of
-// image 2 against image 1, in the row forms the tensor cores read); lane 0
-// then stores the NN found, applies the convergence test, refreshes the old
-// copies at the end of an iteration, and appends the seed to the next list
-// if it stays active.  In basin mode the NN2 half-step deactivates no one and
-// the NN1 half-step records basin[U_old] = U for every seed it served.  A
-// seed's result does not depend on its place in the list, so the order in
-// which the appends land changes nothing.
+// seed): the warp resolves the exact index inside the kept chunk (NN2
+// queries are rows U of image 1 against image 2, NN1 queries rows V of image
+// 2 against image 1, in the row forms the tensor cores read), then lane 0
+// applies it (frm_apply).
 template <bool kBf16>
 __global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter) {
   const int32_t* cnt_in = st.cnt[h % 3];
@@ -804,22 +827,7 @@ __global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter)
     const int j = locate_chunk<kBf16>(Dq + qr * st.ld, Dx, n_cand, st.ld, key_index(key));
     if ((threadIdx.x & 31) == 0) {
       st.keys[base + i] = 0ull;
-      st.nq[base + s] += 1;
-      int still;
-      if (nn2_half) {
-        st.V[base + s] = j;
-        still = st.basin ? 1 : j != st.Vold[base + s];
-      } else {
-        st.U[base + s] = j;
-        if (st.basin) st.basin[static_cast<int64_t>(b) * (st.N1 + 1) + st.Uold[base + s]] = j;
-        still = j != st.Uold[base + s];
-        if (still && !last_iter) {
-          st.Uold[base + s] = j;
-          st.Vold[base + s] = st.V[base + s];
-        }
-      }
-      if (still) list_out[base + atomicAdd(cnt_out + b, 1)] = s;
-      else st.act[base + s] = 0;
+      frm_apply(st, b, base, s, j, nn2_half, last_iter, list_out, cnt_out);
     }
   }
 }
@@ -890,6 +898,13 @@ __global__ void frm_merge_kernel(FrmState st, int W1, int32_t* pairs, int64_t ca
   if (threadIdx.x == 0) count_out[b] = tot;
 }
 
+}  // namespace rnn
+
+// 3-D point kernels (they use FrmState, frm_apply and block_exclusive_scan)
+#include "points.cuh"
+
+namespace rnn {
+
 static int grid_for(int64_t n, int sms) {
   int64_t g = (n + kSmallThreads - 1) / kSmallThreads;
   if (g > 4LL * sms) g = 4LL * sms;
@@ -925,6 +940,30 @@ static rnn_status prep_rows(const void* src, int64_t bstride, int64_t rows, int 
   else
     prep_rows_kernel<false><<<grid, kSmallThreads, 0, s>>>(in, bstride, rows, nbatch, d, dst,
                                                           kpad, form);
+  return launched();
+}
+
+// Seeds of every pair: the grid of stride S, or the given starts made
+// unique and ascending; state, bitmaps and basin array cleared.
+static rnn_status frm_seed(const FrmState& st, const int32_t* init, int64_t n_init, int W1,
+                           int S, DeviceInfo* di, cudaStream_t s) {
+  const int64_t B = st.B, k = st.k;
+  const int64_t nbasin = st.basin ? B * (static_cast<int64_t>(st.N1) + 1) : 0;
+  rnn_status r;
+  if (init) {
+    frm_starts_clear_kernel<<<grid_for(B * st.nwords + nbasin, di->sms), kSmallThreads, 0, s>>>(
+        st);
+    if ((r = launched()) != RNN_OK) return r;
+    if (n_init > 0) {
+      frm_starts_mark_kernel<<<grid_for(B * n_init, di->sms), kSmallThreads, 0, s>>>(st, init,
+                                                                                    n_init);
+      if ((r = launched()) != RNN_OK) return r;
+    }
+    frm_starts_compact_kernel<<<static_cast<int>(B), kSmallThreads, 0, s>>>(st);
+  } else {
+    frm_init_kernel<<<grid_for(B * k + B * st.nwords + nbasin, di->sms), kSmallThreads, 0, s>>>(
+        st, W1, S);
+  }
   return launched();
 }
 
@@ -1005,21 +1044,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   if ((r = make_map(&map1, st.X1, st.ld, N1, B, st.s1, g)) != RNN_OK) return r;
   if ((r = make_map(&map2, st.X2, st.ld, N2, B, st.s2, g)) != RNN_OK) return r;
 
-  if (init) {
-    frm_starts_clear_kernel<<<grid_for(B * st.nwords + (basin ? B * (N1 + 1) : 0), di->sms),
-                              kSmallThreads, 0, s>>>(st);
-    if ((r = launched()) != RNN_OK) return r;
-    if (n_init > 0) {
-      frm_starts_mark_kernel<<<grid_for(B * n_init, di->sms), kSmallThreads, 0, s>>>(st, init,
-                                                                                    n_init);
-      if ((r = launched()) != RNN_OK) return r;
-    }
-    frm_starts_compact_kernel<<<B, kSmallThreads, 0, s>>>(st);
-  } else {
-    frm_init_kernel<<<grid_for(B * k + B * st.nwords + (basin ? B * (N1 + 1) : 0), di->sms),
-                      kSmallThreads, 0, s>>>(st, W1, S);
-  }
-  if ((r = launched()) != RNN_OK) return r;
+  if ((r = frm_seed(st, init, n_init, W1, S, di, s)) != RNN_OK) return r;
   const int lgrid = grid_for(static_cast<int64_t>(B) * k * 32, di->sms);
 
   NNParams p;
@@ -1059,6 +1084,171 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   return launched();
 }
 
+// ------------------------------------------------------------- 3-D points
+constexpr int64_t kPtsMaxSet = 1 << 28;  // points per set
+
+struct PtsWs {
+  float* part;      // [nblocks][6] block bounding boxes
+  PtsGrid* grids;   // [nsets]
+  int32_t* start;   // [nstart] cell counts, then the first sorted point of each cell
+  int32_t* cell;    // [npts] global cell of each point
+  int32_t* rank;    // [npts] its rank in the cell
+  int32_t* seg;     // [nseg] segment sums of the prefix sum
+  float4* sorted;   // [npts] (x, y, z, index bits) in cell order
+  int64_t nstart = 0, npts = 0;
+  int nblocks = 0, nseg = 0;
+};
+
+// nb sets of n0 points (family 0) and, with nfam = 2, nb sets of n1 points.
+static PtsSets pts_sets(const float* b0, int64_t s0, int64_t n0, const float* b1, int64_t s1,
+                        int64_t n1, int nb, int nfam) {
+  PtsSets ps;
+  std::memset(&ps, 0, sizeof(ps));
+  ps.nb = nb;
+  ps.nfam = nfam;
+  const float* base[2] = {b0, b1};
+  const int64_t bs[2] = {s0, s1}, n[2] = {n0, n1};
+  for (int f = 0; f < nfam; ++f) {
+    ps.base[f] = base[f];
+    ps.bstride[f] = bs[f];
+    ps.n[f] = static_cast<int>(n[f]);
+    ps.cap[f] = static_cast<int>(2 * n[f] + 64);
+    ps.blk[f] = static_cast<int>((n[f] + kPtsChunk - 1) / kPtsChunk);
+  }
+  return ps;
+}
+
+static size_t pts_layout(Carve& c, const PtsSets& ps, PtsWs* w) {
+  int64_t cells = 0, npts = 0, nblocks = 0;
+  for (int f = 0; f < ps.nfam; ++f) {
+    cells += static_cast<int64_t>(ps.nb) * ps.cap[f];
+    npts += static_cast<int64_t>(ps.nb) * ps.n[f];
+    nblocks += static_cast<int64_t>(ps.nb) * ps.blk[f];
+  }
+  w->nstart = cells + 1;
+  w->npts = npts;
+  w->nblocks = static_cast<int>(nblocks);
+  w->nseg = static_cast<int>((w->nstart + kScanSeg - 1) / kScanSeg);
+  w->part = c.take<float>(6 * nblocks);
+  w->grids = c.take<PtsGrid>(pts_nsets(ps));
+  w->start = c.take<int32_t>(w->nstart);
+  w->cell = c.take<int32_t>(npts);
+  w->rank = c.take<int32_t>(npts);
+  w->seg = c.take<int32_t>(w->nseg);
+  w->sorted = c.take<float4>(npts);
+  return c.off;
+}
+
+// Sizes the shared arrays can index (int32 cells and sorted positions).
+static bool pts_fits(const PtsSets& ps) {
+  PtsWs w;
+  Carve c(nullptr);
+  pts_layout(c, ps, &w);
+  return w.nstart <= INT32_MAX && w.npts <= INT32_MAX;
+}
+
+static bool pts_ptr_ok(const float* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Grids of every set: bounds, cells and ranks, prefix sum, scatter.
+static rnn_status pts_build(const PtsSets& ps, const PtsWs& w, int* err, DeviceInfo* di,
+                            cudaStream_t s) {
+  rnn_status r;
+  pts_bounds_kernel<<<w.nblocks, kPtsThreads, 0, s>>>(ps, w.part, w.start, w.nstart, err);
+  if ((r = launched()) != RNN_OK) return r;
+  pts_count_kernel<<<w.nblocks, kPtsThreads, 0, s>>>(ps, w.part, w.grids, w.start, w.cell,
+                                                     w.rank);
+  if ((r = launched()) != RNN_OK) return r;
+  pts_scan_sum_kernel<<<w.nseg, kScanThreads, 0, s>>>(w.start, w.nstart, w.seg);
+  if ((r = launched()) != RNN_OK) return r;
+  pts_scan_seg_kernel<<<1, kScanThreads, 0, s>>>(w.seg, w.nseg);
+  if ((r = launched()) != RNN_OK) return r;
+  pts_scan_apply_kernel<<<w.nseg, kScanThreads, 0, s>>>(w.start, w.nstart, w.seg);
+  if ((r = launched()) != RNN_OK) return r;
+  pts_scatter_kernel<<<grid_for(w.npts, di->sms), kSmallThreads, 0, s>>>(ps, w.start, w.cell,
+                                                                         w.rank, w.sorted,
+                                                                         w.npts);
+  return launched();
+}
+
+// Blocks of kPtsThreads for one thread per query, grid-stride beyond 8 per SM.
+static int pts_query_grid(int64_t n, int sms) {
+  int64_t g = (n + kPtsThreads - 1) / kPtsThreads;
+  if (g > 8LL * sms) g = 8LL * sms;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+static size_t pts_frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, FrmState* st,
+                             PtsSets* ps, PtsWs* w) {
+  FrmCopies cp;
+  const size_t off = frm_layout(ws, B, k, N1, N2, 0, RNN_L2, st, &cp);
+  Carve c(ws);
+  c.off = off;
+  *ps = pts_sets(nullptr, 3 * N1, N1, nullptr, 3 * N2, N2, B, 2);
+  return pts_layout(c, *ps, w);
+}
+
+// FRM on point maps: as frm_run, with the NN of each half-step found by the
+// grid search (frm_pts_step_kernel) instead of the tensor-core kernel.
+static rnn_status frm_run_pts(int B, const float* P1, int64_t bs1, const float* P2, int64_t bs2,
+                              int H1, int W1, int H2, int W2, const int32_t* init,
+                              int64_t n_init, int S, int max_iter, float pixel_tol,
+                              int32_t* pairs, int64_t cap, int32_t* count_out,
+                              int32_t* seed_state, int32_t* basin, void* ws, size_t ws_bytes,
+                              cudaStream_t s) {
+  if (B < 1) return RNN_EINVAL;
+  if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
+  if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || max_iter < 1) return RNN_EINVAL;
+  if (init ? n_init < 0 : S < 1) return RNN_EINVAL;
+  if (!(pixel_tol >= 0.f) || (pixel_tol > 0.f && !init)) return RNN_EINVAL;
+  if (!P1 || !P2) return RNN_EINVAL;
+  if (!pts_ptr_ok(P1) || !pts_ptr_ok(P2)) return RNN_EALIGN;
+  const int64_t N1 = static_cast<int64_t>(H1) * W1, N2 = static_cast<int64_t>(H2) * W2;
+  if (N1 > kPtsMaxSet || N2 > kPtsMaxSet) return RNN_EUNSUPPORTED;
+  if (bs1 < 3 * N1 || bs2 < 3 * N2) return RNN_EINVAL;
+  if (!pairs || !count_out) return RNN_EINVAL;
+  const int64_t k = init ? n_init : num_seeds(H1, W1, S);
+  if (k > INT32_MAX) return RNN_EINVAL;
+  const int64_t need = pixel_tol > 0.f ? k : (k < N2 ? k : N2);
+  if (cap < need) return RNN_ECAPACITY;
+  FrmState st;
+  PtsSets ps;
+  PtsWs w;
+  const size_t bytes = pts_frm_layout(nullptr, B, k, N1, N2, &st, &ps, &w);
+  if (!pts_fits(ps)) return RNN_EUNSUPPORTED;
+  if (!ws || !aligned256(ws) || ws_bytes < bytes) return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  rnn_status r = device_info(&di);
+  if (r != RNN_OK) return r;
+  pts_frm_layout(ws, B, k, N1, N2, &st, &ps, &w);
+  ps.base[0] = P1;
+  ps.base[1] = P2;
+  ps.bstride[0] = bs1;
+  ps.bstride[1] = bs2;
+  st.basin = basin;
+  st.pixel_tol = pixel_tol;
+  st.starts = init ? 1 : 0;
+  if (k == 0) {
+    if (cudaMemsetAsync(count_out, 0, sizeof(int32_t) * B, s) != cudaSuccess) return RNN_ECUDA;
+    if (cudaMemsetAsync(st.err, 0, sizeof(int), s) != cudaSuccess) return RNN_ECUDA;
+    if (basin && cudaMemsetAsync(basin, 0xFF, sizeof(int32_t) * B * (N1 + 1), s) != cudaSuccess)
+      return RNN_ECUDA;
+    return RNN_OK;
+  }
+  if ((r = frm_seed(st, init, n_init, W1, S, di, s)) != RNN_OK) return r;
+  if ((r = pts_build(ps, w, nullptr, di, s)) != RNN_OK) return r;
+  const int qg = pts_query_grid(static_cast<int64_t>(B) * k, di->sms);
+  for (int it = 1; it <= max_iter; ++it) {
+    const int h = 2 * (it - 1);
+    frm_pts_step_kernel<<<qg, kPtsThreads, 0, s>>>(st, ps, w.grids, w.sorted, w.start, h, 1, 0);
+    if ((r = launched()) != RNN_OK) return r;
+    frm_pts_step_kernel<<<qg, kPtsThreads, 0, s>>>(st, ps, w.grids, w.sorted, w.start, h + 1, 0,
+                                                   it == max_iter ? 1 : 0);
+    if ((r = launched()) != RNN_OK) return r;
+  }
+  frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, W1, pairs, cap, count_out, seed_state);
+  return launched();
+}
+
 }  // namespace rnn
 
 // ====================================================================== ABI
@@ -1080,7 +1270,7 @@ const char* rnn_status_string(rnn_status s) {
   return "unknown rnn_status";
 }
 
-int rnn_abi_version(void) { return 2; }
+int rnn_abi_version(void) { return 3; }
 
 uint64_t rnn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -1413,6 +1603,133 @@ rnn_status rnn_frm_match_ex(int B, const void* D1, int64_t d1_batch_stride, cons
                  init_xy1, n_init, seed_stride, max_iter, pixel_tol, pairs_out, cap, count_out,
                  seed_state_out, basin_out, workspace, ws_bytes,
                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------- 3-D points
+static size_t pts_nn_layout(void* ws, int64_t nq, int64_t nx, int** err, PtsSets* ps,
+                            PtsWs* w) {
+  Carve c(ws);
+  *err = c.take<int>(64);
+  (void)nq;
+  *ps = pts_sets(nullptr, 3 * nx, nx, nullptr, 0, 0, 1, 1);
+  return pts_layout(c, *ps, w);
+}
+
+size_t rnn_pts_nn_workspace_size(int64_t nq, int64_t nx) {
+  int* e;
+  PtsSets ps;
+  PtsWs w;
+  return pts_nn_layout(nullptr, nq > 0 ? nq : 0, nx > 0 ? nx : 1, &e, &ps, &w);
+}
+
+rnn_status rnn_pts_nn(const float* Q, int64_t nq, const float* X, int64_t nx, int32_t* idx_out,
+                      float* dist2_out, void* workspace, size_t ws_bytes, rnn_stream_t stream) {
+  if (nq < 0 || nx < 1 || nq > INT32_MAX) return RNN_EINVAL;
+  if (nx > kPtsMaxSet) return RNN_EUNSUPPORTED;
+  if (!X || (nq > 0 && (!Q || !idx_out))) return RNN_EINVAL;
+  if (!pts_ptr_ok(X) || (nq > 0 && !pts_ptr_ok(Q))) return RNN_EALIGN;
+  if (!workspace || !aligned256(workspace) || ws_bytes < rnn_pts_nn_workspace_size(nq, nx))
+    return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  rnn_status r = device_info(&di);
+  if (r != RNN_OK) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* err;
+  PtsSets ps;
+  PtsWs w;
+  pts_nn_layout(workspace, nq, nx, &err, &ps, &w);
+  ps.base[0] = X;
+  if ((r = pts_build(ps, w, err, di, s)) != RNN_OK) return r;
+  if (nq == 0) return RNN_OK;
+  PtsQuery q{Q, nq, 0, idx_out, dist2_out, nullptr};
+  pts_query_kernel<<<pts_query_grid(nq, di->sms), kPtsThreads, 0, s>>>(q, q, 1, w.grids,
+                                                                        w.sorted, w.start);
+  return launched();
+}
+
+static size_t pts_mnn_layout(void* ws, int64_t n1, int64_t n2, MnnWs* m, PtsSets* ps, PtsWs* w) {
+  Carve c(ws);
+  m->err = c.take<int>(64);
+  m->rowk = c.take<unsigned long long>(n1 > 0 ? n1 : 1);
+  m->colk = c.take<unsigned long long>(n2 > 0 ? n2 : 1);
+  m->counts = c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
+  *ps = pts_sets(nullptr, 3 * n1, n1, nullptr, 3 * n2, n2, 1, 2);
+  return pts_layout(c, *ps, w);
+}
+
+size_t rnn_pts_mnn_workspace_size(int H1, int W1, int H2, int W2) {
+  const int64_t n1 = static_cast<int64_t>(H1 > 0 ? H1 : 1) * (W1 > 0 ? W1 : 1);
+  const int64_t n2 = static_cast<int64_t>(H2 > 0 ? H2 : 1) * (W2 > 0 ? W2 : 1);
+  MnnWs m;
+  PtsSets ps;
+  PtsWs w;
+  return pts_mnn_layout(nullptr, n1, n2, &m, &ps, &w);
+}
+
+rnn_status rnn_pts_mnn(const float* P1, int H1, int W1, const float* P2, int H2, int W2,
+                       int32_t* pairs_out, int64_t cap, int32_t* count_out, int32_t* rowarg_out,
+                       float* rowd2_out, int32_t* colarg_out, float* cold2_out, void* workspace,
+                       size_t ws_bytes, rnn_stream_t stream) {
+  if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0) return RNN_EINVAL;
+  if (!P1 || !P2 || !pairs_out || !count_out) return RNN_EINVAL;
+  if (!pts_ptr_ok(P1) || !pts_ptr_ok(P2)) return RNN_EALIGN;
+  const int64_t n1 = static_cast<int64_t>(H1) * W1, n2 = static_cast<int64_t>(H2) * W2;
+  if (n1 > kPtsMaxSet || n2 > kPtsMaxSet) return RNN_EUNSUPPORTED;
+  if (cap < (n1 < n2 ? n1 : n2)) return RNN_ECAPACITY;
+  if (!workspace || !aligned256(workspace) ||
+      ws_bytes < rnn_pts_mnn_workspace_size(H1, W1, H2, W2))
+    return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  rnn_status r = device_info(&di);
+  if (r != RNN_OK) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MnnWs m;
+  PtsSets ps;
+  PtsWs w;
+  pts_mnn_layout(workspace, n1, n2, &m, &ps, &w);
+  ps.base[0] = P1;
+  ps.base[1] = P2;
+  if ((r = pts_build(ps, w, m.err, di, s)) != RNN_OK) return r;
+  // sweep 1: points of image 1 in the image-2 grid (set 1) -> NN2; sweep 2
+  // the other way -> NN1
+  PtsQuery q1{P1, n1, 1, nullptr, nullptr, m.rowk};
+  PtsQuery q2{P2, n2, 0, nullptr, nullptr, m.colk};
+  pts_query_kernel<<<pts_query_grid(n1 + n2, di->sms), kPtsThreads, 0, s>>>(
+      q1, q2, 2, w.grids, w.sorted, w.start);
+  if ((r = launched()) != RNN_OK) return r;
+  const int nblk1 = static_cast<int>((n1 + kMnnChunk - 1) / kMnnChunk);
+  const int nblk2 = static_cast<int>((n2 + kMnnChunk - 1) / kMnnChunk);
+  const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
+  mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(m.rowk, n1, m.colk, n2, m.counts, nblk1,
+                                                rowarg_out, rowd2_out, colarg_out, cold2_out);
+  if ((r = launched()) != RNN_OK) return r;
+  mnn_write_kernel<<<nblk1, kSmallThreads, 0, s>>>(m.rowk, n1, m.colk, m.counts, nblk1,
+                                                   pairs_out, count_out);
+  return launched();
+}
+
+size_t rnn_pts_frm_workspace_size(int B, int H1, int W1, int H2, int W2, int seed_stride,
+                                  int64_t n_init) {
+  if (B < 1) B = 1;
+  const int64_t N1 = static_cast<int64_t>(H1 > 0 ? H1 : 1) * (W1 > 0 ? W1 : 1);
+  const int64_t N2 = static_cast<int64_t>(H2 > 0 ? H2 : 1) * (W2 > 0 ? W2 : 1);
+  const int64_t k = n_init >= 0 ? n_init : (seed_stride >= 1 ? num_seeds(H1, W1, seed_stride) : 0);
+  FrmState st;
+  PtsSets ps;
+  PtsWs w;
+  return pts_frm_layout(nullptr, B, k, N1, N2, &st, &ps, &w);
+}
+
+rnn_status rnn_pts_frm_match(int B, const float* P1, int64_t p1_batch_stride, const float* P2,
+                             int64_t p2_batch_stride, int H1, int W1, int H2, int W2,
+                             const int32_t* init_xy1, int64_t n_init, int seed_stride,
+                             int max_iter, float pixel_tol, int32_t* pairs_out, int64_t cap,
+                             int32_t* count_out, int32_t* seed_state_out, int32_t* basin_out,
+                             void* workspace, size_t ws_bytes, rnn_stream_t stream) {
+  return frm_run_pts(B, P1, p1_batch_stride, P2, p2_batch_stride, H1, W1, H2, W2, init_xy1,
+                     n_init, seed_stride, max_iter, pixel_tol, pairs_out, cap, count_out,
+                     seed_state_out, basin_out, workspace, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

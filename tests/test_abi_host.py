@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rnn_abi_version() == 2
+    assert lib.rnn_abi_version() == 3
     for code, name in _lib.STATUS.items():
         assert lib.rnn_status_string(code).decode().startswith(name)
 
@@ -185,3 +185,65 @@ def test_frm_ex_argument_errors(lib):
     mnn = lib.rnn_mnn_exhaustive_ex
     assert mnn(FAKE, 4, 4, FAKE, 4, 4, 16, 0, 9, FAKE, 16, FAKE, None, None, None, None, FAKE,
                1 << 20, None) == EINVAL
+
+
+def test_pts_workspace_sizes(lib):
+    n = 384 * 512
+    nn = lib.rnn_pts_nn_workspace_size(1000, n)
+    # sorted points (16 bytes), cell and rank (4 + 4) and about 2 cells per point
+    assert nn >= n * (16 + 8) + 2 * n * 4
+    mnn = lib.rnn_pts_mnn_workspace_size(384, 512, 384, 512)
+    assert mnn >= 2 * n * (16 + 8 + 8) + 4 * n * 4
+    one = lib.rnn_pts_frm_workspace_size(1, 384, 512, 384, 512, 8, -1)
+    many = lib.rnn_pts_frm_workspace_size(4, 384, 512, 384, 512, 8, -1)
+    assert many > 3 * one
+    assert lib.rnn_pts_frm_workspace_size(1, 384, 512, 384, 512, 0, 500) > 0
+    for v in (nn, mnn, one, many):
+        assert v % 256 == 0
+
+
+def test_pts_argument_errors(lib):
+    ws = lib.rnn_pts_nn_workspace_size(10, 10)
+    nn = lib.rnn_pts_nn
+    assert nn(FAKE, 10, FAKE, 0, FAKE, None, FAKE, ws, None) == EINVAL
+    assert nn(FAKE, -1, FAKE, 10, FAKE, None, FAKE, ws, None) == EINVAL
+    assert nn(None, 10, FAKE, 10, FAKE, None, FAKE, ws, None) == EINVAL
+    assert nn(FAKE, 10, None, 10, FAKE, None, FAKE, ws, None) == EINVAL
+    assert nn(FAKE, 10, FAKE, 10, None, None, FAKE, ws, None) == EINVAL
+    assert nn(FAKE + 2, 10, FAKE, 10, FAKE, None, FAKE, ws, None) == EALIGN
+    assert nn(FAKE, 10, FAKE, (1 << 28) + 1, FAKE, None, FAKE, 1 << 40, None) == EUNSUP
+    assert nn(FAKE, 10, FAKE, 10, FAKE, None, FAKE, ws - 4, None) == EWS
+    assert nn(FAKE, 10, FAKE, 10, FAKE, None, FAKE + 16, ws, None) == EWS
+
+    wm = lib.rnn_pts_mnn_workspace_size(4, 4, 4, 4)
+    mnn = lib.rnn_pts_mnn
+    assert mnn(FAKE, 0, 4, FAKE, 4, 4, FAKE, 16, FAKE, None, None, None, None, FAKE, wm,
+               None) == EINVAL
+    assert mnn(FAKE, 4, 4, FAKE + 1, 4, 4, FAKE, 16, FAKE, None, None, None, None, FAKE, wm,
+               None) == EALIGN
+    assert mnn(FAKE, 4, 4, FAKE, 4, 4, FAKE, 15, FAKE, None, None, None, None, FAKE, wm,
+               None) == ECAP
+    assert mnn(FAKE, 4, 4, FAKE, 4, 4, FAKE, 16, FAKE, None, None, None, None, FAKE, wm - 1,
+               None) == EWS
+
+    wf = lib.rnn_pts_frm_workspace_size(2, 8, 8, 8, 8, 2, -1)
+    f = lib.rnn_pts_frm_match
+
+    def call(**kw):
+        a = dict(B=2, P1=FAKE, s1=8 * 8 * 3, P2=FAKE, s2=8 * 8 * 3, H1=8, W1=8, H2=8, W2=8,
+                 init=None, n=0, S=2, it=10, tol=0.0, pairs=FAKE, cap=16, count=FAKE, ws=FAKE,
+                 wsb=wf)
+        a.update(kw)
+        return f(a["B"], a["P1"], a["s1"], a["P2"], a["s2"], a["H1"], a["W1"], a["H2"],
+                 a["W2"], a["init"], a["n"], a["S"], a["it"], a["tol"], a["pairs"], a["cap"],
+                 a["count"], None, None, a["ws"], a["wsb"], None)
+
+    assert call(B=0) == EINVAL
+    assert call(B=_lib.RNN_MAX_BATCH + 1) == EUNSUP
+    assert call(S=0) == EINVAL
+    assert call(it=0) == EINVAL
+    assert call(tol=1.0) == EINVAL                  # a tolerance needs given starts
+    assert call(s1=8 * 8 * 3 - 1) == EINVAL
+    assert call(P2=FAKE + 2) == EALIGN
+    assert call(cap=15) == ECAP
+    assert call(wsb=wf - 1) == EWS
