@@ -32,8 +32,8 @@ import time
 # the fused kernel in the bench step, from one ncu capture of the step's
 # first FRM call (20 launches averaged).  It belongs to the kernel sources it
 # was taken on: with any other sources the bench reports traffic as null.
-TRAFFIC = {"sources_sha256": "bc38bcce7e358f6b8e111af581462b336795c3a8ef7103877e8ad4560c70ded4",
-           "frm_nn_bytes_per_launch": 37.33e6}
+TRAFFIC = {"sources_sha256": "cadc7e907d68d3620a1a24cd60b4b5f86bd577ea1a0381a1339a3c076e8cea32",
+           "frm_nn_bytes_per_launch": 37.24e6}
 
 
 def _kernel_sources_sha256() -> str:
@@ -437,6 +437,47 @@ def run_native(args):
                              "outputs": int(r.count.sum().item()),
                              "note": "includes the binding's output and workspace allocation"}
 
+    # ------------------------- 3-D point maps (the K-d tree workload, exact NN)
+    pts = None
+    if not args.skip_mnn:
+        pts = {}
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        pm = [synth.pointmap_pair(700 + i, w.H, w.W) for i in range(P)]
+        p1 = torch.from_numpy(np.stack([m[0] for m in pm]).astype(np.float32)).to(dev)
+        p2 = torch.from_numpy(np.stack([m[1] for m in pm]).astype(np.float32)).to(dev)
+        n1 = w.H * w.W
+        ws_m = torch.empty(lib.rnn_pts_mnn_workspace_size(w.H, w.W, w.H, w.W),
+                           dtype=torch.uint8, device=dev)
+        ws_f = torch.empty(lib.rnn_pts_frm_workspace_size(P, w.H, w.W, w.H, w.W,
+                                                          w.seed_stride, -1),
+                           dtype=torch.uint8, device=dev)
+        cases = (("mnn", lambda: rnn.pts_mnn(p1[0], p2[0], workspace=ws_m), 2 * n1,
+                  "queries/s", "exhaustive reciprocal set of two 512x384 point maps "
+                  "(both directions)"),
+                 ("frm", lambda: rnn.pts_frm_match(p1, p2, seed_stride=w.seed_stride,
+                                                   max_iter=w.max_iter, workspace=ws_f),
+                  P, "pairs/s", f"FRM on {P} pairs of 512x384 point maps, stride "
+                  f"{w.seed_stride}, max_iter {w.max_iter}"))
+        for name, fn, units, unit, what in cases:
+            for _ in range(3):
+                r = fn()
+            reps = 10
+            oa = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            ob = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+            for i in range(reps):
+                flush.fill_(i & 0xFF)
+                oa[i].record()
+                r = fn()
+                ob[i].record()
+            torch.cuda.synchronize()
+            ms = statistics.median(_event_ms(oa, ob, reps))
+            pts[name] = {"metric": what, "value": units / (ms * 1e-3), "unit": unit,
+                         "ms_per_call": ms, "outputs": int(r.count.sum().item()),
+                         "dtype": "f32",
+                         "note": "includes the binding's output allocation; 256 MB L2 flush "
+                                 "before every call"}
+        del flush
+
     # ----------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -456,7 +497,7 @@ def run_native(args):
                        "global_batch": world * P, "parallelism": f"replicas x{world}",
                        "l2": f"step inputs {2 * A_h.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
             "e2e": e2e, "roofline": roofline, "mnn": mnn, "frm_options": options,
-            "cpu_baseline": cpu,
+            "points": pts, "cpu_baseline": cpu,
             "clocks": clocks, "gpu_launches": int(launches),
         }
         print(json.dumps(line), flush=True)
