@@ -25,6 +25,14 @@ What each function computes, with its source:
   unique and sorted), the ``pixel_tol`` convergence rule that returns the
   start pixel, the basin output, and the Euclidean-distance metric of its
   brute-force matcher (``metric="l2"``; also for ``nn`` and ``mnn``).
+* ``c2f_crops`` / ``c2f``: coarse-to-fine matching (cv-learn.com "MASt3R"
+  note, paragraph "Coarse-to-fine matching"; staskaer.github.io blog, the
+  step after FRM that returns to full resolution and matches again block by
+  block): the reciprocal set of the coarse maps, crops of image 1 on a grid,
+  each paired with a crop of image 2 centred on its coarse matches, FRM per
+  crop pair on the full-resolution maps, and the matches mapped back.  The
+  pages give no formulas for the crops; the integer rules written out in
+  ``c2f_crops`` are this implementation's reading.
 """
 from __future__ import annotations
 
@@ -270,3 +278,95 @@ def frm_refine(D1, D2, init, pixel_tol: float = 0.0, metric: str = "dot",
     (``max_iter`` = 1), the ``pixel_tol`` rule, (start, match) pairs."""
     return frm_ex(D1, D2, init=init, max_iter=1, pixel_tol=pixel_tol, metric=metric,
                   threads=threads)
+
+
+# --------------------------------------------------------- coarse-to-fine
+
+def c2f_crop_origins(L: int, c: int) -> list:
+    """Origins of the ceil(L/c) crops of length c that cover [0, L), the first
+    at 0 and the last at L - c, spread evenly (floor)."""
+    n = -(-L // c)
+    if n <= 1:
+        return [0]
+    return [(a * (L - c)) // (n - 1) for a in range(n)]
+
+
+def c2f_fine_pixel(i: int, Hc: int, Wc: int, H: int, W: int):
+    """Full-resolution (y, x) of the centre of coarse pixel i = yc*Wc + xc:
+    floor((2*yc + 1) * H / (2*Hc)), floor((2*xc + 1) * W / (2*Wc))."""
+    yc, xc = divmod(int(i), Wc)
+    return ((2 * yc + 1) * H) // (2 * Hc), ((2 * xc + 1) * W) // (2 * Wc)
+
+
+def c2f_crop_size(H1, W1, H2, W2, crop):
+    ch, cw = crop
+    return min(ch, H1, H2), min(cw, W1, W2)
+
+
+def c2f_crops(coarse_pairs, Hc1, Wc1, Hc2, Wc2, H1, W1, H2, W2, crop, min_coarse=1):
+    """Crop table ``int32 [n][6]``: y0_1, x0_1, y0_2, x0_2, n_coarse, on.
+
+    Crops of image 1 are the row-major grid of ``c2f_crop_origins`` along each
+    axis.  A coarse pair (i, j) belongs to crop b when the full-resolution
+    pixel of i lies inside it.  With n >= min_coarse such pairs, crop b is on
+    and its image-2 crop is centred on the floor of the mean full-resolution
+    position of their j, clamped into image 2; otherwise it is off (origin
+    0, 0) and is not matched."""
+    ch, cw = c2f_crop_size(H1, W1, H2, W2, crop)
+    ys, xs = c2f_crop_origins(H1, ch), c2f_crop_origins(W1, cw)
+    p1 = [c2f_fine_pixel(i, Hc1, Wc1, H1, W1) for i, _ in coarse_pairs]
+    p2 = [c2f_fine_pixel(j, Hc2, Wc2, H2, W2) for _, j in coarse_pairs]
+    rows = []
+    for y0 in ys:
+        for x0 in xs:
+            inside = [t for t, (y, x) in enumerate(p1) if y0 <= y < y0 + ch and x0 <= x < x0 + cw]
+            n = len(inside)
+            if n >= max(min_coarse, 1):
+                cy = sum(p2[t][0] for t in inside) // n
+                cx = sum(p2[t][1] for t in inside) // n
+                y2 = min(max(cy - ch // 2, 0), H2 - ch)
+                x2 = min(max(cx - cw // 2, 0), W2 - cw)
+                rows.append((y0, x0, y2, x2, n, 1))
+            else:
+                rows.append((y0, x0, 0, 0, n, 0))
+    return np.array(rows, dtype=np.int32).reshape(-1, 6)
+
+
+@dataclass
+class C2FResult:
+    pairs: np.ndarray    # int32 [n][2] full-resolution (u, v), one per u, sorted by u
+    crops: np.ndarray    # int32 [ncrops][6] (see c2f_crops)
+    coarse: np.ndarray   # int32 [m][2] reciprocal pairs of the coarse maps
+
+
+def c2f(C1, C2, F1, F2, crop=(384, 512), seed_stride: int = 8, max_iter: int = 10,
+        min_coarse: int = 1, metric: str = "dot", threads: int = 0) -> C2FResult:
+    """Coarse-to-fine matching of full-resolution maps F1, F2 ``[H][W][d]``
+    guided by coarse maps C1, C2 ``[Hc][Wc][dc]``: M of the coarse maps
+    (``mnn``), the crop table (``c2f_crops``), FRM with grid seeds of stride
+    ``seed_stride`` on every crop pair that is on (``frm_ex``), each pair
+    mapped back by its crops' origins; where crops overlap, the first crop
+    in table order that outputs an image-1 pixel gives its pair."""
+    c1, c2 = as_f64(C1), as_f64(C2)
+    f1, f2 = as_f64(F1), as_f64(F2)
+    Hc1, Wc1, _ = c1.shape
+    Hc2, Wc2, _ = c2.shape
+    H1, W1, _ = f1.shape
+    H2, W2, _ = f2.shape
+    coarse = mnn(c1, c2, threads=threads, metric=metric).pairs
+    crops = c2f_crops(coarse.tolist(), Hc1, Wc1, Hc2, Wc2, H1, W1, H2, W2, crop, min_coarse)
+    ch, cw = c2f_crop_size(H1, W1, H2, W2, crop)
+    best = {}
+    for y0, x0, y2, x2, _, on in crops.tolist():
+        if not on:
+            continue
+        a = f1[y0:y0 + ch, x0:x0 + cw]
+        b = f2[y2:y2 + ch, x2:x2 + cw]
+        r = frm_ex(a, b, seed_stride, max_iter, metric=metric, threads=threads)
+        for u, v in r.pairs.tolist():
+            gu = (y0 + u // cw) * W1 + (x0 + u % cw)
+            gv = (y2 + v // cw) * W2 + (x2 + v % cw)
+            if gu not in best:
+                best[gu] = gv
+    pairs = np.array(sorted(best.items()), dtype=np.int32).reshape(-1, 2)
+    return C2FResult(pairs, crops, coarse)

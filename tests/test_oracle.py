@@ -506,3 +506,54 @@ def test_pointmap_generator_ranges():
         assert np.array_equal(P * 64, np.rint(P * 64))
     Q = synth.quantised_points(np.random.default_rng(1), 1000)
     assert np.abs(Q).max() <= 16.0 and np.array_equal(Q * 64, np.rint(Q * 64))
+
+
+# ------------------------------------------------------------- coarse-to-fine
+
+def test_golden_c2f_crops(golden_dir):
+    g = _load(golden_dir, "c2f_crops_8x12.json")
+    for L, c, want in g["origins"]:
+        assert oracle.c2f_crop_origins(L, c) == want
+    for i, Hc, Wc, H, W, want in g["fine_pixel"]:
+        assert list(oracle.c2f_fine_pixel(i, Hc, Wc, H, W)) == want
+    sizes = (g["Hc1"], g["Wc1"], g["Hc2"], g["Wc2"], g["H1"], g["W1"], g["H2"], g["W2"])
+    for m, key in ((1, "crops_min1"), (2, "crops_min2")):
+        t = oracle.c2f_crops(g["coarse"], *sizes, tuple(g["crop"]), min_coarse=m)
+        assert t.tolist() == g[key]
+
+
+def _pool(D, s):
+    """Mean over s x s pixel blocks, renormalised (the coarse stand-in)."""
+    H, W, d = D.shape
+    P = D[: H // s * s, : W // s * s].reshape(H // s, s, W // s, s, d).mean(axis=(1, 3))
+    return P / np.linalg.norm(P, axis=-1, keepdims=True)
+
+
+def test_c2f_one_crop_is_plain_frm():
+    """A crop as large as the images leaves one crop pair, (0,0)-(0,0): the
+    result is FRM on the full-resolution maps."""
+    F1, F2 = synth.smooth_pair(21, 24, 32, 16)
+    C1, C2 = _pool(F1, 4), _pool(F2, 4)
+    r = oracle.c2f(C1, C2, F1, F2, crop=(64, 64), seed_stride=3, max_iter=10)
+    assert r.crops.tolist() == [[0, 0, 0, 0, len(r.coarse), 1]]
+    assert np.array_equal(r.pairs, oracle.frm_ex(F1, F2, 3, 10).pairs)
+
+
+def test_c2f_pairs_are_mutual_in_their_crops():
+    F1, F2 = synth.smooth_pair(22, 40, 48, 16)
+    C1, C2 = _pool(F1, 4), _pool(F2, 4)
+    crop = (16, 20)
+    r = oracle.c2f(C1, C2, F1, F2, crop=crop, seed_stride=2, max_iter=10)
+    assert len(r.pairs) > 50 and r.crops[:, 5].sum() >= 4
+    W1 = W2 = 48
+    seen = set()
+    for y0, x0, y2, x2, n, on in r.crops.tolist():
+        if not on:
+            continue
+        a, b = F1[y0:y0 + 16, x0:x0 + 20], F2[y2:y2 + 16, x2:x2 + 20]
+        m = oracle.mnn(a, b)
+        for u, v in m.pairs.tolist():
+            seen.add(((y0 + u // 20) * W1 + x0 + u % 20, (y2 + v // 20) * W2 + x2 + v % 20))
+    # every output pair is a reciprocal pair of some crop pair's windows
+    assert all((int(u), int(v)) in seen for u, v in r.pairs)
+    assert np.all(np.diff(r.pairs[:, 0]) > 0)
