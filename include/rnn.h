@@ -243,6 +243,56 @@ rnn_status rnn_frm_match_ex(int B, const void *D1, int64_t d1_batch_stride, cons
                             size_t ws_bytes, rnn_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Coarse-to-fine matching (cv-learn.com "MASt3R" note, paragraph
+ * "Coarse-to-fine matching": high-resolution images are matched coarsely
+ * first, the coarse matches guide the matching of enumerated local crops,
+ * and the fine matches are mapped back to full resolution; the
+ * staskaer.github.io DUSt3R/MASt3R blog describes the same step as matching
+ * again block by block at full resolution).  The pages give no formulas for
+ * the crops; these integer rules are this library's:
+ *
+ *   coarse     M of the coarse maps C1 [Hc1][Wc1][dc], C2 [Hc2][Wc2][dc]
+ *              (rnn_mnn_exhaustive_ex with `metric`).
+ *   pixel      coarse pixel (yc, xc) of an Hc x Wc map stands for the
+ *              full-resolution pixel (floor((2yc+1)H/(2Hc)), floor((2xc+1)W/(2Wc))).
+ *   crops      ch = min(crop_h, H1, H2), cw = min(crop_w, W1, W2); image 1 is
+ *              covered by ceil(H1/ch) x ceil(W1/cw) crops, row-major, at
+ *              origins floor(a*(L-c)/(n-1)) along each axis (0 when n = 1).
+ *              At most RNN_MAX_BATCH crops (RNN_EUNSUPPORTED).
+ *   pairing    crop b holds the coarse pairs whose image-1 pixel lies inside
+ *              it; with at least max(min_coarse, 1) of them it is on, and its
+ *              image-2 crop is centred on the floor of the mean of their
+ *              image-2 pixels, clamped into image 2.
+ *   fine       FRM (grid seeds of stride seed_stride inside the crop,
+ *              max_iter) between the windows of F1 [H1][W1][d] and F2
+ *              [H2][W2][d] of every crop pair that is on, batched.
+ *   output     each pair mapped back by its crops' origins; where crops
+ *              overlap, the lowest crop index that outputs an image-1 pixel
+ *              gives its pair; pairs_out [cap][2] sorted by the image-1
+ *              pixel, count_out [1].  cap >= rnn_c2f_max_pairs(...).
+ *   crops_out  NULL or device int32 [ncrops][6]: y0_1, x0_1, y0_2, x0_2,
+ *              coarse pairs inside, on.
+ * All four maps share dtype; C1/C2 and F1/F2 follow the descriptor rules
+ * (16-byte aligned, dc and d multiples of 8).  rnn_workspace_status() on the
+ * workspace reports a timed-out wait of any part.  No host synchronisation;
+ * 13 + 4*max_iter kernel launches, plus the row copies: 2 when dc needs
+ * padding (dc = 8, 24, 40, ...), and with RNN_L2 4 for the coarse and 4 for
+ * the fine Euclidean forms.
+ */
+int rnn_c2f_num_crops(int H1, int W1, int H2, int W2, int crop_h, int crop_w);
+int64_t rnn_c2f_max_pairs(int H1, int W1, int H2, int W2, int crop_h, int crop_w,
+                          int seed_stride);
+size_t rnn_c2f_workspace_size(int Hc1, int Wc1, int Hc2, int Wc2, int dc, int H1, int W1,
+                              int H2, int W2, int d, rnn_metric metric, int crop_h, int crop_w,
+                              int seed_stride);
+rnn_status rnn_c2f_match(const void *C1, int Hc1, int Wc1, const void *C2, int Hc2, int Wc2,
+                         int dc, const void *F1, int H1, int W1, const void *F2, int H2, int W2,
+                         int d, rnn_dtype dtype, rnn_metric metric, int crop_h, int crop_w,
+                         int seed_stride, int max_iter, int min_coarse, int32_t *pairs_out,
+                         int64_t cap, int32_t *count_out, int32_t *crops_out, void *workspace,
+                         size_t ws_bytes, rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * 3-D points.  MASt3R picks the NN function of reciprocal matching by the
  * dimension of its input, and matches 3-D points (its point maps) with K-d
  * trees (MASt3R paper text quoted in the staskaer.github.io DUSt3R/MASt3R

@@ -21,6 +21,9 @@ contiguous fp16/bf16 CUDA tensors; pixel index ``p = y*W + x``.
 * ``metric="l2"`` (``nn_argmax``, ``mnn_exhaustive``, ``frm_match_ex``,
   ``frm_refine``): the smallest Euclidean distance instead of the largest dot
   product; scores are then squared distances.
+* ``c2f_match``: coarse-to-fine matching: the reciprocal set of coarse maps
+  places crop pairs, FRM runs on the full-resolution windows, and the pairs
+  are mapped back (cv-learn.com "MASt3R" note, "Coarse-to-fine matching").
 * ``pts_nn`` / ``pts_mnn`` / ``pts_frm_match``: the same operations on 3-D
   points (fp32 ``[..., 3]``), where MASt3R's NN function is the exact nearest
   point in Euclidean distance (a K-d tree query in its reference code).
@@ -43,7 +46,7 @@ __all__ = [
     "nn_argmax", "mnn_exhaustive", "frm_match", "frm_match_batched", "frm_num_seeds",
     "frm_max_pairs", "workspace_status", "trim", "MNNResult", "FRMResult", "RNNError",
     "RNNLibraryError", "FRMPlan", "frm_match_ex", "frm_refine", "pts_nn", "pts_mnn",
-    "pts_frm_match",
+    "pts_frm_match", "c2f_match", "C2FResult",
 ]
 
 _DT = {torch.float16: _lib.RNN_F16, torch.bfloat16: _lib.RNN_BF16}
@@ -437,4 +440,52 @@ def pts_frm_match(P1: torch.Tensor, P2: torch.Tensor, *, seed_stride: int = 8,
         max(n_init, 0), seed_stride, max_iter, float(pixel_tol), out.pairs.data_ptr(), cap,
         out.count.data_ptr(), _ptr(out.seed_state), _ptr(out.basin), workspace.data_ptr(),
         workspace.numel(), _stream(P1)), "rnn_pts_frm_match")
+    return out
+
+
+# ------------------------------------------------------------ coarse-to-fine
+
+@dataclass
+class C2FResult:
+    pairs: torch.Tensor    # [cap, 2] int32 full-resolution (image-1, image-2) pixels
+    count: torch.Tensor    # [1] int32
+    crops: torch.Tensor    # [ncrops, 6]: y0_1, x0_1, y0_2, x0_2, coarse pairs inside, on
+
+    def trimmed(self) -> torch.Tensor:
+        return trim(self.pairs, self.count)
+
+
+def c2f_match(C1: torch.Tensor, C2: torch.Tensor, F1: torch.Tensor, F2: torch.Tensor, *,
+              crop=(384, 512), seed_stride: int = 8, max_iter: int = 10, min_coarse: int = 1,
+              metric: str = "dot", workspace: Optional[torch.Tensor] = None) -> C2FResult:
+    """Coarse-to-fine matching of full-resolution maps ``F1 [H1, W1, d]``,
+    ``F2 [H2, W2, d]`` guided by coarse maps ``C1 [Hc1, Wc1, dc]``,
+    ``C2 [Hc2, Wc2, dc]`` (all one dtype); ``crop`` is ``(height, width)``."""
+    for t, n in ((C1, "C1"), (C2, "C2"), (F1, "F1"), (F2, "F2")):
+        _check_map(t, n, 3)
+    if len({C1.dtype, C2.dtype, F1.dtype, F2.dtype}) != 1:
+        raise ValueError("all four maps must share one dtype")
+    if C1.shape[2] != C2.shape[2] or F1.shape[2] != F2.shape[2]:
+        raise ValueError("C1/C2 and F1/F2 must share their depth")
+    lib = _lib.load()
+    Hc1, Wc1, dc = C1.shape
+    Hc2, Wc2, _ = C2.shape
+    H1, W1, d = F1.shape
+    H2, W2, _ = F2.shape
+    ch, cw = int(crop[0]), int(crop[1])
+    m = _metric(metric)
+    dev = F1.device
+    nc = int(lib.rnn_c2f_num_crops(H1, W1, H2, W2, ch, cw))
+    cap = max(1, int(lib.rnn_c2f_max_pairs(H1, W1, H2, W2, ch, cw, seed_stride)))
+    out = C2FResult(torch.empty((cap, 2), dtype=torch.int32, device=dev),
+                    torch.zeros(1, dtype=torch.int32, device=dev),
+                    torch.empty((max(nc, 1), 6), dtype=torch.int32, device=dev))
+    if workspace is None:
+        workspace = _workspace(lib.rnn_c2f_workspace_size(Hc1, Wc1, Hc2, Wc2, dc, H1, W1, H2,
+                                                          W2, d, m, ch, cw, seed_stride), dev)
+    _lib.check(lib.rnn_c2f_match(
+        C1.data_ptr(), Hc1, Wc1, C2.data_ptr(), Hc2, Wc2, dc, F1.data_ptr(), H1, W1,
+        F2.data_ptr(), H2, W2, d, _dtype_code(F1), m, ch, cw, seed_stride, max_iter, min_coarse,
+        out.pairs.data_ptr(), cap, out.count.data_ptr(), out.crops.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(F1)), "rnn_c2f_match")
     return out

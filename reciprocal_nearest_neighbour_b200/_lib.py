@@ -40,6 +40,10 @@ EXPORTS = (
     "rnn_pts_mnn",
     "rnn_pts_frm_workspace_size",
     "rnn_pts_frm_match",
+    "rnn_c2f_num_crops",
+    "rnn_c2f_max_pairs",
+    "rnn_c2f_workspace_size",
+    "rnn_c2f_match",
 )
 
 STATUS = {
@@ -113,6 +117,11 @@ def load():
         "rnn_pts_frm_workspace_size": (SZ, [I, I, I, I, I, I, I64]),
         "rnn_pts_frm_match": (I, [I, P, I64, P, I64, I, I, I, I, P, I64, I, I, ctypes.c_float,
                                   P, I64, P, P, P, P, SZ, P]),
+        "rnn_c2f_num_crops": (I, [I, I, I, I, I, I]),
+        "rnn_c2f_max_pairs": (I64, [I, I, I, I, I, I, I]),
+        "rnn_c2f_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I, I, I, I, I, I]),
+        "rnn_c2f_match": (I, [P, I, I, P, I, I, I, P, I, I, P, I, I, I, I, I, I, I, I, I, I,
+                              P, I64, P, P, P, SZ, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -597,6 +598,7 @@ struct FrmState {
   int ld;
   float pixel_tol;  // > 0: converged when the move from U_old is below it
   int starts;       // 1: the seeds were given (output U_old with pixel_tol)
+  const int32_t* pair_on;  // [B] or null: grid seeds only for the pairs marked 1
   int B, k, N1, N2, nwords;
 };
 
@@ -657,6 +659,7 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int
   st->N2 = static_cast<int>(N2);
   st->nwords = static_cast<int>(nwords);
   st->basin = nullptr;
+  st->pair_on = nullptr;
   return c.off;
 }
 
@@ -700,9 +703,10 @@ __global__ void frm_init_kernel(FrmState st, int W1, int S) {
   }
   if (blockIdx.x == 0) {
     for (int b = threadIdx.x; b < st.B; b += blockDim.x) {
-      st.cnt[0][b] = st.k;
+      const int k = st.pair_on && !st.pair_on[b] ? 0 : st.k;
+      st.cnt[0][b] = k;
       st.cnt[1][b] = 0;
-      st.nseeds[b] = st.k;
+      st.nseeds[b] = k;
     }
     if (threadIdx.x == 0) *st.err = 0;
   }
@@ -902,6 +906,8 @@ __global__ void frm_merge_kernel(FrmState st, int W1, int32_t* pairs, int64_t ca
 
 // 3-D point kernels (they use FrmState, frm_apply and block_exclusive_scan)
 #include "points.cuh"
+// coarse-to-fine kernels (they use block_exclusive_scan)
+#include "c2f.cuh"
 
 namespace rnn {
 
@@ -973,11 +979,12 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
                           const int32_t* init, int64_t n_init, int S, int max_iter,
                           float pixel_tol, int32_t* pairs, int64_t cap, int32_t* count_out,
                           int32_t* seed_state, int32_t* basin, void* ws, size_t ws_bytes,
-                          cudaStream_t s) {
+                          cudaStream_t s, const int32_t* pair_on = nullptr) {
   if (B < 1) return RNN_EINVAL;
   if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
   if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || max_iter < 1) return RNN_EINVAL;
   if (!valid_dtype(dt) || !valid_metric(metric)) return RNN_EINVAL;
+  if (pair_on && init) return RNN_EINVAL;  // per-pair enable is for grid seeds
   if (init ? n_init < 0 : S < 1) return RNN_EINVAL;
   if (!(pixel_tol >= 0.f) || (pixel_tol > 0.f && !init)) return RNN_EINVAL;
   rnn_status st0 = check_desc(D1, d);
@@ -1006,6 +1013,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   st.basin = basin;
   st.pixel_tol = pixel_tol;
   st.starts = init ? 1 : 0;
+  st.pair_on = pair_on;
   const Geometry g = geometry(d + (metric == RNN_L2 ? kAugCols : 0));
   const int mode = copies_for(d, metric);
   if (k == 0) {
@@ -1603,6 +1611,173 @@ rnn_status rnn_frm_match_ex(int B, const void* D1, int64_t d1_batch_stride, cons
                  init_xy1, n_init, seed_stride, max_iter, pixel_tol, pairs_out, cap, count_out,
                  seed_state_out, basin_out, workspace, ws_bytes,
                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+// --------------------------------------------------------- coarse-to-fine
+// Crop geometry of a call; false when a size is not positive.
+static bool c2f_geom(int Hc1, int Wc1, int Hc2, int Wc2, int H1, int W1, int H2, int W2,
+                     int crop_h, int crop_w, int min_coarse, C2FGeom* g) {
+  if (Hc1 <= 0 || Wc1 <= 0 || Hc2 <= 0 || Wc2 <= 0 || H1 <= 0 || W1 <= 0 || H2 <= 0 ||
+      W2 <= 0 || crop_h <= 0 || crop_w <= 0)
+    return false;
+  g->Hc1 = Hc1;
+  g->Wc1 = Wc1;
+  g->Hc2 = Hc2;
+  g->Wc2 = Wc2;
+  g->H1 = H1;
+  g->W1 = W1;
+  g->H2 = H2;
+  g->W2 = W2;
+  g->ch = std::min(crop_h, std::min(H1, H2));
+  g->cw = std::min(crop_w, std::min(W1, W2));
+  g->ny = (H1 + g->ch - 1) / g->ch;
+  g->nx = (W1 + g->cw - 1) / g->cw;
+  g->min_coarse = min_coarse;
+  return true;
+}
+
+struct C2FWs {
+  int* status;              // header: OR of the parts' status words
+  int32_t* coarse;          // [mc][2] reciprocal pairs of the coarse maps
+  int32_t* coarse_count;
+  int32_t* crops;           // [B][6] crop table (the caller's, when given)
+  int32_t* pair_on;         // [B]
+  uint16_t *crop1, *crop2;  // [B][ch*cw][dp] windows
+  int32_t* lpairs;          // [B][capc][2] FRM pairs of each crop pair
+  int32_t* lcount;          // [B]
+  int32_t* tag;             // [N1] lowest crop index outputting each pixel
+  int32_t* partner;         // [N1]
+  uint32_t* bm;             // [nwords]
+  int* bcounts;             // [nblk]
+  void* mnn_ws;
+  size_t mnn_bytes;
+  void* frm_ws;
+  size_t frm_bytes;
+  int64_t mc, k, capc, rows, n1, nwords;
+  int B, dp, nblk;
+};
+
+static size_t c2f_layout(void* ws, const C2FGeom& g, int dc, int d, rnn_metric metric, int S,
+                         C2FWs* w) {
+  Carve c(ws);
+  w->B = g.ny * g.nx;
+  w->rows = static_cast<int64_t>(g.ch) * g.cw;
+  w->k = num_seeds(g.ch, g.cw, S);
+  w->capc = std::max<int64_t>(1, std::min(w->k, w->rows));
+  w->mc = std::min(static_cast<int64_t>(g.Hc1) * g.Wc1, static_cast<int64_t>(g.Hc2) * g.Wc2);
+  w->n1 = static_cast<int64_t>(g.H1) * g.W1;
+  w->nwords = (w->n1 + 31) / 32;
+  w->nblk = static_cast<int>((w->nwords + kEmitWords - 1) / kEmitWords);
+  w->dp = metric == RNN_DOT ? padded_depth(d) : d;
+  w->status = c.take<int>(64);
+  w->coarse = c.take<int32_t>(2 * w->mc);
+  w->coarse_count = c.take<int32_t>(1);
+  w->crops = c.take<int32_t>(static_cast<int64_t>(w->B) * kC2FCropCols);
+  w->pair_on = c.take<int32_t>(w->B);
+  w->crop1 = c.take<uint16_t>(w->B * w->rows * w->dp);
+  w->crop2 = c.take<uint16_t>(w->B * w->rows * w->dp);
+  w->lpairs = c.take<int32_t>(2 * w->B * w->capc);
+  w->lcount = c.take<int32_t>(w->B);
+  w->tag = c.take<int32_t>(w->n1);
+  w->partner = c.take<int32_t>(w->n1);
+  w->bm = c.take<uint32_t>(w->nwords);
+  w->bcounts = c.take<int>(w->nblk);
+  w->mnn_bytes = rnn_mnn_workspace_size_ex(g.Hc1, g.Wc1, g.Hc2, g.Wc2, dc, metric);
+  w->mnn_ws = c.take<uint8_t>(w->mnn_bytes);
+  w->frm_bytes = frm_bytes(w->B, w->k, w->rows, w->rows, w->dp, metric);
+  w->frm_ws = c.take<uint8_t>(w->frm_bytes);
+  return c.off;
+}
+
+int rnn_c2f_num_crops(int H1, int W1, int H2, int W2, int crop_h, int crop_w) {
+  C2FGeom g;
+  if (!c2f_geom(1, 1, 1, 1, H1, W1, H2, W2, crop_h, crop_w, 1, &g)) return 0;
+  return g.ny * g.nx;
+}
+
+int64_t rnn_c2f_max_pairs(int H1, int W1, int H2, int W2, int crop_h, int crop_w,
+                          int seed_stride) {
+  C2FGeom g;
+  if (seed_stride < 1 || !c2f_geom(1, 1, 1, 1, H1, W1, H2, W2, crop_h, crop_w, 1, &g)) return 0;
+  const int64_t rows = static_cast<int64_t>(g.ch) * g.cw;
+  const int64_t per = std::min(num_seeds(g.ch, g.cw, seed_stride), rows);
+  return std::min(static_cast<int64_t>(H1) * W1, per * g.ny * g.nx);
+}
+
+size_t rnn_c2f_workspace_size(int Hc1, int Wc1, int Hc2, int Wc2, int dc, int H1, int W1,
+                              int H2, int W2, int d, rnn_metric metric, int crop_h, int crop_w,
+                              int seed_stride) {
+  C2FGeom g;
+  if (!valid_metric(metric) || dc <= 0 || d <= 0 || seed_stride < 1 ||
+      !c2f_geom(Hc1, Wc1, Hc2, Wc2, H1, W1, H2, W2, crop_h, crop_w, 1, &g))
+    return 0;
+  C2FWs w;
+  return c2f_layout(nullptr, g, dc, d, metric, seed_stride, &w);
+}
+
+rnn_status rnn_c2f_match(const void* C1, int Hc1, int Wc1, const void* C2, int Hc2, int Wc2,
+                         int dc, const void* F1, int H1, int W1, const void* F2, int H2, int W2,
+                         int d, rnn_dtype dtype, rnn_metric metric, int crop_h, int crop_w,
+                         int seed_stride, int max_iter, int min_coarse, int32_t* pairs_out,
+                         int64_t cap, int32_t* count_out, int32_t* crops_out, void* workspace,
+                         size_t ws_bytes, rnn_stream_t stream) {
+  C2FGeom g;
+  if (!c2f_geom(Hc1, Wc1, Hc2, Wc2, H1, W1, H2, W2, crop_h, crop_w, min_coarse, &g))
+    return RNN_EINVAL;
+  if (!valid_dtype(dtype) || !valid_metric(metric)) return RNN_EINVAL;
+  if (seed_stride < 1 || max_iter < 1 || !pairs_out || !count_out) return RNN_EINVAL;
+  rnn_status r;
+  if ((r = check_desc(C1, dc)) != RNN_OK || (r = check_desc(C2, dc)) != RNN_OK ||
+      (r = check_desc(F1, d)) != RNN_OK || (r = check_desc(F2, d)) != RNN_OK)
+    return r;
+  const int64_t n1 = static_cast<int64_t>(H1) * W1, n2 = static_cast<int64_t>(H2) * W2;
+  if (n1 >= INT32_MAX || n2 >= INT32_MAX) return RNN_EINVAL;
+  if (g.ny * static_cast<int64_t>(g.nx) > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
+  if (cap < rnn_c2f_max_pairs(H1, W1, H2, W2, crop_h, crop_w, seed_stride))
+    return RNN_ECAPACITY;
+  if (!workspace || !aligned256(workspace) ||
+      ws_bytes < rnn_c2f_workspace_size(Hc1, Wc1, Hc2, Wc2, dc, H1, W1, H2, W2, d, metric,
+                                        crop_h, crop_w, seed_stride))
+    return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  if ((r = device_info(&di)) != RNN_OK) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  C2FWs w;
+  c2f_layout(workspace, g, dc, d, metric, seed_stride, &w);
+  if (crops_out) w.crops = crops_out;
+  // 1. the reciprocal set of the coarse maps
+  if ((r = rnn_mnn_exhaustive_ex(C1, Hc1, Wc1, C2, Hc2, Wc2, dc, dtype, metric, w.coarse, w.mc,
+                                 w.coarse_count, nullptr, nullptr, nullptr, nullptr, w.mnn_ws,
+                                 w.mnn_bytes, stream)) != RNN_OK)
+    return r;
+  // 2. crop table; 3. windows of the crop pairs that are on
+  c2f_place_kernel<<<w.B, 256, 0, s>>>(g, w.coarse, w.coarse_count, w.crops, w.pair_on);
+  if ((r = launched()) != RNN_OK) return r;
+  const int64_t items = 2 * static_cast<int64_t>(w.B) * w.rows * (w.dp / 8) + w.n1 + w.nwords;
+  c2f_gather_kernel<<<grid_for(items, di->sms), kSmallThreads, 0, s>>>(
+      g, static_cast<const uint16_t*>(F1), static_cast<const uint16_t*>(F2), d, w.dp, w.crops,
+      w.B, w.crop1, w.crop2, w.tag, w.n1, w.bm, w.nwords);
+  if ((r = launched()) != RNN_OK) return r;
+  // 4. FRM on every crop pair that is on (grid seeds), in one batched loop
+  const int64_t bs = w.rows * w.dp;
+  if ((r = frm_run(w.B, w.crop1, bs, w.crop2, bs, g.ch, g.cw, g.ch, g.cw, w.dp, dtype, metric,
+                   nullptr, 0, seed_stride, max_iter, 0.f, w.lpairs, w.capc, w.lcount, nullptr,
+                   nullptr, w.frm_ws, w.frm_bytes, s, w.pair_on)) != RNN_OK)
+    return r;
+  // 5. map back, first crop per image-1 pixel, pixel order
+  const int mg = grid_for(static_cast<int64_t>(w.B) * w.capc, di->sms);
+  c2f_mapback_kernel<<<mg, kSmallThreads, 0, s>>>(g, w.B, w.crops, w.lpairs, w.capc, w.lcount,
+                                                  w.tag, w.partner, w.bm, 1);
+  if ((r = launched()) != RNN_OK) return r;
+  c2f_mapback_kernel<<<mg, kSmallThreads, 0, s>>>(g, w.B, w.crops, w.lpairs, w.capc, w.lcount,
+                                                  w.tag, w.partner, w.bm, 0);
+  if ((r = launched()) != RNN_OK) return r;
+  c2f_count_kernel<<<w.nblk, kSmallThreads, 0, s>>>(w.bm, w.nwords, w.bcounts);
+  if ((r = launched()) != RNN_OK) return r;
+  c2f_emit_kernel<<<w.nblk, kSmallThreads, 0, s>>>(
+      w.bm, w.nwords, w.bcounts, w.partner, pairs_out, count_out, w.status,
+      static_cast<const int*>(w.mnn_ws), static_cast<const int*>(w.frm_ws));
+  return launched();
 }
 
 // ------------------------------------------------------------- 3-D points

@@ -25,6 +25,10 @@ weights here, so these maps stand in for them:
   random similarity, plus noise; optionally rounded to multiples of 1/64.
 * ``quantised_points``: ``n`` points with coordinates ``k/64`` in [-16, 16]
   drawn in clusters, with repeated points (ties).
+* ``coarse_map``: the coarse maps of coarse-to-fine matching, standing in for
+  the network's output on a downscaled image: the full-resolution map read at
+  the centre pixel of each coarse cell, optionally through a fixed random
+  projection to another depth and renormalised.
 
 Arrays are float64 ``[H][W][d]`` (channel-last, row-major, pixel index
 ``y*W + x``) holding values that are exactly representable in the requested
@@ -46,6 +50,7 @@ __all__ = [
     "smooth_pair",
     "pointmap_pair",
     "quantised_points",
+    "coarse_map",
     "to_storage",
     "Workload",
     "WORKLOADS",
@@ -207,6 +212,22 @@ def quantised_points(rng: np.random.Generator, n: int, clusters: int = 8,
         src = (rng.random(nrep) * dst).astype(np.int64)
         p[dst] = p[src]
     return p
+
+
+def coarse_map(F: np.ndarray, Hc: int, Wc: int, dc: int = 0, seed: int = 0) -> np.ndarray:
+    """``[Hc][Wc][dc]`` map read from ``F [H][W][d]`` at row
+    ``int((yc + 0.5) * H / Hc)`` and column ``int((xc + 0.5) * W / Wc)``.
+    With ``dc`` > 0 the samples go through a fixed ``dc x d`` Gaussian matrix
+    drawn from ``default_rng(seed)`` and are renormalised; otherwise they are
+    the samples themselves (quantised inputs stay exact)."""
+    H, W, d = F.shape
+    ys = ((np.arange(Hc) + 0.5) * H / Hc).astype(np.int64)
+    xs = ((np.arange(Wc) + 0.5) * W / Wc).astype(np.int64)
+    S = F[ys][:, xs]
+    if dc:
+        R = np.random.default_rng(seed).standard_normal((dc, d))
+        S = _unit(S @ R.T)
+    return S
 
 
 def to_storage(a: np.ndarray, dtype: str):

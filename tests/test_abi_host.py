@@ -247,3 +247,46 @@ def test_pts_argument_errors(lib):
     assert call(P2=FAKE + 2) == EALIGN
     assert call(cap=15) == ECAP
     assert call(wsb=wf - 1) == EWS
+
+
+def test_c2f_host_functions(lib):
+    assert lib.rnn_c2f_num_crops(768, 1024, 768, 1024, 384, 512) == 4
+    assert lib.rnn_c2f_num_crops(1000, 1000, 1000, 1000, 384, 384) == 9
+    assert lib.rnn_c2f_num_crops(100, 100, 50, 60, 384, 512) == 4      # crop cut to 50x60
+    assert lib.rnn_c2f_num_crops(0, 10, 10, 10, 4, 4) == 0
+    k = len(oracle.frm_seeds(384, 512, 8))
+    assert lib.rnn_c2f_max_pairs(768, 1024, 768, 1024, 384, 512, 8) == 4 * k
+    assert lib.rnn_c2f_max_pairs(16, 16, 16, 16, 8, 8, 1) == 256      # one pair per pixel
+    ws = lib.rnn_c2f_workspace_size(64, 80, 64, 80, 256, 768, 1024, 768, 1024, 32, 0, 384,
+                                    512, 8)
+    assert ws >= 2 * 4 * 384 * 512 * 32 * 2 and ws % 256 == 0
+    assert lib.rnn_c2f_workspace_size(64, 80, 64, 80, 256, 768, 1024, 768, 1024, 32, 5, 384,
+                                      512, 8) == 0
+
+
+def test_c2f_argument_errors(lib):
+    ws = lib.rnn_c2f_workspace_size(4, 4, 4, 4, 16, 16, 16, 16, 16, 16, 0, 8, 8, 2)
+    cap = lib.rnn_c2f_max_pairs(16, 16, 16, 16, 8, 8, 2)
+    f = lib.rnn_c2f_match
+
+    def call(**kw):
+        a = dict(C1=FAKE, Hc1=4, Wc1=4, C2=FAKE, Hc2=4, Wc2=4, dc=16, F1=FAKE, H1=16, W1=16,
+                 F2=FAKE, H2=16, W2=16, d=16, dt=0, metric=0, ch=8, cw=8, S=2, it=10, mc=1,
+                 pairs=FAKE, cap=cap, count=FAKE, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return f(a["C1"], a["Hc1"], a["Wc1"], a["C2"], a["Hc2"], a["Wc2"], a["dc"], a["F1"],
+                 a["H1"], a["W1"], a["F2"], a["H2"], a["W2"], a["d"], a["dt"], a["metric"],
+                 a["ch"], a["cw"], a["S"], a["it"], a["mc"], a["pairs"], a["cap"], a["count"],
+                 None, a["ws"], a["wsb"], None)
+
+    assert call(Hc1=0) == EINVAL
+    assert call(ch=0) == EINVAL
+    assert call(S=0) == EINVAL
+    assert call(it=0) == EINVAL
+    assert call(metric=3) == EINVAL
+    assert call(pairs=None) == EINVAL
+    assert call(dc=12) == EALIGN
+    assert call(F2=FAKE + 8) == EALIGN
+    assert call(cap=cap - 1) == ECAP
+    # 40 x 40 crops of 1 x 1 pixel: more crops than RNN_MAX_BATCH
+    assert call(H1=40, W1=40, H2=40, W2=40, ch=1, cw=1) == EUNSUP
