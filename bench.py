@@ -478,6 +478,41 @@ def run_native(args):
                                  "before every call"}
         del flush
 
+    # ------------- coarse-to-fine: 1024x768, d = 32, coarse 80x64 cells, d = 256
+    c2f = None
+    if not args.skip_mnn:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        big = synth.WORKLOADS["frm_1024x768"]
+        F1, F2 = synth.make_workload(big)
+        C1 = synth.coarse_map(F1, 64, 80, dc=256, seed=11)
+        C2 = synth.coarse_map(F2, 64, 80, dc=256, seed=11)
+        c1, c2, f1, f2 = (synth.to_storage(x, "f16").to(dev) for x in (C1, C2, F1, F2))
+        kw = dict(crop=(384, 512), seed_stride=big.seed_stride, max_iter=big.max_iter)
+        ws_c = torch.empty(lib.rnn_c2f_workspace_size(64, 80, 64, 80, 256, big.H, big.W, big.H,
+                                                      big.W, big.d, 0, 384, 512,
+                                                      big.seed_stride),
+                           dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            r = rnn.c2f_match(c1, c2, f1, f2, workspace=ws_c, **kw)
+        reps = 10
+        oa = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        ob = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            oa[i].record()
+            r = rnn.c2f_match(c1, c2, f1, f2, workspace=ws_c, **kw)
+            ob[i].record()
+        torch.cuda.synchronize()
+        ms = statistics.median(_event_ms(oa, ob, reps))
+        c2f = {"metric": "coarse-to-fine image pairs/s: 1024x768 maps, d=32, coarse M on 80x64 "
+                         "cells (d=256), 2x2 crops of 512x384, FRM stride 8, max_iter 15",
+               "value": 1e3 / ms, "unit": "pairs/s", "ms_per_call": ms,
+               "outputs": int(r.count.item()), "crops_on": int(r.crops[:, 5].sum().item()),
+               "dtype": "f16",
+               "note": "includes the binding's output allocation; 256 MB L2 flush before "
+                       "every call"}
+        del flush
+
     # ----------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
@@ -497,7 +532,7 @@ def run_native(args):
                        "global_batch": world * P, "parallelism": f"replicas x{world}",
                        "l2": f"step inputs {2 * A_h.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
             "e2e": e2e, "roofline": roofline, "mnn": mnn, "frm_options": options,
-            "points": pts, "cpu_baseline": cpu,
+            "points": pts, "coarse_to_fine": c2f, "cpu_baseline": cpu,
             "clocks": clocks, "gpu_launches": int(launches),
         }
         print(json.dumps(line), flush=True)
