@@ -438,80 +438,9 @@ def run_native(args):
                              "note": "includes the binding's output and workspace allocation"}
 
     # ------------------------- 3-D point maps (the K-d tree workload, exact NN)
-    pts = None
-    if not args.skip_mnn:
-        pts = {}
-        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        pm = [synth.pointmap_pair(700 + i, w.H, w.W) for i in range(P)]
-        p1 = torch.from_numpy(np.stack([m[0] for m in pm]).astype(np.float32)).to(dev)
-        p2 = torch.from_numpy(np.stack([m[1] for m in pm]).astype(np.float32)).to(dev)
-        n1 = w.H * w.W
-        ws_m = torch.empty(lib.rnn_pts_mnn_workspace_size(w.H, w.W, w.H, w.W),
-                           dtype=torch.uint8, device=dev)
-        ws_f = torch.empty(lib.rnn_pts_frm_workspace_size(P, w.H, w.W, w.H, w.W,
-                                                          w.seed_stride, -1),
-                           dtype=torch.uint8, device=dev)
-        cases = (("mnn", lambda: rnn.pts_mnn(p1[0], p2[0], workspace=ws_m), 2 * n1,
-                  "queries/s", "exhaustive reciprocal set of two 512x384 point maps "
-                  "(both directions)"),
-                 ("frm", lambda: rnn.pts_frm_match(p1, p2, seed_stride=w.seed_stride,
-                                                   max_iter=w.max_iter, workspace=ws_f),
-                  P, "pairs/s", f"FRM on {P} pairs of 512x384 point maps, stride "
-                  f"{w.seed_stride}, max_iter {w.max_iter}"))
-        for name, fn, units, unit, what in cases:
-            for _ in range(3):
-                r = fn()
-            reps = 10
-            oa = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
-            ob = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
-            for i in range(reps):
-                flush.fill_(i & 0xFF)
-                oa[i].record()
-                r = fn()
-                ob[i].record()
-            torch.cuda.synchronize()
-            ms = statistics.median(_event_ms(oa, ob, reps))
-            pts[name] = {"metric": what, "value": units / (ms * 1e-3), "unit": unit,
-                         "ms_per_call": ms, "outputs": int(r.count.sum().item()),
-                         "dtype": "f32",
-                         "note": "includes the binding's output allocation; 256 MB L2 flush "
-                                 "before every call"}
-        del flush
-
+    pts = None if args.skip_mnn else _points_leg(dev, lib, w, P, 10)
     # ------------- coarse-to-fine: 1024x768, d = 32, coarse 80x64 cells, d = 256
-    c2f = None
-    if not args.skip_mnn:
-        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        big = synth.WORKLOADS["frm_1024x768"]
-        F1, F2 = synth.make_workload(big)
-        C1 = synth.coarse_map(F1, 64, 80, dc=256, seed=11)
-        C2 = synth.coarse_map(F2, 64, 80, dc=256, seed=11)
-        c1, c2, f1, f2 = (synth.to_storage(x, "f16").to(dev) for x in (C1, C2, F1, F2))
-        kw = dict(crop=(384, 512), seed_stride=big.seed_stride, max_iter=big.max_iter)
-        ws_c = torch.empty(lib.rnn_c2f_workspace_size(64, 80, 64, 80, 256, big.H, big.W, big.H,
-                                                      big.W, big.d, 0, 384, 512,
-                                                      big.seed_stride),
-                           dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            r = rnn.c2f_match(c1, c2, f1, f2, workspace=ws_c, **kw)
-        reps = 10
-        oa = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
-        ob = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
-        for i in range(reps):
-            flush.fill_(i & 0xFF)
-            oa[i].record()
-            r = rnn.c2f_match(c1, c2, f1, f2, workspace=ws_c, **kw)
-            ob[i].record()
-        torch.cuda.synchronize()
-        ms = statistics.median(_event_ms(oa, ob, reps))
-        c2f = {"metric": "coarse-to-fine image pairs/s: 1024x768 maps, d=32, coarse M on 80x64 "
-                         "cells (d=256), 2x2 crops of 512x384, FRM stride 8, max_iter 15",
-               "value": 1e3 / ms, "unit": "pairs/s", "ms_per_call": ms,
-               "outputs": int(r.count.item()), "crops_on": int(r.crops[:, 5].sum().item()),
-               "dtype": "f16",
-               "note": "includes the binding's output allocation; 256 MB L2 flush before "
-                       "every call"}
-        del flush
+    c2f = None if args.skip_mnn else _c2f_leg(dev, lib, 10)
 
     # ----------------------------------------------------------- CPU baseline
     cpu = None
@@ -541,6 +470,99 @@ def run_native(args):
     return 0
 
 
+def _timed_calls(fn, reps, flush):
+    """Median CUDA-event time of `reps` calls, each after an L2 flush."""
+    import torch
+    oa = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    ob = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    r = None
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        oa[i].record()
+        r = fn()
+        ob[i].record()
+    torch.cuda.synchronize()
+    return statistics.median(_event_ms(oa, ob, reps)), r
+
+
+def _points_leg(dev, lib, w, P, reps, warmup=3):
+    """Reciprocal set and FRM on 512x384 point maps (fp32, exact Euclidean NN)."""
+    import numpy as np
+    import torch
+    import reciprocal_nearest_neighbour_b200 as rnn
+    from reciprocal_nearest_neighbour_b200 import synth
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    pm = [synth.pointmap_pair(700 + i, w.H, w.W) for i in range(P)]
+    p1 = torch.from_numpy(np.stack([m[0] for m in pm]).astype(np.float32)).to(dev)
+    p2 = torch.from_numpy(np.stack([m[1] for m in pm]).astype(np.float32)).to(dev)
+    n1 = w.H * w.W
+    ws_m = torch.empty(lib.rnn_pts_mnn_workspace_size(w.H, w.W, w.H, w.W),
+                       dtype=torch.uint8, device=dev)
+    ws_f = torch.empty(lib.rnn_pts_frm_workspace_size(P, w.H, w.W, w.H, w.W, w.seed_stride, -1),
+                       dtype=torch.uint8, device=dev)
+    cases = (("mnn", lambda: rnn.pts_mnn(p1[0], p2[0], workspace=ws_m), 2 * n1, "queries/s",
+              "exhaustive reciprocal set of two 512x384 point maps (both directions)"),
+             ("frm", lambda: rnn.pts_frm_match(p1, p2, seed_stride=w.seed_stride,
+                                               max_iter=w.max_iter, workspace=ws_f),
+              P, "pairs/s", f"FRM on {P} pairs of 512x384 point maps, stride "
+              f"{w.seed_stride}, max_iter {w.max_iter}"))
+    out = {}
+    for name, fn, units, unit, what in cases:
+        for _ in range(warmup):
+            fn()
+        ms, r = _timed_calls(fn, reps, flush)
+        out[name] = {"metric": what, "value": units / (ms * 1e-3), "unit": unit,
+                     "ms_per_call": ms, "outputs": int(r.count.sum().item()), "dtype": "f32",
+                     "note": "includes the binding's output allocation; 256 MB L2 flush "
+                             "before every call"}
+    return out
+
+
+def _c2f_leg(dev, lib, reps, warmup=3):
+    """Coarse-to-fine: 1024x768 maps (d = 32), coarse M on 80x64 cells (d = 256)."""
+    import torch
+    import reciprocal_nearest_neighbour_b200 as rnn
+    from reciprocal_nearest_neighbour_b200 import synth
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    big = synth.WORKLOADS["frm_1024x768"]
+    F1, F2 = synth.make_workload(big)
+    C1 = synth.coarse_map(F1, 64, 80, dc=256, seed=11)
+    C2 = synth.coarse_map(F2, 64, 80, dc=256, seed=11)
+    c1, c2, f1, f2 = (synth.to_storage(x, "f16").to(dev) for x in (C1, C2, F1, F2))
+    kw = dict(crop=(384, 512), seed_stride=big.seed_stride, max_iter=big.max_iter)
+    ws_c = torch.empty(lib.rnn_c2f_workspace_size(64, 80, 64, 80, 256, big.H, big.W, big.H,
+                                                  big.W, big.d, 0, 384, 512, big.seed_stride),
+                       dtype=torch.uint8, device=dev)
+
+    def fn():
+        return rnn.c2f_match(c1, c2, f1, f2, workspace=ws_c, **kw)
+
+    for _ in range(warmup):
+        fn()
+    ms, r = _timed_calls(fn, reps, flush)
+    return {"metric": "coarse-to-fine image pairs/s: 1024x768 maps, d=32, coarse M on 80x64 "
+                      "cells (d=256), 2x2 crops of 512x384, FRM stride 8, max_iter 15",
+            "value": 1e3 / ms, "unit": "pairs/s", "ms_per_call": ms,
+            "outputs": int(r.count.item()), "crops_on": int(r.crops[:, 5].sum().item()),
+            "dtype": "f16",
+            "note": "includes the binding's output allocation; 256 MB L2 flush before every call"}
+
+
+def run_leg(name, steps, warmup):
+    """One leg alone (for profiling): its calls, then one JSON line."""
+    import torch
+    from reciprocal_nearest_neighbour_b200 import _lib, synth
+    lib = _lib.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if name == "points":
+        res = _points_leg(dev, lib, synth.WORKLOADS[WORKLOAD], 8, steps, warmup)
+    else:
+        res = _c2f_leg(dev, lib, steps, warmup)
+    print(json.dumps({"leg": name, "result": res}), flush=True)
+    return 0
+
+
 def run_nn_case(nq, d, nx):
     """One small nearest-neighbour case for an ncu capture of the fused kernel."""
     import torch
@@ -566,10 +588,14 @@ def main(argv=None):
     ap.add_argument("--skip-mnn", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--leg", choices=["points", "c2f"],
+                    help="run one secondary leg alone (for profiling) and exit")
     ap.add_argument("--nn-case", type=int, nargs=3, metavar=("NQ", "D", "NX"),
                     help="profiling aid: run nn_argmax three times on seeded fp16 "
                          "queries/candidates of these sizes and exit (no timing)")
     args = ap.parse_args(argv)
+    if args.leg:
+        return run_leg(args.leg, args.steps, args.warmup)
     if args.nn_case:
         return run_nn_case(*args.nn_case)
     if args.warmup < 3:

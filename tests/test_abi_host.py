@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rnn_abi_version() == 3
+    assert lib.rnn_abi_version() == 4
     for code, name in _lib.STATUS.items():
         assert lib.rnn_status_string(code).decode().startswith(name)
 
