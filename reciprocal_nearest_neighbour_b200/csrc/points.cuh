@@ -330,7 +330,8 @@ __global__ void pts_scatter_kernel(PtsSets ps, const int32_t* start, const int32
   }
 }
 
-// Points of cells [c0, c1] of one grid row, against the best so far.
+// Points of cells [c0, c1] of one grid row (a contiguous run of sorted
+// points) against the best so far.
 __device__ __forceinline__ void pts_scan_cells(const float4* __restrict__ sorted,
                                                const int32_t* __restrict__ start, int64_t c0,
                                                int64_t c1, float qx, float qy, float qz,
@@ -348,16 +349,26 @@ __device__ __forceinline__ void pts_scan_cells(const float4* __restrict__ sorted
   }
 }
 
-// Nearest point of a set to q: Chebyshev shells k = 0, 1, ... of cells
-// around q's (clamped) cell.  After shell k, every unsearched cell lies
-// beyond one of the cube's open faces; a point there is at least the face
-// distance away along that axis and at least q's distance to the box along
-// the others.  The search stops when the best squared distance is below
-// that bound (less a rounding allowance), or when no face is open.  Returns
-// the squared distance; *idx is the point's index in its set.
+// Nearest point of a set to q, searched by G lanes together (G a power of
+// two; the G lanes of an aligned group pass the same q): Chebyshev shells
+// k = 0, 1, ... of cells around q's (clamped) cell.  A shell is (2k+1)^2
+// grid rows (dz, dy); rows on a z or y face of the cube are scanned whole
+// (one contiguous run of sorted points), the others at their two end cells.
+// Rows are dealt round-robin to the lanes, and the group's best is merged
+// after each shell.  After shell k every unsearched cell lies beyond one of
+// the cube's open faces; a point there is at least the face distance away
+// along that axis and at least q's distance to the box along the others.
+// The search stops when the best squared distance is below that bound (less
+// a rounding allowance), or when no face is open.  Returns the squared
+// distance; *idx is the point's index in its set (the same in every lane of
+// the group).
+template <int G>
 __device__ float pts_nearest(const PtsGrid g, const float4* __restrict__ sorted,
                              const int32_t* __restrict__ start, float qx, float qy, float qz,
                              int* idx) {
+  const int lane = threadIdx.x & 31;
+  const int r = lane & (G - 1);
+  const unsigned gmask = G == 32 ? 0xffffffffu : (((1u << G) - 1u) << (lane & ~(G - 1)));
   const float q[3] = {qx, qy, qz};
   int c[3];
   float out2[3];  // squared distance from q to the box along each axis
@@ -371,20 +382,31 @@ __device__ float pts_nearest(const PtsGrid g, const float4* __restrict__ sorted,
   int bi = 0x7fffffff;
   const int64_t plane = static_cast<int64_t>(g.dim[0]) * g.dim[1];
   for (int k = 0;; ++k) {
+    // the cube's rows clipped to the grid, numbered row-major over (z, y)
     const int z0 = max(c[2] - k, 0), z1 = min(c[2] + k, g.dim[2] - 1);
     const int y0 = max(c[1] - k, 0), y1 = min(c[1] + k, g.dim[1] - 1);
     const int x0 = max(c[0] - k, 0), x1 = min(c[0] + k, g.dim[0] - 1);
-    for (int z = z0; z <= z1; ++z) {
-      const bool zface = z == c[2] - k || z == c[2] + k;
-      for (int y = y0; y <= y1; ++y) {
-        const int64_t row = g.cell0 + z * plane + static_cast<int64_t>(y) * g.dim[0];
-        if (zface || y == c[1] - k || y == c[1] + k) {
-          pts_scan_cells(sorted, start, row + x0, row + x1, qx, qy, qz, best, bi);
-        } else {
-          if (c[0] - k >= 0) pts_scan_cells(sorted, start, row + x0, row + x0, qx, qy, qz, best, bi);
-          if (c[0] + k < g.dim[0] && k > 0)
-            pts_scan_cells(sorted, start, row + x1, row + x1, qx, qy, qz, best, bi);
-        }
+    const int ny = y1 - y0 + 1;
+    const int nrows = (z1 - z0 + 1) * ny;
+    for (int j = r; j < nrows; j += G) {
+      const int zi = j / ny;
+      const int z = z0 + zi, y = y0 + (j - zi * ny);
+      const int64_t row = g.cell0 + z * plane + static_cast<int64_t>(y) * g.dim[0];
+      if (z == c[2] - k || z == c[2] + k || y == c[1] - k || y == c[1] + k) {
+        pts_scan_cells(sorted, start, row + x0, row + x1, qx, qy, qz, best, bi);
+      } else {
+        if (c[0] - k >= 0) pts_scan_cells(sorted, start, row + x0, row + x0, qx, qy, qz, best, bi);
+        if (c[0] + k < g.dim[0])
+          pts_scan_cells(sorted, start, row + x1, row + x1, qx, qy, qz, best, bi);
+      }
+    }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(gmask, best, o);
+      const int oi = __shfl_xor_sync(gmask, bi, o);
+      if (ob < best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
       }
     }
     // lower bound on the squared distance to any unsearched cell
@@ -412,10 +434,16 @@ __device__ float pts_nearest(const PtsGrid g, const float4* __restrict__ sorted,
   return best;
 }
 
+// Lanes per query (measured on 512x384 point maps): four for the
+// reciprocal-set sweeps, sixteen for the FRM half-steps, which have a query
+// per active seed only and need the extra parallelism to hide latency.
+constexpr int kPtsGroupQuery = 4;
+constexpr int kPtsGroup = 16;
+
 // Nearest neighbours of nq query points (Q, [nq][3]) in set `set`: index
 // and squared distance, or packed keys (score = the squared distance) for
 // the mutual test.  Two query families share one launch (the two sweeps of
-// the reciprocal set).
+// the reciprocal set).  kPtsGroupQuery lanes per query.
 struct PtsQuery {
   const float* Q;
   int64_t nq;
@@ -428,27 +456,31 @@ struct PtsQuery {
 __global__ void pts_query_kernel(PtsQuery q0, PtsQuery q1, int nfam, const PtsGrid* grids,
                                  const float4* sorted, const int32_t* start) {
   const int64_t n = q0.nq + (nfam > 1 ? q1.nq : 0);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < n;
+  constexpr int G = kPtsGroupQuery;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x / G;
+  const bool lead = (threadIdx.x & (G - 1)) == 0;
+  for (int64_t t = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) / G; t < n;
        t += stride) {
     const bool first = t < q0.nq;
     const PtsQuery& Qf = first ? q0 : q1;
     const int64_t i = first ? t : t - q0.nq;
     const float* p = Qf.Q + 3 * i;
     int j;
-    const float d2 = pts_nearest(grids[Qf.set], sorted, start, __ldg(p), __ldg(p + 1),
-                                 __ldg(p + 2), &j);
-    if (Qf.idx) Qf.idx[i] = j;
-    if (Qf.dist2) Qf.dist2[i] = d2;
-    if (Qf.keys) Qf.keys[i] = pack_key(d2, j);
+    const float d2 =
+        pts_nearest<G>(grids[Qf.set], sorted, start, __ldg(p), __ldg(p + 1), __ldg(p + 2), &j);
+    if (lead) {
+      if (Qf.idx) Qf.idx[i] = j;
+      if (Qf.dist2) Qf.dist2[i] = d2;
+      if (Qf.keys) Qf.keys[i] = pack_key(d2, j);
+    }
   }
 }
 
-// Half-step h of FRM on point maps, one thread per active seed of every
-// pair: the NN of the seed's point (NN2: U of image 1 in the image-2 grid of
-// its pair; NN1: V of image 2 in the image-1 grid), then frm_apply.  Sets
-// 0..B-1 are the image-1 maps, B..2B-1 the image-2 maps.  The list and count
-// buffers rotate as in frm_step_kernel.
+// Half-step h of FRM on point maps, kPtsGroup lanes per active seed of
+// every pair: the NN of the seed's point (NN2: U of image 1 in the image-2
+// grid of its pair; NN1: V of image 2 in the image-1 grid), then frm_apply
+// by the group's first lane.  Sets 0..B-1 are the image-1 maps, B..2B-1 the
+// image-2 maps.  The list and count buffers rotate as in frm_step_kernel.
 __global__ void frm_pts_step_kernel(FrmState st, PtsSets ps, const PtsGrid* grids,
                                     const float4* sorted, const int32_t* start, int h,
                                     int nn2_half, int last_iter) {
@@ -461,8 +493,9 @@ __global__ void frm_pts_step_kernel(FrmState st, PtsSets ps, const PtsGrid* grid
     for (int b = threadIdx.x; b < st.B; b += blockDim.x) cnt_next[b] = 0;
   }
   const int32_t* rows = nn2_half ? st.U : st.V;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t x = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const bool lead = (threadIdx.x & (kPtsGroup - 1)) == 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x / kPtsGroup;
+  for (int64_t x = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) / kPtsGroup;
        x < static_cast<int64_t>(st.B) * st.k; x += stride) {
     const int b = static_cast<int>(x / st.k);
     const int i = static_cast<int>(x - static_cast<int64_t>(b) * st.k);
@@ -472,9 +505,9 @@ __global__ void frm_pts_step_kernel(FrmState st, PtsSets ps, const PtsGrid* grid
     const int64_t r = rows[base + s];
     const float* p = nn2_half ? pts_set_base(ps, b) + 3 * r : pts_set_base(ps, ps.nb + b) + 3 * r;
     int j;
-    (void)pts_nearest(grids[nn2_half ? ps.nb + b : b], sorted, start, __ldg(p), __ldg(p + 1),
-                      __ldg(p + 2), &j);
-    frm_apply(st, b, base, s, j, nn2_half, last_iter, list_out, cnt_out);
+    (void)pts_nearest<kPtsGroup>(grids[nn2_half ? ps.nb + b : b], sorted, start, __ldg(p),
+                                 __ldg(p + 1), __ldg(p + 2), &j);
+    if (lead) frm_apply(st, b, base, s, j, nn2_half, last_iter, list_out, cnt_out);
   }
 }
 

@@ -1178,9 +1178,10 @@ static rnn_status pts_build(const PtsSets& ps, const PtsWs& w, int* err, DeviceI
   return launched();
 }
 
-// Blocks of kPtsThreads for one thread per query, grid-stride beyond 8 per SM.
-static int pts_query_grid(int64_t n, int sms) {
-  int64_t g = (n + kPtsThreads - 1) / kPtsThreads;
+// Blocks of kPtsThreads for `lanes` lanes per query, grid-stride beyond 8
+// blocks per SM.
+static int pts_query_grid(int64_t n, int sms, int lanes) {
+  int64_t g = (n * lanes + kPtsThreads - 1) / kPtsThreads;
   if (g > 8LL * sms) g = 8LL * sms;
   return static_cast<int>(g < 1 ? 1 : g);
 }
@@ -1244,7 +1245,7 @@ static rnn_status frm_run_pts(int B, const float* P1, int64_t bs1, const float* 
   }
   if ((r = frm_seed(st, init, n_init, W1, S, di, s)) != RNN_OK) return r;
   if ((r = pts_build(ps, w, nullptr, di, s)) != RNN_OK) return r;
-  const int qg = pts_query_grid(static_cast<int64_t>(B) * k, di->sms);
+  const int qg = pts_query_grid(static_cast<int64_t>(B) * k, di->sms, kPtsGroup);
   for (int it = 1; it <= max_iter; ++it) {
     const int h = 2 * (it - 1);
     frm_pts_step_kernel<<<qg, kPtsThreads, 0, s>>>(st, ps, w.grids, w.sorted, w.start, h, 1, 0);
@@ -1817,8 +1818,8 @@ rnn_status rnn_pts_nn(const float* Q, int64_t nq, const float* X, int64_t nx, in
   if ((r = pts_build(ps, w, err, di, s)) != RNN_OK) return r;
   if (nq == 0) return RNN_OK;
   PtsQuery q{Q, nq, 0, idx_out, dist2_out, nullptr};
-  pts_query_kernel<<<pts_query_grid(nq, di->sms), kPtsThreads, 0, s>>>(q, q, 1, w.grids,
-                                                                        w.sorted, w.start);
+  pts_query_kernel<<<pts_query_grid(nq, di->sms, kPtsGroupQuery), kPtsThreads, 0, s>>>(
+      q, q, 1, w.grids, w.sorted, w.start);
   return launched();
 }
 
@@ -1869,7 +1870,7 @@ rnn_status rnn_pts_mnn(const float* P1, int H1, int W1, const float* P2, int H2,
   // the other way -> NN1
   PtsQuery q1{P1, n1, 1, nullptr, nullptr, m.rowk};
   PtsQuery q2{P2, n2, 0, nullptr, nullptr, m.colk};
-  pts_query_kernel<<<pts_query_grid(n1 + n2, di->sms), kPtsThreads, 0, s>>>(
+  pts_query_kernel<<<pts_query_grid(n1 + n2, di->sms, kPtsGroupQuery), kPtsThreads, 0, s>>>(
       q1, q2, 2, w.grids, w.sorted, w.start);
   if ((r = launched()) != RNN_OK) return r;
   const int nblk1 = static_cast<int>((n1 + kMnnChunk - 1) / kMnnChunk);
