@@ -1279,7 +1279,7 @@ const char* rnn_status_string(rnn_status s) {
   return "unknown rnn_status";
 }
 
-int rnn_abi_version(void) { return 3; }
+int rnn_abi_version(void) { return 4; }
 
 uint64_t rnn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
