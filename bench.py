@@ -152,10 +152,8 @@ class ClockSampler:
 
 
 def _dist():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
+    from reciprocal_nearest_neighbour_b200 import replicas
+    return replicas.env()
 
 
 def _oracle_frm_pairs_per_s(maps, budget_s: float, max_pairs: int):
@@ -220,7 +218,7 @@ def run_native(args):
     import torch.distributed as dist
 
     import reciprocal_nearest_neighbour_b200 as rnn
-    from reciprocal_nearest_neighbour_b200 import _lib, synth
+    from reciprocal_nearest_neighbour_b200 import _lib, replicas, synth
 
     world, rank, local = _dist()
     if world != args.gpus:
@@ -236,21 +234,16 @@ def run_native(args):
                                 device_id=dev)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(world)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, world, dev)
 
     lib = _lib.load()
     peaks = _peaks()
     w = synth.WORKLOADS[WORKLOAD]
     P = args.pairs
-    pair_ids = range(rank * P, rank * P + P)      # each rank matches its own pairs
+    pair_ids = replicas.pair_ids(rank, P)         # each rank matches its own pairs
     A_h, B_h = synth.make_workload_storage(w, "f16", pairs=pair_ids,
                                            workers=min(P, max(1, (os.cpu_count() or 2) // world)))
     A_h, B_h = A_h.pin_memory(), B_h.pin_memory()
@@ -294,7 +287,7 @@ def run_native(args):
     clocks = clk.summary()
     step_ms = t0e.elapsed_time(t1e) / args.steps
     step_ms = max_over_ranks(step_ms)
-    value = world * P / (step_ms * 1e-3)
+    value = replicas.aggregate_rate(P, world, step_ms)
     rnn.workspace_status(plan.workspace)
 
     # roofline of the fused similarity+argmax kernel over the recorded launches
