@@ -243,6 +243,26 @@ rnn_status rnn_frm_match_ex(int B, const void *D1, int64_t d1_batch_stride, cons
                             size_t ws_bytes, rnn_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The reciprocal set from NN arrays computed elsewhere (cv-learn.com "MASt3R"
+ * note, paragraph "Fast reciprocal matching (FRM)": M = {(i, j) | j = NN2(i)
+ * and i = NN1(j)}), e.g. when the rows of both maps are split over several
+ * GPUs, each computes NN2 / NN1 for its rows, and the arrays are gathered.
+ *
+ *   rowarg     device int32 [n1]: NN2 of every image-1 pixel.
+ *   colarg     device int32 [n2]: NN1 of every image-2 pixel.
+ *   pairs_out  [cap][2] int32: (i, rowarg[i]) for every i with
+ *              colarg[rowarg[i]] == i, in increasing i; cap >= min(n1, n2).
+ *              Indices outside [0, n2) in rowarg are never mutual.
+ *   count_out  [1] int32.
+ *   workspace  at least rnn_mnn_mutual_workspace_size(n1) bytes.
+ * 2 kernel launches (and one memset of the workspace header).
+ */
+size_t rnn_mnn_mutual_workspace_size(int64_t n1);
+rnn_status rnn_mnn_mutual(const int32_t *rowarg, int64_t n1, const int32_t *colarg, int64_t n2,
+                          int32_t *pairs_out, int64_t cap, int32_t *count_out, void *workspace,
+                          size_t ws_bytes, rnn_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Coarse-to-fine matching (cv-learn.com "MASt3R" note, paragraph
  * "Coarse-to-fine matching": high-resolution images are matched coarsely
  * first, the coarse matches guide the matching of enumerated local crops,

@@ -46,7 +46,7 @@ __all__ = [
     "nn_argmax", "mnn_exhaustive", "frm_match", "frm_match_batched", "frm_num_seeds",
     "frm_max_pairs", "workspace_status", "trim", "MNNResult", "FRMResult", "RNNError",
     "RNNLibraryError", "FRMPlan", "frm_match_ex", "frm_refine", "pts_nn", "pts_mnn",
-    "pts_frm_match", "c2f_match", "C2FResult",
+    "pts_frm_match", "c2f_match", "C2FResult", "mnn_mutual",
 ]
 
 _DT = {torch.float16: _lib.RNN_F16, torch.bfloat16: _lib.RNN_BF16}
@@ -172,6 +172,29 @@ def mnn_exhaustive(D1: torch.Tensor, D2: torch.Tensor, *, with_nn: bool = False,
         _ptr(out.rowmax), _ptr(out.colarg), _ptr(out.colmax), workspace.data_ptr(),
         workspace.numel(), _stream(D1)), "rnn_mnn_exhaustive_ex")
     return out
+
+
+def mnn_mutual(rowarg: torch.Tensor, colarg: torch.Tensor, *,
+               workspace: Optional[torch.Tensor] = None):
+    """The reciprocal set from NN arrays: ``(i, rowarg[i])`` for every i with
+    ``colarg[rowarg[i]] == i``, in increasing i.  ``rowarg`` (NN2 of every
+    image-1 pixel) and ``colarg`` (NN1 of every image-2 pixel) are int32 CUDA
+    tensors.  Returns ``(pairs [min(n1, n2), 2], count [1])``."""
+    for t, n in ((rowarg, "rowarg"), (colarg, "colarg")):
+        _check_map(t, n, 1)
+        if t.dtype != torch.int32:
+            raise ValueError(f"{n} must be int32")
+    lib = _lib.load()
+    n1, n2 = rowarg.numel(), colarg.numel()
+    dev = rowarg.device
+    pairs = torch.empty((max(1, min(n1, n2)), 2), dtype=torch.int32, device=dev)
+    count = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _workspace(lib.rnn_mnn_mutual_workspace_size(n1), dev)
+    _lib.check(lib.rnn_mnn_mutual(rowarg.data_ptr(), n1, colarg.data_ptr(), n2, pairs.data_ptr(),
+                                  pairs.shape[0], count.data_ptr(), workspace.data_ptr(),
+                                  workspace.numel(), _stream(rowarg)), "rnn_mnn_mutual")
+    return pairs, count
 
 
 def frm_num_seeds(H1: int, W1: int, seed_stride: int) -> int:

@@ -44,6 +44,8 @@ EXPORTS = (
     "rnn_c2f_max_pairs",
     "rnn_c2f_workspace_size",
     "rnn_c2f_match",
+    "rnn_mnn_mutual_workspace_size",
+    "rnn_mnn_mutual",
 )
 
 STATUS = {
@@ -122,6 +124,8 @@ def load():
         "rnn_c2f_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I, I, I, I, I, I]),
         "rnn_c2f_match": (I, [P, I, I, P, I, I, I, P, I, I, P, I, I, I, I, I, I, I, I, I, I,
                               P, I64, P, P, P, SZ, P]),
+        "rnn_mnn_mutual_workspace_size": (SZ, [I64]),
+        "rnn_mnn_mutual": (I, [P, I64, P, I64, P, I64, P, P, SZ, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

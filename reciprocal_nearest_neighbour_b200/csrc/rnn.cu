@@ -563,6 +563,67 @@ __global__ void mnn_write_kernel(const unsigned long long* rowk, int64_t n1,
   if (blockIdx.x == nblocks - 1 && threadIdx.x == 0) *count_out = off + btot;
 }
 
+// Mutual test on plain argmax arrays (the reciprocal set assembled from NN
+// results computed elsewhere, e.g. on several GPUs): pass 1 counts per block
+// of kMnnChunk rows; pass 2 writes the pairs in increasing i.  An index out of
+// range is never mutual.
+__device__ __forceinline__ bool is_mutual_arg(const int32_t* rowarg, const int32_t* colarg,
+                                              int64_t n2, int64_t i, int* j) {
+  *j = rowarg[i];
+  return *j >= 0 && *j < n2 && colarg[*j] == static_cast<int32_t>(i);
+}
+
+__global__ void mutual_count_kernel(const int32_t* rowarg, int64_t n1, const int32_t* colarg,
+                                    int64_t n2, int* block_counts) {
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kMnnChunk;
+  int c = 0;
+  for (int e = 0; e < kMnnChunk / kSmallThreads; ++e) {
+    const int64_t i = base + static_cast<int64_t>(e) * kSmallThreads + threadIdx.x;
+    int j;
+    if (i < n1 && is_mutual_arg(rowarg, colarg, n2, i, &j)) ++c;
+  }
+  int total;
+  (void)block_exclusive_scan(c, &total);
+  if (threadIdx.x == 0) block_counts[blockIdx.x] = total;
+}
+
+__global__ void mutual_write_kernel(const int32_t* rowarg, int64_t n1, const int32_t* colarg,
+                                    int64_t n2, const int* block_counts, int32_t* pairs,
+                                    int32_t* count_out) {
+  __shared__ int s_off;
+  int part = 0;
+  for (int b = threadIdx.x; b < static_cast<int>(blockIdx.x); b += blockDim.x)
+    part += block_counts[b];
+  int tot;
+  (void)block_exclusive_scan(part, &tot);
+  if (threadIdx.x == 0) s_off = tot;
+  __syncthreads();
+  const int off = s_off;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kMnnChunk;
+  constexpr int per = kMnnChunk / kSmallThreads;
+  int js[per];
+  bool ms[per];
+  int c = 0;
+#pragma unroll
+  for (int e = 0; e < per; ++e) {
+    const int64_t i = base + static_cast<int64_t>(threadIdx.x) * per + e;
+    ms[e] = i < n1 && is_mutual_arg(rowarg, colarg, n2, i, &js[e]);
+    c += ms[e] ? 1 : 0;
+  }
+  int btot;
+  int pos = off + block_exclusive_scan(c, &btot);
+#pragma unroll
+  for (int e = 0; e < per; ++e) {
+    if (ms[e]) {
+      const int64_t i = base + static_cast<int64_t>(threadIdx.x) * per + e;
+      pairs[2 * static_cast<int64_t>(pos)] = static_cast<int32_t>(i);
+      pairs[2 * static_cast<int64_t>(pos) + 1] = js[e];
+      ++pos;
+    }
+  }
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) *count_out = off + btot;
+}
+
 // ------------------------------------------------------------------- FRM
 // Options of the quoted fast_reciprocal_NNs (staskaer.github.io DUSt3R/MASt3R
 // blog, MASt3R matching section) besides the grid stride: given start pixels
@@ -1279,7 +1340,7 @@ const char* rnn_status_string(rnn_status s) {
   return "unknown rnn_status";
 }
 
-int rnn_abi_version(void) { return 4; }
+int rnn_abi_version(void) { return 5; }
 
 uint64_t rnn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -1612,6 +1673,38 @@ rnn_status rnn_frm_match_ex(int B, const void* D1, int64_t d1_batch_stride, cons
                  init_xy1, n_init, seed_stride, max_iter, pixel_tol, pairs_out, cap, count_out,
                  seed_state_out, basin_out, workspace, ws_bytes,
                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------ mutual test of NN arrays
+size_t rnn_mnn_mutual_workspace_size(int64_t n1) {
+  Carve c(nullptr);
+  c.take<int>(64);
+  c.take<int>((n1 > 0 ? n1 : 1) / kMnnChunk + 2);
+  return c.off;
+}
+
+rnn_status rnn_mnn_mutual(const int32_t* rowarg, int64_t n1, const int32_t* colarg, int64_t n2,
+                          int32_t* pairs_out, int64_t cap, int32_t* count_out, void* workspace,
+                          size_t ws_bytes, rnn_stream_t stream) {
+  if (n1 < 1 || n2 < 1 || n1 > INT32_MAX || n2 > INT32_MAX) return RNN_EINVAL;
+  if (!rowarg || !colarg || !pairs_out || !count_out) return RNN_EINVAL;
+  if (cap < (n1 < n2 ? n1 : n2)) return RNN_ECAPACITY;
+  if (!workspace || !aligned256(workspace) || ws_bytes < rnn_mnn_mutual_workspace_size(n1))
+    return RNN_EWORKSPACE;
+  DeviceInfo* di = nullptr;
+  rnn_status r = device_info(&di);
+  if (r != RNN_OK) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(workspace);
+  int* err = c.take<int>(64);
+  int* counts = c.take<int>(n1 / kMnnChunk + 2);
+  if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return RNN_ECUDA;
+  const int nblk = static_cast<int>((n1 + kMnnChunk - 1) / kMnnChunk);
+  mutual_count_kernel<<<nblk, kSmallThreads, 0, s>>>(rowarg, n1, colarg, n2, counts);
+  if ((r = launched()) != RNN_OK) return r;
+  mutual_write_kernel<<<nblk, kSmallThreads, 0, s>>>(rowarg, n1, colarg, n2, counts, pairs_out,
+                                                     count_out);
+  return launched();
 }
 
 // --------------------------------------------------------- coarse-to-fine

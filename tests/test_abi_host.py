@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rnn_abi_version() == 4
+    assert lib.rnn_abi_version() == 5
     for code, name in _lib.STATUS.items():
         assert lib.rnn_status_string(code).decode().startswith(name)
 
@@ -290,3 +290,14 @@ def test_c2f_argument_errors(lib):
     assert call(cap=cap - 1) == ECAP
     # 40 x 40 crops of 1 x 1 pixel: more crops than RNN_MAX_BATCH
     assert call(H1=40, W1=40, H2=40, W2=40, ch=1, cw=1) == EUNSUP
+
+
+def test_mnn_mutual_argument_errors(lib):
+    ws = lib.rnn_mnn_mutual_workspace_size(100)
+    assert ws > 0 and ws % 256 == 0
+    f = lib.rnn_mnn_mutual
+    assert f(FAKE, 0, FAKE, 10, FAKE, 10, FAKE, FAKE, ws, None) == EINVAL
+    assert f(None, 100, FAKE, 10, FAKE, 10, FAKE, FAKE, ws, None) == EINVAL
+    assert f(FAKE, 100, FAKE, 10, FAKE, 9, FAKE, FAKE, ws, None) == ECAP
+    assert f(FAKE, 100, FAKE, 10, FAKE, 10, FAKE, FAKE, ws - 1, None) == EWS
+    assert f(FAKE, 100, FAKE, 10, FAKE, 10, FAKE, FAKE + 8, ws, None) == EWS

@@ -206,3 +206,39 @@ def test_golden_basin_on_gpu(golden_dir, case):
     assert r.basin[0].cpu().tolist() == c["basin"]
     if "seed_queries" in c:
         assert seed_state_np(r)[2].tolist() == c["seed_queries"]
+
+
+# ------------------------------------------ reciprocal set from NN arrays
+
+def test_mnn_mutual_matches_numpy():
+    rng = np.random.default_rng(90)
+    n1, n2 = 20000, 13001
+    rowarg = rng.integers(0, n2, n1).astype(np.int32)
+    colarg = rng.integers(0, n1, n2).astype(np.int32)
+    # plant mutual pairs and a few out-of-range indices
+    i = rng.choice(n1, 3000, replace=False)
+    j = rng.choice(n2, 3000, replace=False)
+    rowarg[i] = j
+    colarg[j] = i
+    rowarg[:5] = [-1, n2, n2 + 7, -100, 2 ** 30]
+    pairs, count = rnn.mnn_mutual(torch.from_numpy(rowarg).cuda(), torch.from_numpy(colarg).cuda())
+    ok = np.array([0 <= rowarg[k] < n2 and colarg[rowarg[k]] == k for k in range(n1)])
+    ref = np.stack([np.nonzero(ok)[0], rowarg[ok]], axis=1)
+    assert np.array_equal(pairs[: int(count.item())].cpu().numpy(), ref)
+
+
+def test_sharded_single_rank_equals_exhaustive():
+    from reciprocal_nearest_neighbour_b200 import replicas
+
+    rng = np.random.default_rng(91)
+    D1 = synth.to_storage(synth.quantised_map(rng, 37, 41, 24), "f16")
+    D2 = synth.to_storage(synth.quantised_map(rng, 29, 53, 24), "f16")
+    pairs, count = replicas.mnn_sharded(dev(D1), dev(D2), 1, 0)
+    ref = oracle.mnn(D1, D2).pairs
+    assert np.array_equal(pairs[: int(count.item())].cpu().numpy(), ref)
+    # the rank-0 half of a two-rank split finds the NN of its own rows exactly
+    r1 = replicas.row_slice(37 * 41, 2, 0)
+    idx, _ = rnn.nn_argmax(dev(D1).reshape(-1, 24)[r1.start:r1.stop], dev(D2).reshape(-1, 24))
+    ref_rows = oracle.nn(D1.reshape(-1, 24)[r1.start:r1.stop], D2.reshape(-1, 24)).arg
+    assert len(ref_rows) == len(r1)
+    assert np.array_equal(idx.cpu().numpy(), ref_rows)
