@@ -244,9 +244,10 @@ __device__ __forceinline__ float max32(const float (&v)[32]) {
 }
 
 // kEpiWarps: epilogue warps (8 or 16); kChunks: 32-column chunks of each
-// tile read by one of them (block_n * nacc / (8 * kEpiWarps)); kBatch:
-// chunks per copy from tensor memory to registers.
-template <int kEpiWarps, int kChunks, int kBatch>
+// tile read by one of them; kBatch: chunks per copy from tensor memory to
+// registers; kOneGroup: all epilogue warps take every tile (each a column
+// part of it) instead of one group per accumulator.
+template <int kEpiWarps, int kChunks, int kBatch, bool kOneGroup = false>
 __global__ void __launch_bounds__((kEpiWarp0 + kEpiWarps) * 32, 1)
 nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUtensorMap tmap0,
                  const __grid_constant__ CUtensorMap tmap1,
@@ -282,7 +283,9 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
   SharedTables* T = reinterpret_cast<SharedTables*>(scan_scratch + 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int epi_per_group = kEpiWarps / p.nacc;  // epilogue warps sharing one accumulator
+  // epilogue warps per group: one group per accumulator, or with kOneGroup a
+  // single group taking every tile
+  const int epi_per_group = kOneGroup ? kEpiWarps : kEpiWarps / p.nacc;
   // tensor-memory allocation: a power of two of at least 32 columns
   uint32_t ncols = 32;
   while (ncols < static_cast<uint32_t>(p.nacc * p.block_n)) ncols <<= 1;
@@ -567,19 +570,24 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
     }
   } else {
     // --------------------------------------------------------- epilogue
-    // Group `grp` owns accumulator grp and reduces the tiles g with
-    // g % nacc == grp; within it, warp w covers TMEM lanes 32*(w%4).. and
-    // column part `part` of each tile, kBatch chunks of 32 columns per copy
-    // to registers.  After the last copy of a tile the accumulator goes back
-    // to the MMA warps, before that copy is folded.
+    // Group `grp` reduces the tiles of accumulator grp (one group per
+    // accumulator), or with kOneGroup the one group takes every tile; within
+    // it, warp w covers TMEM lanes
+    // 32*(w%4).. and column part `part` of each tile, kBatch chunks of 32
+    // columns per copy to registers.  After the last copy of a tile the
+    // accumulator goes back to the MMA warps, before that copy is folded: with
+    // one copy per tile (kChunks == kBatch) it is held for one round trip.
     const int ew = warp - kEpiWarp0;
     const int quad = warp & 3;
     const int grp = ew / epi_per_group;
     const int part = (ew - grp * epi_per_group) >> 2;
     const int row = quad * 32 + lane;
     constexpr int cols_part = kChunk * kChunks;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                               static_cast<uint32_t>(grp * p.block_n + part * cols_part);
+    // with one group per accumulator the group's accumulator column is fixed;
+    // with kOneGroup it is added per tile
+    const uint32_t lane_base =
+        tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+        static_cast<uint32_t>((kOneGroup ? 0 : grp * p.block_n) + part * cols_part);
     int acc = 0, stage = 0;  // position of tile t in this CTA's tile sequence
     uint32_t phase = 0;
     bool ok = true;
@@ -589,7 +597,7 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
       float best = -__int_as_float(0x7f800000);
       int bcol = -1;  // first column of the first chunk that reached `best`
       for (int t = ui.t0; t < ui.t1; ++t) {
-        if (acc == grp) {
+        if (kOneGroup || acc == grp) {
           // stages is a multiple of nacc, so done_bar[stage] is only ever
           // used by this group's tiles, and its next phase needs this tile's
           // accumulator back: the parity below cannot be a phase behind
@@ -605,7 +613,10 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
           for (int h = 0; h < kChunks; h += kBatch) {
             float v[kBatch][kChunk];
 #pragma unroll
-            for (int c = 0; c < kBatch; ++c) tmem_ld32(lane_base + kChunk * (h + c), v[c]);
+            for (int c = 0; c < kBatch; ++c)
+              tmem_ld32(lane_base + static_cast<uint32_t>((kOneGroup ? acc * p.block_n : 0) +
+                                                          kChunk * (h + c)),
+                        v[c]);
             tmem_wait_ld_regs(v[0]);
 #pragma unroll
             for (int c = 1; c < kBatch; ++c) reg_fence(v[c]);
