@@ -189,12 +189,9 @@ static rnn_status launched() {
   return RNN_OK;
 }
 
-// one_group: all epilogue warps take every tile (the FRM half-steps: short
-// units over partly live query tiles); otherwise one group per accumulator
-// (long sweeps, where each group has two tiles' time for its fold).
 static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const CUtensorMap& m1,
                             const CUtensorMap& q0, const CUtensorMap& q1, const Geometry& g,
-                            DeviceInfo* di, cudaStream_t s, bool one_group = false) {
+                            DeviceInfo* di, cudaStream_t s) {
   NNParams p = p_in;
   p.kb = g.kb;
   p.nkb = g.nkb;
@@ -217,8 +214,7 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
       if (cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2>, attr, sm) != cudaSuccess ||
           cudaFuncSetAttribute(nn_argmax_kernel<16, 4, 2>, attr, sm) != cudaSuccess ||
           cudaFuncSetAttribute(nn_argmax_kernel<8, 4, 4>, attr, sm) != cudaSuccess ||
-          cudaFuncSetAttribute(nn_argmax_kernel<8, 8, 4>, attr, sm) != cudaSuccess ||
-          cudaFuncSetAttribute(nn_argmax_kernel<8, 4, 4, true>, attr, sm) != cudaSuccess)
+          cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2, true>, attr, sm) != cudaSuccess)
         return RNN_ECUDA;
       di->smem_set = true;
     }
@@ -233,19 +229,17 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
       slot = -1;
     }
   }
-  // Epilogue layout.  Two 256-column accumulators: eight warps, either one
-  // group per accumulator (each warp 256 columns of every other tile, two
-  // copies) or, with one_group, all of them on every tile (each 128 columns
-  // of its lane quadrant in one copy, so an accumulator is held for one copy
-  // and the fold follows its release).  Two 128-column accumulators: eight
-  // warps, one group per accumulator.  Four: sixteen warps copying 64.
+  // Epilogue layout.  Two 256-column accumulators: sixteen warps, all on
+  // every tile, each 64 columns of its lane quadrant in one copy, so an
+  // accumulator is held for one round trip to tensor memory and the fold
+  // follows its release.  Two 128-column accumulators: eight warps, one group
+  // per accumulator.  Four: sixteen warps copying 64, one group per
+  // accumulator.
   const bool wide = g.block_n * g.nacc == 512;
   if (RNN_EPI_WARPS == 8 && g.nacc == 2) {
-    if (wide && one_group)
-      nn_argmax_kernel<8, 4, 4, true><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0,
-                                                                                    q1);
-    else if (wide)
-      nn_argmax_kernel<8, 8, 4><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
+    if (wide)
+      nn_argmax_kernel<16, 2, 2, true><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1,
+                                                                                      q0, q1);
     else
       nn_argmax_kernel<8, 4, 4><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
   } else {
@@ -1146,7 +1140,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_bstride = st.s1;
     F.q_index = st.U;
     F.n_cand = static_cast<int32_t>(N2);
-    if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s, true)) != RNN_OK) return r;
+    if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s)) != RNN_OK) return r;
     if ((r = frm_step(st, h, 1, 0, dt, lgrid, s)) != RNN_OK) return r;
     // half-step 2: U = NN1(V)
     F.q_list = st.list[(h + 1) % 2];
@@ -1155,7 +1149,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_bstride = st.s2;
     F.q_index = st.V;
     F.n_cand = static_cast<int32_t>(N1);
-    if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s, true)) != RNN_OK) return r;
+    if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s)) != RNN_OK) return r;
     if ((r = frm_step(st, h + 1, 0, it == max_iter ? 1 : 0, dt, lgrid, s)) != RNN_OK) return r;
   }
   frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, W1, pairs, cap, count_out, seed_state);
