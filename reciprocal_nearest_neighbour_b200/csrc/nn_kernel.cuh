@@ -28,12 +28,14 @@
 //               serially on every tile; two warps overlap them.
 //   warp 3      query tiles: a TMA box when the rows are contiguous, else
 //               indexed rows gathered with plain loads into the same swizzle
-//   warps 4..   epilogue (8 or 16 warps), in groups that each own one
-//               accumulator (tiles g, g+nacc, ...), so that one group reduces
-//               while another waits.  Warp w reads TMEM lanes 32*(w%4).. and
-//               its part of the columns, folds them 32 at a time into its
-//               row's running maximum, and keeps the first 32-column chunk
-//               that reached it.
+//   warps 4..   epilogue (8 or 16 warps).  With kOneGroup all of them take
+//               every tile, each a column part; otherwise they form groups
+//               that each own one accumulator (tiles g, g+nacc, ...), so that
+//               one group reduces while another waits.  Warp w reads TMEM
+//               lanes 32*(w%4).. and its part of the columns, hands the
+//               accumulator back after its last copy of the tile, folds the
+//               values 32 at a time into its row's running maximum, and keeps
+//               the first 32-column chunk that reached it.
 //
 // The exact lowest index inside the kept chunk is not resolved here: the
 // packed key carries the chunk's first column, and a small pass afterwards

@@ -91,11 +91,6 @@ struct Geometry {
 
 static size_t tables_bytes() { return sizeof(SharedTables); }
 
-// Epilogue warps of the fused kernel: 8 (two accumulators) or 16.
-#ifndef RNN_EPI_WARPS
-#define RNN_EPI_WARPS 8
-#endif
-
 // Candidate tile width for K <= 64: 128 (four accumulators) or 256 (two).
 #ifndef RNN_SMALL_K_BLOCK_N
 #define RNN_SMALL_K_BLOCK_N 256
@@ -211,8 +206,7 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
     if (!di->smem_set) {
       const int sm = 227 * 1024;
       const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-      if (cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2>, attr, sm) != cudaSuccess ||
-          cudaFuncSetAttribute(nn_argmax_kernel<16, 4, 2>, attr, sm) != cudaSuccess ||
+      if (cudaFuncSetAttribute(nn_argmax_kernel<16, 4, 2>, attr, sm) != cudaSuccess ||
           cudaFuncSetAttribute(nn_argmax_kernel<8, 4, 4>, attr, sm) != cudaSuccess ||
           cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2, true>, attr, sm) != cudaSuccess)
         return RNN_ECUDA;
@@ -235,19 +229,13 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
   // follows its release.  Two 128-column accumulators: eight warps, one group
   // per accumulator.  Four: sixteen warps copying 64, one group per
   // accumulator.
-  const bool wide = g.block_n * g.nacc == 512;
-  if (RNN_EPI_WARPS == 8 && g.nacc == 2) {
-    if (wide)
-      nn_argmax_kernel<16, 2, 2, true><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1,
-                                                                                      q0, q1);
-    else
-      nn_argmax_kernel<8, 4, 4><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
-  } else {
-    if (wide)
-      nn_argmax_kernel<16, 4, 2><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
-    else
-      nn_argmax_kernel<16, 2, 2><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
-  }
+  if (g.nacc == 2 && g.block_n == 256)
+    nn_argmax_kernel<16, 2, 2, true><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0,
+                                                                                    q1);
+  else if (g.nacc == 2)
+    nn_argmax_kernel<8, 4, 4><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
+  else
+    nn_argmax_kernel<16, 4, 2><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
   const rnn_status r = launched();
   if (r == RNN_OK && slot >= 0 &&
       cudaEventRecord(static_cast<cudaEvent_t>(g_timer_stop[slot]), s) != cudaSuccess)
