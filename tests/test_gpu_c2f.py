@@ -77,3 +77,22 @@ def test_c2f_large_maps_bitexact():
     maps = [synth.to_storage(x, "f16") for x in (C1, C2, F1, F2)]
     r, ref = _check(maps, (384, 512), 8, 10)
     assert len(ref.crops) == 4 and len(ref.pairs) > 5000
+
+
+def test_c2f_all_crops_off_gives_no_pairs():
+    C1, C2, F1, F2 = _maps(6, 32, 40, 32, 40, 16, 4)
+    r = rnn.c2f_match(dev(C1), dev(C2), dev(F1), dev(F2), crop=(16, 16), seed_stride=4,
+                      min_coarse=10 ** 6)
+    ref = oracle.c2f(C1, C2, F1, F2, crop=(16, 16), seed_stride=4, min_coarse=10 ** 6)
+    assert int(r.count.item()) == 0 and len(ref.pairs) == 0
+    assert np.array_equal(r.crops.cpu().numpy(), ref.crops)
+    assert not ref.crops[:, 5].any()
+
+
+@pytest.mark.parametrize("metric", ["dot", "l2"])
+def test_c2f_bf16_unequal_coarse_ratio(metric):
+    # coarse cells of 3 x 5 pixels (not a divisor of the crops), bf16 maps
+    C1, C2, F1, F2 = _maps(7, 45, 70, 51, 65, 24, 1, "bf16")
+    C1 = synth.to_storage(synth.coarse_map(F1.float().numpy().astype(np.float64), 15, 14), "bf16")
+    C2 = synth.to_storage(synth.coarse_map(F2.float().numpy().astype(np.float64), 17, 13), "bf16")
+    _check([C1, C2, F1, F2], (20, 24), 3, 8, metric=metric)

@@ -192,3 +192,15 @@ def test_pts_frm_continuous_matches_oracle():
     # handful of pairs out of the whole set may differ
     assert len(got ^ exp) <= max(2, len(exp) // 200)
     assert len(exp) > 100
+
+
+def test_pts_frm_starts_out_of_image_are_dropped():
+    H, W = 20, 30
+    P1, P2 = synth.pointmap_pair(120, H, W, quantised=True)
+    rng = np.random.default_rng(121)
+    good = rng.integers(0, H * W, 80).astype(np.int32)
+    starts = np.concatenate([good, np.array([-1, H * W, H * W + 9, -50], np.int32)])
+    r = rnn.pts_frm_match(_cuda32(P1), _cuda32(P2), max_iter=1, pixel_tol=1.5,
+                          init=torch.from_numpy(starts).cuda())
+    ref = oracle.frm_refine(P1, P2, good, pixel_tol=1.5, metric="l2")
+    assert np.array_equal(r.trimmed().cpu().numpy(), ref.pairs.reshape(-1, 2))
