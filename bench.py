@@ -453,6 +453,11 @@ def run_native(args):
     pts = None if args.skip_mnn else _points_leg(dev, lib, w, P, 10)
     # ------------- coarse-to-fine: 1024x768, d = 32, coarse 80x64 cells, d = 256
     c2f = None if args.skip_mnn else _c2f_leg(dev, lib, 10)
+    # -------------- the other FRM configurations: 64 pairs of 512x288; 1024x768
+    configs = None
+    if not args.skip_mnn:
+        configs = {n: _frm_config_leg(dev, n, 5) for n in ("frm_batched_64x512x288",
+                                                          "frm_1024x768")}
 
     # ----------------------------------------------------------- CPU baseline
     cpu = None
@@ -473,7 +478,7 @@ def run_native(args):
                        "global_batch": world * P, "parallelism": f"replicas x{world}",
                        "l2": f"step inputs {2 * A_h.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
             "e2e": e2e, "roofline": roofline, "mnn": mnn, "frm_options": options,
-            "points": pts, "coarse_to_fine": c2f, "cpu_baseline": cpu,
+            "points": pts, "coarse_to_fine": c2f, "frm_configs": configs, "cpu_baseline": cpu,
             "clocks": clocks, "gpu_launches": int(launches),
         }
         print(json.dumps(line), flush=True)
@@ -560,6 +565,32 @@ def _c2f_leg(dev, lib, reps, warmup=3):
             "note": "includes the binding's output allocation; 256 MB L2 flush before every call"}
 
 
+def _frm_config_leg(dev, name, reps, warmup=3):
+    """FRM on a whole workload (all its pairs in one batched call): pairs/s,
+    and the tensor work it did (2*d*N*sum of live queries) per second."""
+    import torch
+    import reciprocal_nearest_neighbour_b200 as rnn
+    from reciprocal_nearest_neighbour_b200 import synth
+    w = synth.WORKLOADS[name]
+    A_h, B_h = synth.make_workload_storage(w, "f16", workers=min(w.pairs, os.cpu_count() or 1))
+    A, B = A_h.to(dev), B_h.to(dev)
+    plan = rnn.FRMPlan(w.pairs, w.H, w.W, w.H, w.W, w.d, torch.float16, w.seed_stride,
+                       w.max_iter, dev, with_seed_state=True)
+    for _ in range(warmup):
+        plan.run(A, B)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    ms, r = _timed_calls(lambda: plan.run(A, B), reps, flush)
+    queries = int(r.seed_state[:, :, 2].sum().item())
+    flops = 2.0 * w.d * w.H * w.W * queries
+    return {"metric": f"FRM image pairs/s, {w.pairs} pair(s) of {w.W}x{w.H}, d={w.d}, stride "
+                      f"{w.seed_stride}, max_iter {w.max_iter}",
+            "value": w.pairs / (ms * 1e-3), "unit": "pairs/s", "ms_per_call": ms,
+            "outputs": int(r.count.sum().item()), "active_queries_per_pair": queries / w.pairs,
+            "tensor_tflops_per_call": flops / (ms * 1e-3) / 1e12, "dtype": "f16",
+            "note": "whole-call time (256 MB L2 flush before every call); the tensor rate counts "
+                    "the live queries' flops over the call, not one kernel"}
+
+
 def run_leg(name, steps, warmup):
     """One leg alone (for profiling): its calls, then one JSON line."""
     import torch
@@ -569,8 +600,10 @@ def run_leg(name, steps, warmup):
     torch.cuda.set_device(dev)
     if name == "points":
         res = _points_leg(dev, lib, synth.WORKLOADS[WORKLOAD], 8, steps, warmup)
-    else:
+    elif name == "c2f":
         res = _c2f_leg(dev, lib, steps, warmup)
+    else:
+        res = _frm_config_leg(dev, name, steps, warmup)
     print(json.dumps({"leg": name, "result": res}), flush=True)
     return 0
 
@@ -600,7 +633,7 @@ def main(argv=None):
     ap.add_argument("--skip-mnn", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
-    ap.add_argument("--leg", choices=["points", "c2f"],
+    ap.add_argument("--leg", choices=["points", "c2f", "frm_batched_64x512x288", "frm_1024x768"],
                     help="run one secondary leg alone (for profiling) and exit")
     ap.add_argument("--nn-case", type=int, nargs=3, metavar=("NQ", "D", "NX"),
                     help="profiling aid: run nn_argmax three times on seeded fp16 "

@@ -317,3 +317,31 @@ def test_workspace_status_ok_after_calls():
                      dtype=torch.uint8, device="cuda")
     rnn.frm_match(a, a, 2, 10, workspace=ws)
     rnn.workspace_status(ws)
+
+
+def test_frm_large_map_fp16():
+    """1024x768 maps, d = 32, 2 % outlier pixels, stride 8 (12 288 seeds),
+    max_iter 15: the whole oracle run."""
+    w = synth.WORKLOADS["frm_1024x768"]
+    D1, D2 = synth.make_workload(w)
+    a, b = synth.to_storage(D1, "f16"), synth.to_storage(D2, "f16")
+    r = rnn.frm_match(dev(a), dev(b), w.seed_stride, w.max_iter, with_seed_state=True)
+    # at 786 432 candidates about a tenth of the trajectories pass a top-2 gap
+    # below 1e-3 somewhere; those are held to the tolerance rule, the rest
+    # must match exactly
+    _frm_tolerant(a, b, w.seed_stride, w.max_iter, r)
+    assert int(r.count[0]) > 1000
+
+
+def test_mnn_coarse_tokens_fp16():
+    """The coarse reciprocal set on 80x64 tokens, d = 256, fp16 unit vectors."""
+    w = synth.WORKLOADS["mnn_coarse_80x64"]
+    D1, D2 = synth.make_workload(w)
+    a, b = synth.to_storage(D1, "f16"), synth.to_storage(D2, "f16")
+    r = rnn.mnn_exhaustive(dev(a), dev(b), with_nn=True)
+    ref = oracle.mnn(a, b)
+    A, B = a.reshape(-1, w.d), b.reshape(-1, w.d)
+    check_nn_tolerant(A, B, r.rowarg.cpu().numpy(), r.rowmax.cpu().numpy(), ref.row)
+    check_nn_tolerant(B, A, r.colarg.cpu().numpy(), r.colmax.cpu().numpy(), ref.col)
+    assert check_mnn_tolerant(r.trimmed().cpu().numpy(), ref) <= 5
+    assert len(ref.pairs) > 1000
