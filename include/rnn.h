@@ -412,6 +412,19 @@ uint64_t rnn_launch_count(void);
 void rnn_set_kernel_timer(void *const *start_events, void *const *stop_events, int capacity,
                           int *recorded);
 
+/*
+ * Failure-detection test hook (no use in production).  While `on` is
+ * nonzero, every launch of the fused similarity+argmax kernel loads no
+ * candidate tile, so the bounded wait of its MMA warps on the first tile runs
+ * out after `wait_limit_ns` (0: the default of 1 s); the kernel then stops
+ * all its warps, frees tensor memory and returns, and the call's workspace
+ * status reads RNN_ETIMEOUT (rnn_workspace_status).  Results of those calls
+ * are undefined but every index written is in range.  Nothing faults, traps
+ * or hangs; later calls with the hook off are unaffected.  Global to the
+ * process, not thread-safe against concurrent calls.
+ */
+void rnn_test_stall_loads(int on, uint64_t wait_limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

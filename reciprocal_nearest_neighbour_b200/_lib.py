@@ -46,6 +46,7 @@ EXPORTS = (
     "rnn_c2f_match",
     "rnn_mnn_mutual_workspace_size",
     "rnn_mnn_mutual",
+    "rnn_test_stall_loads",
 )
 
 STATUS = {
@@ -126,6 +127,7 @@ def load():
                               P, I64, P, P, P, SZ, P]),
         "rnn_mnn_mutual_workspace_size": (SZ, [I64]),
         "rnn_mnn_mutual": (I, [P, I64, P, I64, P, I64, P, P, SZ, P]),
+        "rnn_test_stall_loads": (None, [I, ctypes.c_uint64]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

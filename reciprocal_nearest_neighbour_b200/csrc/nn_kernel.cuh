@@ -99,6 +99,8 @@ struct NNParams {
   int min_tiles;    // fewest candidate tiles per unit (amortises the query-tile load)
   int* err;         // device error word
   unsigned long long wait_limit_ns;
+  int stall_loads;  // failure-detection test: the producer loads no candidate tile, so the
+                    // MMA warps' bounded wait on it runs out and the kernel reports a timeout
 };
 
 // Packed key: larger is better (higher score, then lower index).
@@ -370,11 +372,13 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
             break;
           }
           const uint32_t fb = smem_u32(&full_bar[stage]);
-          mbar_arrive_expect_tx(fb, stage_bytes);
-          const uint32_t dst = smem_u32(x_tiles + static_cast<size_t>(stage) * stage_bytes);
-          for (int kk = 0; kk < p.nkb; ++kk)
-            tma_load_3d(dst + kk * kblk_bytes_x, map, fb, kk * p.kb, t * p.block_n, ui.b);
-          ++issued;
+          if (!p.stall_loads) {
+            mbar_arrive_expect_tx(fb, stage_bytes);
+            const uint32_t dst = smem_u32(x_tiles + static_cast<size_t>(stage) * stage_bytes);
+            for (int kk = 0; kk < p.nkb; ++kk)
+              tma_load_3d(dst + kk * kblk_bytes_x, map, fb, kk * p.kb, t * p.block_n, ui.b);
+            ++issued;
+          }
           if (++stage == p.stages) {
             stage = 0;
             phase ^= 1u;
@@ -603,6 +607,9 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
           // stages is a multiple of nacc, so done_bar[stage] is only ever
           // used by this group's tiles, and its next phase needs this tile's
           // accumulator back: the parity below cannot be a phase behind
+          // every lane polls the same barrier and abort word, so the outcome
+          // is the same in all lanes unless the barrier completes during an
+          // abort; a warp-wide vote here costs 8 % of the sweep
           if (!mbar_wait_sleep(smem_u32(&done_bar[stage]), phase, abort_flag, p.err,
                                kErrWaitEpilogue, lim)) {
             ok = false;

@@ -172,6 +172,9 @@ static rnn_status make_map(CUtensorMap* m, const void* base, int d, int64_t rows
 
 // ------------------------------------------------------------- diagnostics
 static std::atomic<uint64_t> g_launches{0};
+// failure-detection test hook (rnn_test_stall_loads)
+static std::atomic<int> g_stall_loads{0};
+static std::atomic<unsigned long long> g_stall_limit_ns{kWaitLimitNs};
 static void* const* g_timer_start = nullptr;
 static void* const* g_timer_stop = nullptr;
 static int g_timer_cap = 0;
@@ -200,7 +203,9 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
     const int tile_cycles = (g.kpad / 16) * (g.block_n / 2);
     p.min_tiles = 4096 / tile_cycles > 2 ? 4096 / tile_cycles : 2;
   }
-  p.wait_limit_ns = kWaitLimitNs;
+  p.stall_loads = g_stall_loads.load(std::memory_order_relaxed);
+  p.wait_limit_ns = p.stall_loads ? g_stall_limit_ns.load(std::memory_order_relaxed)
+                                  : kWaitLimitNs;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!di->smem_set) {
@@ -378,6 +383,9 @@ __device__ __forceinline__ float dot_rows(const uint16_t* a, const uint16_t* b, 
 template <bool kBf16>
 __device__ __forceinline__ int locate_chunk(const uint16_t* q, const uint16_t* X, int n_cand,
                                             int ld, int c0, float* best = nullptr) {
+  // a key no candidate reached (only after a fused kernel that gave up on a
+  // wait) leaves index -1: locate chunk 0 so that every later index is valid
+  if (c0 < 0 || c0 >= n_cand) c0 = 0;
   const int lane = threadIdx.x & 31;
   const int j = c0 + lane;
   float sc = -__int_as_float(0x7f800000);
@@ -1331,7 +1339,7 @@ const char* rnn_status_string(rnn_status s) {
   return "unknown rnn_status";
 }
 
-int rnn_abi_version(void) { return 5; }
+int rnn_abi_version(void) { return 6; }
 
 uint64_t rnn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -1343,6 +1351,12 @@ void rnn_set_kernel_timer(void* const* start_events, void* const* stop_events, i
   g_timer_stop = on ? stop_events : nullptr;
   g_timer_cap = on ? capacity : 0;
   g_timer_count = on ? recorded : nullptr;
+}
+
+void rnn_test_stall_loads(int on, uint64_t wait_limit_ns) {
+  g_stall_limit_ns.store(on && wait_limit_ns > 0 ? wait_limit_ns : kWaitLimitNs,
+                         std::memory_order_relaxed);
+  g_stall_loads.store(on ? 1 : 0, std::memory_order_relaxed);
 }
 
 rnn_status rnn_workspace_status(const void* workspace, rnn_stream_t stream) {

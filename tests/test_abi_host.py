@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rnn_abi_version() == 5
+    assert lib.rnn_abi_version() == 6
     for code, name in _lib.STATUS.items():
         assert lib.rnn_status_string(code).decode().startswith(name)
 
@@ -301,3 +301,9 @@ def test_mnn_mutual_argument_errors(lib):
     assert f(FAKE, 100, FAKE, 10, FAKE, 9, FAKE, FAKE, ws, None) == ECAP
     assert f(FAKE, 100, FAKE, 10, FAKE, 10, FAKE, FAKE, ws - 1, None) == EWS
     assert f(FAKE, 100, FAKE, 10, FAKE, 10, FAKE, FAKE + 8, ws, None) == EWS
+
+
+def test_stall_hook_is_a_host_switch(lib):
+    # sets and clears process-global state only; nothing is launched
+    lib.rnn_test_stall_loads(1, 1000)
+    lib.rnn_test_stall_loads(0, 0)
