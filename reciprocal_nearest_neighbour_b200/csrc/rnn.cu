@@ -16,6 +16,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "nn_kernel.cuh"
 #include "rnn.h"
 
@@ -28,6 +30,15 @@ constexpr int kMnnChunk = 4096;  // rows per block in the mutual test (4 per thr
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
 
 static size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// An NVTX range over one ABI call (visible in Nsight Systems; a no-op
+// unless a tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 struct Carve {
   uint8_t* base;
@@ -1040,6 +1051,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
                           float pixel_tol, int32_t* pairs, int64_t cap, int32_t* count_out,
                           int32_t* seed_state, int32_t* basin, void* ws, size_t ws_bytes,
                           cudaStream_t s, const int32_t* pair_on = nullptr) {
+  NvtxRange nvtx_range("rnn_frm_match");
   if (B < 1) return RNN_EINVAL;
   if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
   if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || max_iter < 1) return RNN_EINVAL;
@@ -1264,6 +1276,7 @@ static rnn_status frm_run_pts(int B, const float* P1, int64_t bs1, const float* 
                               int32_t* pairs, int64_t cap, int32_t* count_out,
                               int32_t* seed_state, int32_t* basin, void* ws, size_t ws_bytes,
                               cudaStream_t s) {
+  NvtxRange nvtx_range("rnn_pts_frm_match");
   if (B < 1) return RNN_EINVAL;
   if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
   if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || max_iter < 1) return RNN_EINVAL;
@@ -1398,6 +1411,7 @@ rnn_status rnn_nn_argmax_ex(const void* Q, int64_t nq, const void* X, int64_t nx
                             rnn_dtype dtype, rnn_metric metric, int32_t* idx_out,
                             float* score_out, void* workspace, size_t ws_bytes,
                             rnn_stream_t stream) {
+  NvtxRange nvtx_range("rnn_nn_argmax");
   if (nq < 0 || nx < 1 || nq > INT32_MAX || nx > INT32_MAX) return RNN_EINVAL;
   if (!valid_dtype(dtype) || !valid_metric(metric)) return RNN_EINVAL;
   rnn_status r = check_desc(X, d);
@@ -1516,6 +1530,7 @@ rnn_status rnn_mnn_exhaustive_ex(const void* D1, int H1, int W1, const void* D2,
                                  int64_t cap, int32_t* count_out, int32_t* rowarg_out,
                                  float* rowmax_out, int32_t* colarg_out, float* colmax_out,
                                  void* workspace, size_t ws_bytes, rnn_stream_t stream) {
+  NvtxRange nvtx_range("rnn_mnn_exhaustive");
   if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0) return RNN_EINVAL;
   if (!valid_dtype(dtype) || !valid_metric(metric)) return RNN_EINVAL;
   rnn_status r = check_desc(D1, d);
@@ -1691,6 +1706,7 @@ size_t rnn_mnn_mutual_workspace_size(int64_t n1) {
 rnn_status rnn_mnn_mutual(const int32_t* rowarg, int64_t n1, const int32_t* colarg, int64_t n2,
                           int32_t* pairs_out, int64_t cap, int32_t* count_out, void* workspace,
                           size_t ws_bytes, rnn_stream_t stream) {
+  NvtxRange nvtx_range("rnn_mnn_mutual");
   if (n1 < 1 || n2 < 1 || n1 > INT32_MAX || n2 > INT32_MAX) return RNN_EINVAL;
   if (!rowarg || !colarg || !pairs_out || !count_out) return RNN_EINVAL;
   if (cap < (n1 < n2 ? n1 : n2)) return RNN_ECAPACITY;
@@ -1820,6 +1836,7 @@ rnn_status rnn_c2f_match(const void* C1, int Hc1, int Wc1, const void* C2, int H
                          int seed_stride, int max_iter, int min_coarse, int32_t* pairs_out,
                          int64_t cap, int32_t* count_out, int32_t* crops_out, void* workspace,
                          size_t ws_bytes, rnn_stream_t stream) {
+  NvtxRange nvtx_range("rnn_c2f_match");
   C2FGeom g;
   if (!c2f_geom(Hc1, Wc1, Hc2, Wc2, H1, W1, H2, W2, crop_h, crop_w, min_coarse, &g))
     return RNN_EINVAL;
@@ -1898,6 +1915,7 @@ size_t rnn_pts_nn_workspace_size(int64_t nq, int64_t nx) {
 
 rnn_status rnn_pts_nn(const float* Q, int64_t nq, const float* X, int64_t nx, int32_t* idx_out,
                       float* dist2_out, void* workspace, size_t ws_bytes, rnn_stream_t stream) {
+  NvtxRange nvtx_range("rnn_pts_nn");
   if (nq < 0 || nx < 1 || nq > INT32_MAX) return RNN_EINVAL;
   if (nx > kPtsMaxSet) return RNN_EUNSUPPORTED;
   if (!X || (nq > 0 && (!Q || !idx_out))) return RNN_EINVAL;
@@ -1944,6 +1962,7 @@ rnn_status rnn_pts_mnn(const float* P1, int H1, int W1, const float* P2, int H2,
                        int32_t* pairs_out, int64_t cap, int32_t* count_out, int32_t* rowarg_out,
                        float* rowd2_out, int32_t* colarg_out, float* cold2_out, void* workspace,
                        size_t ws_bytes, rnn_stream_t stream) {
+  NvtxRange nvtx_range("rnn_pts_mnn");
   if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0) return RNN_EINVAL;
   if (!P1 || !P2 || !pairs_out || !count_out) return RNN_EINVAL;
   if (!pts_ptr_ok(P1) || !pts_ptr_ok(P2)) return RNN_EALIGN;

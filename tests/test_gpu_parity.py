@@ -345,3 +345,28 @@ def test_mnn_coarse_tokens_fp16():
     check_nn_tolerant(B, A, r.colarg.cpu().numpy(), r.colmax.cpu().numpy(), ref.col)
     assert check_mnn_tolerant(r.trimmed().cpu().numpy(), ref) <= 5
     assert len(ref.pairs) > 1000
+
+
+def test_repeat_runs_are_identical_other_paths():
+    """Deterministic reductions: three runs of coarse-to-fine, point-map FRM
+    and the Euclidean exhaustive set give identical bits (a race would show
+    as run-to-run differences)."""
+    w = synth.WORKLOADS["frm_512x384"]
+    D1, D2 = synth.make_workload(w)
+    a, b = dev(synth.to_storage(D1, "f16")), dev(synth.to_storage(D2, "f16"))
+    C1 = dev(synth.to_storage(synth.coarse_map(D1, 48, 64), "f16"))
+    C2 = dev(synth.to_storage(synth.coarse_map(D2, 48, 64), "f16"))
+    c = [rnn.c2f_match(C1, C2, a, b, crop=(192, 256), seed_stride=4) for _ in range(3)]
+    for o in c[1:]:
+        assert torch.equal(o.trimmed(), c[0].trimmed()) and torch.equal(o.crops, c[0].crops)
+    P1, P2 = synth.pointmap_pair(9, w.H, w.W)
+    p1 = torch.from_numpy(P1.astype(np.float32)).cuda()
+    p2 = torch.from_numpy(P2.astype(np.float32)).cuda()
+    f = [rnn.pts_frm_match(p1, p2, seed_stride=8, with_seed_state=True) for _ in range(3)]
+    for o in f[1:]:
+        assert torch.equal(o.seed_state, f[0].seed_state)
+        assert torch.equal(o.trimmed(), f[0].trimmed())
+    m = [rnn.mnn_exhaustive(a[:128], b[:128], with_nn=True, metric="l2") for _ in range(3)]
+    for o in m[1:]:
+        assert torch.equal(o.rowmax, m[0].rowmax) and torch.equal(o.colarg, m[0].colarg)
+        assert torch.equal(o.trimmed(), m[0].trimmed())
