@@ -60,6 +60,7 @@ constexpr int kChunk = 32;       // columns folded per maximum; the locate pass 
 constexpr int kMaxBatchTable = 1024;
 constexpr int kMaxStages = 16;   // candidate ring depth limit
 constexpr int kMaxAcc = 4;       // accumulator buffers in tensor memory (512 columns in all)
+constexpr int kUnitTiles = 8;    // fixed cost of a work unit, in tiles (split-count choice)
 
 // Error bits written to the device error word.
 constexpr int kErrWaitProducer = 1 << 0;
@@ -314,11 +315,6 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
     if (p.fam[0].q_tma) tma_prefetch_desc(&qmap0);
     if (p.nfam > 1 && p.fam[1].q_tma) tma_prefetch_desc(&qmap1);
   }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(misc), ncols);
-    tmem_relinquish();
-  }
-
   // unit table
   for (int f = 0; f < 2; ++f) {
     if (f < p.nfam) {
@@ -337,8 +333,34 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
       }
       tiles_total += T->fam_tiles[f];
     }
-    int S = tiles_total > 0 ? (p.target_units + tiles_total - 1) / tiles_total : 1;
-    if (S < 1) S = 1;
+    // split count: at least enough units for the target, and among the
+    // counts up to 2x that (units of at least min_tiles tiles) the one whose
+    // round-robin deal gives the CTAs the smallest largest share
+    int S0 = tiles_total > 0 ? (p.target_units + tiles_total - 1) / tiles_total : 1;
+    if (S0 < 1) S0 = 1;
+    int Smax = 1;
+    for (int f = 0; f < 2; ++f)
+      if (f < p.nfam) Smax = max(Smax, T->ntiles[f] / max(1, p.min_tiles));
+    Smax = max(S0, min(2 * S0, Smax));
+    int S = S0;
+    long long best = -1;
+    for (int c = S0; c <= Smax; ++c) {
+      long long units = 0;
+      int biggest = 1;  // tiles of the largest unit
+      for (int f = 0; f < 2; ++f) {
+        if (T->fam_tiles[f] == 0) continue;
+        const int Sf = max(1, min(c, T->ntiles[f] / max(1, p.min_tiles)));
+        units += static_cast<long long>(T->fam_tiles[f]) * Sf;
+        biggest = max(biggest, (T->ntiles[f] + Sf - 1) / Sf);
+      }
+      // each unit also costs about kUnitTiles tiles (query tile, pipeline
+      // fill, final merge)
+      const long long share = (units + gridDim.x - 1) / gridDim.x * (biggest + kUnitTiles);
+      if (best < 0 || share < best) {
+        best = share;
+        S = c;
+      }
+    }
     int total = 0;
     for (int f = 0; f < 2; ++f) {
       const int Sf = max(1, min(S, T->ntiles[f] / max(1, p.min_tiles)));
@@ -348,11 +370,17 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
     }
     T->total_units = total;
   }
+  __syncthreads();
+  const int total_units = T->total_units;
+  if (total_units == 0) return;  // no live query (late FRM half-steps): no tensor memory
+  if (warp == 1) {
+    tmem_alloc(smem_u32(misc), ncols);
+    tmem_relinquish();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = misc[0];
-  const int total_units = T->total_units;
   const uint64_t lim = p.wait_limit_ns;
 
   if (warp == 0) {
