@@ -243,6 +243,35 @@ rnn_status rnn_frm_match_ex(int B, const void *D1, int64_t d1_batch_stride, cons
                             size_t ws_bytes, rnn_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * FRM graph plans.  rnn_frm_graph_create records one rnn_frm_match_ex call
+ * (same arguments, minus the stream) as a CUDA graph and instantiates it;
+ * rnn_frm_graph_launch replays it on a stream.  Iterations 2..max_iter sit
+ * in conditional nodes: the last step kernel of each iteration enables the
+ * next one only while some seed of some pair is still active, so iterations
+ * after convergence launch nothing (the results are those of the call, bit
+ * for bit: an iteration with no active seed changes no state).
+ *   The plan holds the device pointers it was given (maps, starts, outputs,
+ *   workspace): every launch reads the maps' current contents and rewrites
+ *   the outputs; the buffers must outlive the plan, and launches of one plan
+ *   must not overlap (they share the workspace).  max_iter <= 64
+ *   (RNN_EUNSUPPORTED).  The argument checks and errors are those of
+ *   rnn_frm_match_ex, plus RNN_ECUDA if graph creation fails.  The status
+ *   word of the workspace (rnn_workspace_status) reports a launch's errors.
+ *   *graph_out is owned by the caller: release it with rnn_frm_graph_destroy
+ *   (NULL is accepted).
+ */
+typedef struct rnn_frm_graph *rnn_frm_graph_t;
+rnn_status rnn_frm_graph_create(int B, const void *D1, int64_t d1_batch_stride, const void *D2,
+                                int64_t d2_batch_stride, int H1, int W1, int H2, int W2, int d,
+                                rnn_dtype dtype, rnn_metric metric, const int32_t *init_xy1,
+                                int64_t n_init, int seed_stride, int max_iter, float pixel_tol,
+                                int32_t *pairs_out, int64_t cap, int32_t *count_out,
+                                int32_t *seed_state_out, int32_t *basin_out, void *workspace,
+                                size_t ws_bytes, rnn_frm_graph_t *graph_out);
+rnn_status rnn_frm_graph_launch(rnn_frm_graph_t graph, rnn_stream_t stream);
+void rnn_frm_graph_destroy(rnn_frm_graph_t graph);
+
+/* ------------------------------------------------------------------------
  * The reciprocal set from NN arrays computed elsewhere (cv-learn.com "MASt3R"
  * note, paragraph "Fast reciprocal matching (FRM)": M = {(i, j) | j = NN2(i)
  * and i = NN1(j)}), e.g. when the rows of both maps are split over several
@@ -398,7 +427,8 @@ rnn_status rnn_nn_argmax_noalloc(const void *Q, int64_t nq, const void *X, int64
  * Diagnostics for benchmarking (no effect on results).
  *
  * rnn_launch_count: number of kernels this library has launched in this
- *   process (all entry points, all devices).
+ *   process (all entry points, all devices), not counting those that graph
+ *   plans record or replay; recording a plan does not use the timer below.
  * rnn_set_kernel_timer: while set, every launch of the fused
  *   similarity+argmax kernel is bracketed by cudaEventRecord(start_events[i])
  *   and cudaEventRecord(stop_events[i]) on the launch stream, with

@@ -34,6 +34,7 @@ Results stay on the device; pair lists come back as ``(pairs, count)`` with
 """
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass
 from typing import Optional
 
@@ -46,7 +47,7 @@ __all__ = [
     "nn_argmax", "mnn_exhaustive", "frm_match", "frm_match_batched", "frm_num_seeds",
     "frm_max_pairs", "workspace_status", "trim", "MNNResult", "FRMResult", "RNNError",
     "RNNLibraryError", "FRMPlan", "frm_match_ex", "frm_refine", "pts_nn", "pts_mnn",
-    "pts_frm_match", "c2f_match", "C2FResult", "mnn_mutual",
+    "pts_frm_match", "c2f_match", "C2FResult", "mnn_mutual", "FRMGraph",
 ]
 
 _DT = {torch.float16: _lib.RNN_F16, torch.bfloat16: _lib.RNN_BF16}
@@ -359,6 +360,85 @@ def frm_match_ex(D1: torch.Tensor, D2: torch.Tensor, *, seed_stride: int = 8,
         _ptr(out.seed_state), _ptr(out.basin), workspace.data_ptr(), workspace.numel(),
         _stream(D1)), "rnn_frm_match_ex")
     return out
+
+
+class FRMGraph:
+    """FRM of two resident maps recorded once as a CUDA graph plan.
+
+    ``FRMGraph(D1, D2, ...)`` takes the arguments of :func:`frm_match_ex`
+    (without ``workspace``); ``launch()`` re-runs the match on the current
+    contents of ``D1``/``D2`` into the same output tensors, on the current
+    stream.  Iterations after the last active seed converged launch nothing.
+    The plan keeps ``D1``, ``D2`` and ``init`` alive; launches must not
+    overlap.
+    """
+
+    def __init__(self, D1: torch.Tensor, D2: torch.Tensor, *, seed_stride: int = 8,
+                 max_iter: int = 10, metric: str = "dot", init: Optional[torch.Tensor] = None,
+                 pixel_tol: float = 0.0, with_basin: bool = False,
+                 with_seed_state: bool = False):
+        batched = D1.dim() == 4
+        _check_map(D1, "D1", 4 if batched else 3)
+        _check_map(D2, "D2", 4 if batched else 3)
+        if D1.dtype != D2.dtype or D1.shape[-1] != D2.shape[-1]:
+            raise ValueError("D1 and D2 must share dtype and d")
+        if batched and D1.shape[0] != D2.shape[0]:
+            raise ValueError("D1 and D2 must share B")
+        B = D1.shape[0] if batched else 1
+        H1, W1, d = D1.shape[-3:]
+        H2, W2, _ = D2.shape[-3:]
+        lib = _lib.load()
+        m = _metric(metric)
+        dev = D1.device
+        n_init = -1
+        if init is not None:
+            if not isinstance(init, torch.Tensor) or not init.is_cuda or \
+                    init.dtype != torch.int32:
+                raise ValueError("init must be a CUDA int32 tensor")
+            init = init.reshape(B, -1).contiguous()
+            n_init = k = init.shape[1]
+        else:
+            k = int(lib.rnn_frm_num_seeds(H1, W1, seed_stride)) if seed_stride >= 1 else 0
+        cap = max(1, k if pixel_tol > 0 else min(k, H2 * W2))
+        self._keep = (D1, D2, init)
+        self.result = FRMResult(
+            torch.empty((B, cap, 2), dtype=torch.int32, device=dev),
+            torch.zeros(B, dtype=torch.int32, device=dev),
+            torch.empty((B, max(k, 1), 4), dtype=torch.int32, device=dev)
+            if with_seed_state else None,
+            torch.empty((B, H1 * W1 + 1), dtype=torch.int32, device=dev)
+            if with_basin else None)
+        self.workspace = _workspace(lib.rnn_frm_workspace_size_ex(
+            B, H1, W1, H2, W2, d, m, seed_stride, n_init), dev)
+        r = self.result
+        handle = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _lib.check(lib.rnn_frm_graph_create(
+                B, D1.data_ptr(), H1 * W1 * d, D2.data_ptr(), H2 * W2 * d, H1, W1, H2, W2, d,
+                _dtype_code(D1), m, _ptr(init), max(n_init, 0), seed_stride, max_iter,
+                float(pixel_tol), r.pairs.data_ptr(), cap, r.count.data_ptr(),
+                _ptr(r.seed_state), _ptr(r.basin), self.workspace.data_ptr(),
+                self.workspace.numel(), ctypes.byref(handle)), "rnn_frm_graph_create")
+        self._handle = handle
+
+    def launch(self) -> FRMResult:
+        if not self._handle:
+            raise RuntimeError("the graph plan is closed")
+        lib = _lib.load()
+        _lib.check(lib.rnn_frm_graph_launch(self._handle, _stream(self._keep[0])),
+                   "rnn_frm_graph_launch")
+        return self.result
+
+    def close(self) -> None:
+        if getattr(self, "_handle", None):
+            _lib.load().rnn_frm_graph_destroy(self._handle)
+            self._handle = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown: the process releases the graph
+            pass
 
 
 def frm_refine(D1: torch.Tensor, D2: torch.Tensor, init: torch.Tensor, pixel_tol: float = 0.0,

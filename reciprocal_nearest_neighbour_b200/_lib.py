@@ -47,6 +47,9 @@ EXPORTS = (
     "rnn_mnn_mutual_workspace_size",
     "rnn_mnn_mutual",
     "rnn_test_stall_loads",
+    "rnn_frm_graph_create",
+    "rnn_frm_graph_launch",
+    "rnn_frm_graph_destroy",
 )
 
 STATUS = {
@@ -128,6 +131,10 @@ def load():
         "rnn_mnn_mutual_workspace_size": (SZ, [I64]),
         "rnn_mnn_mutual": (I, [P, I64, P, I64, P, I64, P, P, SZ, P]),
         "rnn_test_stall_loads": (None, [I, ctypes.c_uint64]),
+        "rnn_frm_graph_create": (I, [I, P, I64, P, I64, I, I, I, I, I, I, I, P, I64, I, I,
+                                     ctypes.c_float, P, I64, P, P, P, P, SZ, P]),
+        "rnn_frm_graph_launch": (I, [P, P]),
+        "rnn_frm_graph_destroy": (None, [P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)

@@ -15,6 +15,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -28,6 +29,7 @@ constexpr size_t kAlign = 256;
 constexpr int kSmallThreads = 1024;
 constexpr int kMnnChunk = 4096;  // rows per block in the mutual test (4 per thread)
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
+constexpr int kMaxGraphIters = 64;  // max_iter of a graph plan
 
 static size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -191,10 +193,13 @@ static void* const* g_timer_stop = nullptr;
 static int g_timer_cap = 0;
 static int* g_timer_count = nullptr;
 
+// Recording a graph plan: launches are neither counted nor timed.
+static thread_local bool t_capturing = false;
+
 // Check the last launch and count it.
 static rnn_status launched() {
   if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!t_capturing) g_launches.fetch_add(1, std::memory_order_relaxed);
   return RNN_OK;
 }
 
@@ -230,7 +235,7 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
     }
   }
   int slot = -1;
-  if (g_timer_count && g_timer_start && g_timer_stop) {
+  if (!t_capturing && g_timer_count && g_timer_start && g_timer_stop) {
     slot = (*g_timer_count)++;
     if (slot < g_timer_cap) {
       if (cudaEventRecord(static_cast<cudaEvent_t>(g_timer_start[slot]), s) != cudaSuccess)
@@ -641,6 +646,7 @@ __global__ void mutual_write_kernel(const int32_t* rowarg, int64_t n1, const int
 // and the metric of its brute-force matcher.
 struct FrmState {
   int* err;
+  unsigned* done;   // blocks of a step kernel that finished (graph plans: last-block test)
   // Active seeds of half-step h: list[h % 2] (slots, [B][k], in no particular
   // order) and cnt[h % 3] ([B]).  The kernel of half-step h appends the
   // seeds that stay active to list[(h+1) % 2], counting in cnt[(h+1) % 3],
@@ -697,6 +703,7 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int
                          rnn_metric metric, FrmState* st, FrmCopies* cp) {
   Carve c(ws);
   st->err = c.take<int>(64);
+  st->done = c.take<unsigned>(1);
   for (int i = 0; i < 3; ++i) st->cnt[i] = c.take<int32_t>(B);
   st->nseeds = c.take<int32_t>(B);
   const int64_t kk = k > 0 ? k : 1;
@@ -779,7 +786,10 @@ __global__ void frm_init_kernel(FrmState st, int W1, int S) {
       st.cnt[1][b] = 0;
       st.nseeds[b] = k;
     }
-    if (threadIdx.x == 0) *st.err = 0;
+    if (threadIdx.x == 0) {
+      *st.err = 0;
+      *st.done = 0u;
+    }
   }
 }
 
@@ -793,7 +803,10 @@ __global__ void frm_starts_clear_kernel(FrmState st) {
     if (t < nbits) st.bitmap[t] = 0u;
     else st.basin[t - nbits] = -1;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *st.err = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *st.err = 0;
+    *st.done = 0u;
+  }
 }
 
 // Step 2: mark every start in its pair's bitmap (starts outside the image
@@ -876,7 +889,8 @@ __device__ __forceinline__ void frm_apply(const FrmState& st, int b, int64_t bas
 // 2 against image 1, in the row forms the tensor cores read), then lane 0
 // applies it (frm_apply).
 template <bool kBf16>
-__global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter) {
+__global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter,
+                                cudaGraphConditionalHandle next) {
   const int32_t* cnt_in = st.cnt[h % 3];
   int32_t* cnt_out = st.cnt[(h + 1) % 3];
   const int32_t* list_in = st.list[h % 2];
@@ -903,6 +917,22 @@ __global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter)
     if ((threadIdx.x & 31) == 0) {
       st.keys[base + i] = 0ull;
       frm_apply(st, b, base, s, j, nn2_half, last_iter, list_out, cnt_out);
+    }
+  }
+  if (next) {
+    // graph plans: the last block to finish enables the next iteration's
+    // conditional node when some seed of some pair is still active
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(st.done, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (s_last && threadIdx.x == 0) {
+      __threadfence();
+      int any = 0;
+      for (int b = 0; b < st.B; ++b) any |= __ldcg(cnt_out + b) > 0;
+      cudaGraphSetConditional(next, any ? 1u : 0u);
+      *st.done = 0u;
     }
   }
 }
@@ -990,11 +1020,12 @@ static int grid_for(int64_t n, int sms) {
 }
 
 static rnn_status frm_step(const FrmState& st, int h, int nn2_half, int last_iter,
-                           rnn_dtype dt, int grid, cudaStream_t s) {
+                           rnn_dtype dt, int grid, cudaStream_t s,
+                           cudaGraphConditionalHandle next = 0) {
   if (dt == RNN_BF16)
-    frm_step_kernel<true><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter);
+    frm_step_kernel<true><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter, next);
   else
-    frm_step_kernel<false><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter);
+    frm_step_kernel<false><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter, next);
   return launched();
 }
 
@@ -1050,7 +1081,11 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
                           const int32_t* init, int64_t n_init, int S, int max_iter,
                           float pixel_tol, int32_t* pairs, int64_t cap, int32_t* count_out,
                           int32_t* seed_state, int32_t* basin, void* ws, size_t ws_bytes,
-                          cudaStream_t s, const int32_t* pair_on = nullptr) {
+                          cudaStream_t s, const int32_t* pair_on = nullptr,
+                          cudaStream_t body_stream = nullptr) {
+  // body_stream non-null: `s` is capturing a graph plan; iterations 2..max_iter
+  // go into conditional (if) nodes, each enabled by the previous iteration's
+  // last step kernel when a seed is still active, and captured on body_stream
   NvtxRange nvtx_range("rnn_frm_match");
   if (B < 1) return RNN_EINVAL;
   if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
@@ -1139,8 +1174,10 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   F.nbatch = B;
   F.keys = st.keys;
   F.key_bstride = k;
-  for (int it = 1; it <= max_iter; ++it) {
+  // one iteration (two half-steps) on stream q; the NN1 step enables `next`
+  auto iteration = [&](int it, cudaStream_t q, cudaGraphConditionalHandle next) -> rnn_status {
     const int h = 2 * (it - 1);
+    rnn_status e;
     // half-step 1: V = NN2(U)
     F.q_list = st.list[h % 2];
     F.q_count_dev = st.cnt[h % 3];
@@ -1148,8 +1185,8 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_bstride = st.s1;
     F.q_index = st.U;
     F.n_cand = static_cast<int32_t>(N2);
-    if ((r = launch_nn(p, map2, map2, map2, map2, g, di, s)) != RNN_OK) return r;
-    if ((r = frm_step(st, h, 1, 0, dt, lgrid, s)) != RNN_OK) return r;
+    if ((e = launch_nn(p, map2, map2, map2, map2, g, di, q)) != RNN_OK) return e;
+    if ((e = frm_step(st, h, 1, 0, dt, lgrid, q)) != RNN_OK) return e;
     // half-step 2: U = NN1(V)
     F.q_list = st.list[(h + 1) % 2];
     F.q_count_dev = st.cnt[(h + 1) % 3];
@@ -1157,8 +1194,52 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_bstride = st.s2;
     F.q_index = st.V;
     F.n_cand = static_cast<int32_t>(N1);
-    if ((r = launch_nn(p, map1, map1, map1, map1, g, di, s)) != RNN_OK) return r;
-    if ((r = frm_step(st, h + 1, 0, it == max_iter ? 1 : 0, dt, lgrid, s)) != RNN_OK) return r;
+    if ((e = launch_nn(p, map1, map1, map1, map1, g, di, q)) != RNN_OK) return e;
+    return frm_step(st, h + 1, 0, it == max_iter ? 1 : 0, dt, lgrid, q, next);
+  };
+  if (!body_stream) {
+    for (int it = 1; it <= max_iter; ++it)
+      if ((r = iteration(it, s, 0)) != RNN_OK) return r;
+  } else {
+    cudaStreamCaptureStatus cst;
+    cudaGraph_t cg = nullptr;
+    if (cudaStreamGetCaptureInfo(s, &cst, nullptr, &cg, nullptr, nullptr) != cudaSuccess ||
+        cst != cudaStreamCaptureStatusActive || !cg)
+      return RNN_ECUDA;
+    // condition handles of iterations 2..max_iter (0 unless enabled this launch)
+    cudaGraphConditionalHandle hnd[kMaxGraphIters + 1] = {};
+    for (int it = 2; it <= max_iter; ++it)
+      if (cudaGraphConditionalHandleCreate(&hnd[it], cg, 0, cudaGraphCondAssignDefault) !=
+          cudaSuccess)
+        return RNN_ECUDA;
+    if ((r = iteration(1, s, max_iter > 1 ? hnd[2] : 0)) != RNN_OK) return r;
+    for (int it = 2; it <= max_iter; ++it) {
+      const cudaGraphNode_t* deps = nullptr;
+      size_t ndeps = 0;
+      if (cudaStreamGetCaptureInfo(s, &cst, nullptr, nullptr, &deps, &ndeps) != cudaSuccess)
+        return RNN_ECUDA;
+      // the params union has no default constructor: zeroed storage instead
+      alignas(cudaGraphNodeParams) unsigned char cp_raw[sizeof(cudaGraphNodeParams)] = {};
+      cudaGraphNodeParams& cp = *reinterpret_cast<cudaGraphNodeParams*>(cp_raw);
+      cp.type = cudaGraphNodeTypeConditional;
+      cp.conditional.handle = hnd[it];
+      cp.conditional.type = cudaGraphCondTypeIf;
+      cp.conditional.size = 1;
+      cudaGraphNode_t node;
+      if (cudaGraphAddNode(&node, cg, deps, ndeps, &cp) != cudaSuccess) return RNN_ECUDA;
+      if (cudaStreamUpdateCaptureDependencies(s, &node, 1, cudaStreamSetCaptureDependencies) !=
+          cudaSuccess)
+        return RNN_ECUDA;
+      if (cudaStreamBeginCaptureToGraph(body_stream, cp.conditional.phGraph_out[0], nullptr,
+                                        nullptr, 0, cudaStreamCaptureModeThreadLocal) !=
+          cudaSuccess)
+        return RNN_ECUDA;
+      r = iteration(it, body_stream, it < max_iter ? hnd[it + 1] : 0);
+      cudaGraph_t body;
+      const cudaError_t ce = cudaStreamEndCapture(body_stream, &body);
+      if (r != RNN_OK) return r;
+      if (ce != cudaSuccess) return RNN_ECUDA;
+    }
   }
   frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, W1, pairs, cap, count_out, seed_state);
   return launched();
@@ -1352,7 +1433,7 @@ const char* rnn_status_string(rnn_status s) {
   return "unknown rnn_status";
 }
 
-int rnn_abi_version(void) { return 6; }
+int rnn_abi_version(void) { return 7; }
 
 uint64_t rnn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -1693,6 +1774,76 @@ rnn_status rnn_frm_match_ex(int B, const void* D1, int64_t d1_batch_stride, cons
                  init_xy1, n_init, seed_stride, max_iter, pixel_tol, pairs_out, cap, count_out,
                  seed_state_out, basin_out, workspace, ws_bytes,
                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------ graph plans
+struct rnn_frm_graph {
+  cudaGraphExec_t exec;
+};
+
+rnn_status rnn_frm_graph_create(int B, const void* D1, int64_t d1_batch_stride, const void* D2,
+                                int64_t d2_batch_stride, int H1, int W1, int H2, int W2, int d,
+                                rnn_dtype dtype, rnn_metric metric, const int32_t* init_xy1,
+                                int64_t n_init, int seed_stride, int max_iter, float pixel_tol,
+                                int32_t* pairs_out, int64_t cap, int32_t* count_out,
+                                int32_t* seed_state_out, int32_t* basin_out, void* workspace,
+                                size_t ws_bytes, rnn_frm_graph_t* graph_out) {
+  if (!graph_out) return RNN_EINVAL;
+  *graph_out = nullptr;
+  if (max_iter > kMaxGraphIters) return RNN_EUNSUPPORTED;
+  DeviceInfo* di = nullptr;
+  rnn_status r = device_info(&di);  // device queries stay outside the capture
+  if (r != RNN_OK) return r;
+  cudaStream_t s = nullptr, body = nullptr;
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return RNN_ECUDA;
+  if (cudaStreamCreateWithFlags(&body, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaStreamDestroy(s);
+    return RNN_ECUDA;
+  }
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    r = RNN_ECUDA;
+  } else {
+    t_capturing = true;
+    r = frm_run(B, D1, d1_batch_stride, D2, d2_batch_stride, H1, W1, H2, W2, d, dtype, metric,
+                init_xy1, n_init, seed_stride, max_iter, pixel_tol, pairs_out, cap, count_out,
+                seed_state_out, basin_out, workspace, ws_bytes, s, nullptr, body);
+    t_capturing = false;
+    const cudaError_t ce = cudaStreamEndCapture(s, &graph);
+    if (r == RNN_OK && ce != cudaSuccess) r = RNN_ECUDA;
+  }
+  if (r == RNN_OK && cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) r = RNN_ECUDA;
+  if (graph) cudaGraphDestroy(graph);
+  cudaStreamDestroy(body);
+  cudaStreamDestroy(s);
+  cudaGetLastError();  // a failed capture leaves its error; the status says it
+  if (r != RNN_OK) {
+    if (exec) cudaGraphExecDestroy(exec);
+    return r;
+  }
+  rnn_frm_graph* gp = new (std::nothrow) rnn_frm_graph;
+  if (!gp) {
+    cudaGraphExecDestroy(exec);
+    return RNN_ECUDA;
+  }
+  gp->exec = exec;
+  *graph_out = gp;
+  return RNN_OK;
+}
+
+rnn_status rnn_frm_graph_launch(rnn_frm_graph_t graph, rnn_stream_t stream) {
+  if (!graph) return RNN_EINVAL;
+  NvtxRange nvtx_range("rnn_frm_graph_launch");
+  if (cudaGraphLaunch(graph->exec, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RNN_ECUDA;
+  return RNN_OK;
+}
+
+void rnn_frm_graph_destroy(rnn_frm_graph_t graph) {
+  if (!graph) return;
+  cudaGraphExecDestroy(graph->exec);
+  delete graph;
 }
 
 // ------------------------------------------------ mutual test of NN arrays

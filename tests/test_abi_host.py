@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rnn_abi_version() == 6
+    assert lib.rnn_abi_version() == 7
     for code, name in _lib.STATUS.items():
         assert lib.rnn_status_string(code).decode().startswith(name)
 
@@ -307,3 +307,16 @@ def test_stall_hook_is_a_host_switch(lib):
     # sets and clears process-global state only; nothing is launched
     lib.rnn_test_stall_loads(1, 1000)
     lib.rnn_test_stall_loads(0, 0)
+
+
+def test_frm_graph_host_checks(lib):
+    # checks made before any device query: no plan handle, too many iterations
+    import ctypes
+    h = ctypes.c_void_p()
+    args = [1, FAKE, 64 * 24, FAKE, 64 * 24, 8, 8, 8, 8, 24, 0, 0, None, 0, 4]
+    rest = [0.0, FAKE, 64, FAKE, None, None, FAKE, 1 << 20]
+    assert lib.rnn_frm_graph_create(*args, 10, *rest, None) == EINVAL
+    assert lib.rnn_frm_graph_create(*args, 65, *rest, ctypes.byref(h)) == EUNSUP
+    assert not h.value
+    assert lib.rnn_frm_graph_launch(None, None) == EINVAL
+    lib.rnn_frm_graph_destroy(None)
