@@ -12,7 +12,8 @@ rank matches its own pairs: weak scaling, no data-path collective), timed on
 the device with CUDA events between barriers, max over ranks.  Extra keys:
 ``e2e`` (host buffers, copies inside the timed region), ``roofline`` (the
 fused similarity+argmax kernel, timed live with CUDA events), ``mnn`` (the
-exhaustive reciprocal set at 512x384 with its own roofline), ``cpu_baseline``
+exhaustive reciprocal set at 512x384 with its own roofline), ``frm_graph_plan``
+(the same step replayed as a recorded graph plan), ``cpu_baseline``
 (the double-precision oracle on a bounded sample), ``clocks``,
 ``gpu_launches``.
 
@@ -32,8 +33,8 @@ import time
 # the fused kernel in the bench step, from one ncu capture of the step's
 # first FRM call (20 launches averaged).  It belongs to the kernel sources it
 # was taken on: with any other sources the bench reports traffic as null.
-TRAFFIC = {"sources_sha256": "7867991fa9ca6939f36167259b342c3c8a5f2bde1eb392aa1dc03f1295c9a1f6",
-           "frm_nn_bytes_per_launch": 37.26e6}
+TRAFFIC = {"sources_sha256": "251ab8d3799d24c6fb94f6eaf8e7678bb9181b33cc3223258175cc44bb5f989e",
+           "frm_nn_bytes_per_launch": 37.23e6}
 
 
 def _kernel_sources_sha256() -> str:
@@ -311,6 +312,38 @@ def run_native(args):
                 "peak_source": f"bf16 sustained, {peaks['source']} (fp16 runs at the bf16 rate)",
                 "active_queries_per_pair": queries_per_call / P}
 
+    # ------------------------------------ the same step as a recorded graph plan
+    # Iterations after the last active seed converged launch nothing there; the
+    # kernels are the same, so the roofline above stands for both.
+    graph_plan = None
+    if not args.skip_graph_plan:
+        gplan = rnn.FRMGraph(A, B, seed_stride=w.seed_stride, max_iter=w.max_iter,
+                             with_seed_state=True)
+        for _ in range(args.warmup):
+            gplan.launch()
+        torch.cuda.synchronize()
+        barrier()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(args.steps):
+            gplan.launch()
+        g1.record()
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+        barrier()
+        same = bool(torch.equal(gplan.result.count, plan.result.count) and
+                    torch.equal(gplan.result.seed_state, plan.result.seed_state))
+        # iteration it + 1 runs when some seed makes query 2 it + 1; an iteration is
+        # 4 launches (two fused NN launches, two steps)
+        max_q = int(seed_state[:, :, 2].max())
+        iters_run = 1 + min(w.max_iter - 1, max(0, (max_q - 1) // 2))
+        graph_plan = {"value": replicas.aggregate_rate(P, world, graph_ms), "unit": "pairs/s",
+                      "ms_per_step": graph_ms, "iterations_run": iters_run,
+                      "gpu_launches": int(launches) - 4 * (w.max_iter - iters_run) * args.steps,
+                      "results_identical": same}
+        gplan.close()
+
     # ------------------------------------------------------ end to end (host)
     # Every step copies its pairs from pinned host memory and reads its pairs
     # and counts back.  Two input buffers and a copy stream let the copy of
@@ -478,7 +511,8 @@ def run_native(args):
                        "global_batch": world * P, "parallelism": f"replicas x{world}",
                        "l2": f"step inputs {2 * A_h.numel() * 2 / 1e6:.0f} MB > 126 MB L2"},
             "e2e": e2e, "roofline": roofline, "mnn": mnn, "frm_options": options,
-            "points": pts, "coarse_to_fine": c2f, "frm_configs": configs, "cpu_baseline": cpu,
+            "frm_graph_plan": graph_plan, "points": pts, "coarse_to_fine": c2f,
+            "frm_configs": configs, "cpu_baseline": cpu,
             "clocks": clocks, "gpu_launches": int(launches),
         }
         print(json.dumps(line), flush=True)
@@ -633,6 +667,8 @@ def main(argv=None):
     ap.add_argument("--skip-mnn", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--skip-graph-plan", action="store_true",
+                    help="do not time the step as a recorded graph plan")
     ap.add_argument("--leg", choices=["points", "c2f", "frm_batched_64x512x288", "frm_1024x768"],
                     help="run one secondary leg alone (for profiling) and exit")
     ap.add_argument("--nn-case", type=int, nargs=3, metavar=("NQ", "D", "NX"),
