@@ -321,54 +321,68 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
       build_prefix(p.fam[f], T->mt_prefix[f], scan_scratch);
     }
   }
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
+    // every lane derives the same sizes; the split counts are then tried
+    // one per lane and the lanes agree on the best with a min-reduction
+    // (a serial search in one thread costs microseconds of 64-bit division
+    // on every launch)
+    int fam_tiles[2], ntiles[2], caps[2];
     int tiles_total = 0;
     for (int f = 0; f < 2; ++f) {
-      if (f < p.nfam) {
-        T->fam_tiles[f] = T->mt_prefix[f][p.fam[f].nbatch];
-        T->ntiles[f] = (p.fam[f].n_cand + p.block_n - 1) / p.block_n;
-      } else {
-        T->fam_tiles[f] = 0;
-        T->ntiles[f] = 1;
-      }
-      tiles_total += T->fam_tiles[f];
+      fam_tiles[f] = f < p.nfam ? T->mt_prefix[f][p.fam[f].nbatch] : 0;
+      ntiles[f] = f < p.nfam ? (p.fam[f].n_cand + p.block_n - 1) / p.block_n : 1;
+      caps[f] = max(1, ntiles[f] / max(1, p.min_tiles));
+      tiles_total += fam_tiles[f];
     }
-    // split count: at least enough units for the target, and among the
-    // counts up to 2x that (units of at least min_tiles tiles) the one whose
-    // round-robin deal gives the CTAs the smallest largest share
+    // split count: enough units for the target, and among the counts from
+    // there up to 2x that (units of at least min_tiles tiles) the one whose
+    // round-robin deal gives the CTAs the smallest largest share, the
+    // smallest such count on a tie.  When the target needs more splits than
+    // min_tiles allows (a few query tiles, as in the late FRM half-steps),
+    // the counts from half that cap up to it.
     int S0 = tiles_total > 0 ? (p.target_units + tiles_total - 1) / tiles_total : 1;
     if (S0 < 1) S0 = 1;
-    int Smax = 1;
+    int cap = 1;
     for (int f = 0; f < 2; ++f)
-      if (f < p.nfam) Smax = max(Smax, T->ntiles[f] / max(1, p.min_tiles));
-    Smax = max(S0, min(2 * S0, Smax));
-    int S = S0;
-    long long best = -1;
-    for (int c = S0; c <= Smax; ++c) {
-      long long units = 0;
+      if (f < p.nfam) cap = max(cap, caps[f]);
+    const int Smax = max(1, min(2 * S0, cap));
+    const int Smin = max(1, min(S0, Smax / 2));
+    const unsigned grid = gridDim.x;
+    unsigned long long best = ~0ull;  // (share << 24) | count
+    for (int c = Smin + lane; c <= Smax; c += 32) {
+      unsigned units = 0;
       int biggest = 1;  // tiles of the largest unit
       for (int f = 0; f < 2; ++f) {
-        if (T->fam_tiles[f] == 0) continue;
-        const int Sf = max(1, min(c, T->ntiles[f] / max(1, p.min_tiles)));
-        units += static_cast<long long>(T->fam_tiles[f]) * Sf;
-        biggest = max(biggest, (T->ntiles[f] + Sf - 1) / Sf);
+        if (fam_tiles[f] == 0) continue;
+        const int Sf = min(c, caps[f]);
+        units += static_cast<unsigned>(fam_tiles[f]) * static_cast<unsigned>(Sf);
+        biggest = max(biggest, (ntiles[f] + Sf - 1) / Sf);
       }
       // each unit also costs about kUnitTiles tiles (query tile, pipeline
       // fill, final merge)
-      const long long share = (units + gridDim.x - 1) / gridDim.x * (biggest + kUnitTiles);
-      if (best < 0 || share < best) {
-        best = share;
-        S = c;
+      const unsigned long long share =
+          static_cast<unsigned long long>((units + grid - 1) / grid) * (biggest + kUnitTiles);
+      const unsigned long long key = (share << 24) | static_cast<unsigned>(c);
+      best = key < best ? key : best;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+      best = y < best ? y : best;
+    }
+    if (lane == 0) {
+      const int S = best == ~0ull ? Smin : static_cast<int>(best & 0xFFFFFFull);
+      int total = 0;
+      for (int f = 0; f < 2; ++f) {
+        const int Sf = min(S, caps[f]);
+        T->fam_tiles[f] = fam_tiles[f];
+        T->ntiles[f] = ntiles[f];
+        T->split[f] = Sf;
+        T->fam_units[f] = fam_tiles[f] * Sf;
+        total += T->fam_units[f];
       }
+      T->total_units = total;
     }
-    int total = 0;
-    for (int f = 0; f < 2; ++f) {
-      const int Sf = max(1, min(S, T->ntiles[f] / max(1, p.min_tiles)));
-      T->split[f] = Sf;
-      T->fam_units[f] = T->fam_tiles[f] * Sf;
-      total += T->fam_units[f];
-    }
-    T->total_units = total;
   }
   __syncthreads();
   const int total_units = T->total_units;
