@@ -569,6 +569,34 @@ def _points_leg(dev, lib, w, P, reps, warmup=3):
     return out
 
 
+def _graph_of(fn):
+    """fn() recorded into a torch CUDA graph (one eager call on a side stream
+    first); FRM calls inside it record their later iterations as conditional
+    nodes.  Returns the graph and the outputs its replays rewrite."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        out = fn()
+    torch.cuda.synchronize()
+    return g, out
+
+
+def _graph_timing(fn, ref_count, reps, flush):
+    """Median time of replays of fn() recorded as a graph, and whether a
+    replay's counts equal `ref_count` (a copy of the eager call's)."""
+    import torch
+    g, out = _graph_of(fn)
+    ms, _ = _timed_calls(lambda: (g.replay(), out)[1], reps, flush)
+    same = bool(torch.equal(out.count, ref_count))
+    del g
+    return ms, same
+
+
 def _c2f_leg(dev, lib, reps, warmup=3):
     """Coarse-to-fine: 1024x768 maps (d = 32), coarse M on 80x64 cells (d = 256)."""
     import torch
@@ -591,9 +619,13 @@ def _c2f_leg(dev, lib, reps, warmup=3):
     for _ in range(warmup):
         fn()
     ms, r = _timed_calls(fn, reps, flush)
+    gms, same = _graph_timing(fn, r.count.clone(), reps, flush)
     return {"metric": "coarse-to-fine image pairs/s: 1024x768 maps, d=32, coarse M on 80x64 "
                       "cells (d=256), 2x2 crops of 512x384, FRM stride 8, max_iter 15",
             "value": 1e3 / ms, "unit": "pairs/s", "ms_per_call": ms,
+            "graph": {"value": 1e3 / gms, "ms_per_call": gms, "counts_identical": same,
+                      "note": "the call recorded into a CUDA graph and replayed: FRM "
+                              "iterations after convergence launch nothing"},
             "outputs": int(r.count.item()), "crops_on": int(r.crops[:, 5].sum().item()),
             "dtype": "f16",
             "note": "includes the binding's output allocation; 256 MB L2 flush before every call"}
@@ -616,11 +648,16 @@ def _frm_config_leg(dev, name, reps, warmup=3):
     ms, r = _timed_calls(lambda: plan.run(A, B), reps, flush)
     queries = int(r.seed_state[:, :, 2].sum().item())
     flops = 2.0 * w.d * w.H * w.W * queries
+    gms, same = _graph_timing(lambda: plan.run(A, B), r.count.clone(), reps, flush)
     return {"metric": f"FRM image pairs/s, {w.pairs} pair(s) of {w.W}x{w.H}, d={w.d}, stride "
                       f"{w.seed_stride}, max_iter {w.max_iter}",
             "value": w.pairs / (ms * 1e-3), "unit": "pairs/s", "ms_per_call": ms,
             "outputs": int(r.count.sum().item()), "active_queries_per_pair": queries / w.pairs,
             "tensor_tflops_per_call": flops / (ms * 1e-3) / 1e12, "dtype": "f16",
+            "graph": {"value": w.pairs / (gms * 1e-3), "ms_per_call": gms,
+                      "counts_identical": same,
+                      "note": "the call recorded into a CUDA graph and replayed: iterations "
+                              "after convergence launch nothing"},
             "note": "whole-call time (256 MB L2 flush before every call); the tensor rate counts "
                     "the live queries' flops over the call, not one kernel"}
 

@@ -259,6 +259,13 @@ rnn_status rnn_frm_match_ex(int B, const void *D1, int64_t d1_batch_stride, cons
  *   word of the workspace (rnn_workspace_status) reports a launch's errors.
  *   *graph_out is owned by the caller: release it with rnn_frm_graph_destroy
  *   (NULL is accepted).
+ * An FRM call (rnn_frm_match*, rnn_c2f_match) that the caller itself records
+ * into a CUDA graph (stream capture) records its iterations 2..max_iter in
+ * conditional nodes of that graph the same way, when max_iter <= 64 and the
+ * calling thread has made an FRM call outside a capture before: that call
+ * creates the per-thread stream the iteration bodies are recorded on, since
+ * no stream is created inside a capture.  Otherwise every iteration is
+ * recorded.  Either way a replay gives the call's results.
  */
 typedef struct rnn_frm_graph *rnn_frm_graph_t;
 rnn_status rnn_frm_graph_create(int B, const void *D1, int64_t d1_batch_stride, const void *D2,
@@ -427,8 +434,10 @@ rnn_status rnn_nn_argmax_noalloc(const void *Q, int64_t nq, const void *X, int64
  * Diagnostics for benchmarking (no effect on results).
  *
  * rnn_launch_count: number of kernels this library has launched in this
- *   process (all entry points, all devices), not counting those that graph
- *   plans record or replay; recording a plan does not use the timer below.
+ *   process (all entry points, all devices).  Kernels that an FRM call records
+ *   into a graph (a graph plan, or a caller's capture) are not counted, nor
+ *   are replays, and such recordings do not use the timer below; the other
+ *   entry points' kernels recorded in a caller's capture count when recorded.
  * rnn_set_kernel_timer: while set, every launch of the fused
  *   similarity+argmax kernel is bracketed by cudaEventRecord(start_events[i])
  *   and cudaEventRecord(stop_events[i]) on the launch stream, with

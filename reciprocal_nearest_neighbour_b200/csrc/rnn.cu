@@ -196,6 +196,13 @@ static int* g_timer_count = nullptr;
 // Recording a graph plan: launches are neither counted nor timed.
 static thread_local bool t_capturing = false;
 
+// Per device, a stream of this thread that records the bodies of FRM's
+// conditional iteration nodes when an FRM call is captured into a graph by
+// its caller.  It is made by a call that is not being captured, so that no
+// stream is created inside a capture; until then a captured FRM call records
+// every iteration unconditionally (the same results).
+static thread_local cudaStream_t t_body[64] = {};
+
 // Check the last launch and count it.
 static rnn_status launched() {
   if (cudaGetLastError() != cudaSuccess) return RNN_ECUDA;
@@ -1085,7 +1092,9 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
                           cudaStream_t body_stream = nullptr) {
   // body_stream non-null: `s` is capturing a graph plan; iterations 2..max_iter
   // go into conditional (if) nodes, each enabled by the previous iteration's
-  // last step kernel when a seed is still active, and captured on body_stream
+  // last step kernel when a seed is still active, and captured on body_stream.
+  // A call that the caller captures into a graph does the same on this
+  // thread's body stream, when it has one.
   NvtxRange nvtx_range("rnn_frm_match");
   if (B < 1) return RNN_EINVAL;
   if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
@@ -1113,6 +1122,34 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   DeviceInfo* di = nullptr;
   rnn_status r = device_info(&di);
   if (r != RNN_OK) return r;
+  bool caller_capture = false;
+  if (!body_stream) {
+    int dev = 0;
+    cudaStreamCaptureStatus cst = cudaStreamCaptureStatusNone;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RNN_ECUDA;
+    if (cudaStreamIsCapturing(s, &cst) != cudaSuccess) {
+      cudaGetLastError();
+      cst = cudaStreamCaptureStatusNone;
+    }
+    if (cst == cudaStreamCaptureStatusActive) {
+      body_stream = max_iter <= kMaxGraphIters ? t_body[dev] : nullptr;
+      caller_capture = true;
+    } else if (!t_body[dev] &&
+               cudaStreamCreateWithFlags(&t_body[dev], cudaStreamNonBlocking) != cudaSuccess) {
+      t_body[dev] = nullptr;  // no body stream: captures record every iteration
+      cudaGetLastError();
+    }
+  }
+  // recorded into the caller's graph: the launches are neither counted nor timed
+  struct CaptureFlag {
+    bool on, prev;
+    explicit CaptureFlag(bool o) : on(o), prev(t_capturing) {
+      if (on) t_capturing = true;
+    }
+    ~CaptureFlag() {
+      if (on) t_capturing = prev;
+    }
+  } capture_flag(caller_capture);
 
   FrmState st;
   FrmCopies cp;

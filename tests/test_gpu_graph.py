@@ -1,7 +1,9 @@
 """FRM graph plans on the GPU (needs a B200): the recorded match, with its
 conditional iterations, gives the oracle's result and the stream call's,
 bit for bit (pairs, counts, seed state, basin), and a relaunch reads the
-maps' new contents.  Quantised inputs (values k/64) make every score exact.
+maps' new contents.  The same holds for FRM and coarse-to-fine calls that the
+caller records into its own CUDA graph.  Quantised inputs (values k/64) make
+every score exact.
 """
 import numpy as np
 import pytest
@@ -112,3 +114,89 @@ def test_graph_full_size_matches_stream():
     for _ in range(3):
         _same(g.launch(), s)
     assert int(s.count[0]) > 1000
+
+
+# ------------------------------------------- FRM inside a caller's CUDA graph
+
+def _capture(fn):
+    """Record fn() into a torch CUDA graph (after one eager call on the side
+    stream, as torch recommends); returns the graph and fn's outputs."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        out = fn()
+    return g, out
+
+
+@pytest.mark.parametrize("metric", ["dot", "l2"])
+def test_caller_graph_capture_of_frm(metric):
+    """An FRM call captured by the caller records its later iterations as
+    conditional nodes; replays give the oracle's result on whatever the
+    input tensors hold."""
+    D1, D2 = _maps(240, 40, 56, 36, 60)
+    E1, E2 = _maps(241, 40, 56, 36, 60)
+    t1, t2 = dev(D1), dev(D2)
+    g, r = _capture(lambda: rnn.frm_match_ex(t1, t2, seed_stride=3, max_iter=10, metric=metric,
+                                             with_seed_state=True))
+    for A, B in [(D1, D2), (E1, E2), (D1, D2)]:
+        t1.copy_(dev(A))
+        t2.copy_(dev(B))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = oracle.frm_ex(A, B, 3, 10, metric=metric)
+        assert np.array_equal(r.trimmed().cpu().numpy(), ref.pairs)
+        u, v, q, c = seed_state_np(r)
+        assert np.array_equal(q, ref.seed_queries) and np.array_equal(c, ref.seed_converged)
+
+
+def test_caller_graph_capture_of_c2f():
+    A, B = synth.smooth_pair(250, 192, 256, 24)
+    F1, F2 = dev(synth.to_storage(A, "f16")), dev(synth.to_storage(B, "f16"))
+    C1 = dev(synth.to_storage(synth.coarse_map(A, 24, 32, dc=64, seed=3), "f16"))
+    C2 = dev(synth.to_storage(synth.coarse_map(B, 24, 32, dc=64, seed=3), "f16"))
+    kw = dict(crop=(96, 128), seed_stride=4, max_iter=12)
+    eager = rnn.c2f_match(C1, C2, F1, F2, **kw)
+    g, r = _capture(lambda: rnn.c2f_match(C1, C2, F1, F2, **kw))
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(r.count, eager.count) and torch.equal(r.crops, eager.crops)
+        n = int(eager.count[0])
+        assert torch.equal(r.pairs[:n], eager.pairs[:n])
+    assert int(eager.count[0]) > 100
+
+
+def test_capture_in_a_fresh_thread_records_every_iteration():
+    """A thread whose first FRM call is captured has no stream for the
+    conditional bodies yet: every iteration is recorded, same results."""
+    import threading
+    D1, D2 = _maps(260, 32, 48, 32, 48)
+    out = {}
+
+    def body():
+        try:
+            t1, t2 = dev(D1), dev(D2)
+            g = torch.cuda.CUDAGraph()
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    r = rnn.frm_match_ex(t1, t2, seed_stride=2, max_iter=8,
+                                         with_seed_state=True)
+            g.replay()
+            torch.cuda.synchronize()
+            out["r"] = (r.trimmed().cpu().numpy(), seed_state_np(r))
+        except Exception as e:  # reported below, in the test's thread
+            out["e"] = e
+
+    th = threading.Thread(target=body)
+    th.start()
+    th.join()
+    assert "e" not in out, out.get("e")
+    ref = oracle.frm_ex(D1, D2, 2, 8)
+    pairs, (u, v, q, c) = out["r"]
+    assert np.array_equal(pairs, ref.pairs)
+    assert np.array_equal(q, ref.seed_queries)
