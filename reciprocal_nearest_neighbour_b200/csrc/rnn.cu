@@ -322,52 +322,77 @@ __device__ __forceinline__ uint16_t f_to_bits(float x, bool bf16) {
 }
 
 // One thread per 16-byte chunk of the output, so that reads and writes are
-// coalesced.  d is a multiple of 8, so a chunk lies wholly among the channels
-// or wholly past them; the first chunk past them holds the augmentation (its
-// thread reads the whole row for |x|^2), the rest are zero.
+// coalesced; map b of the batch is grid row blockIdx.y.  d is a multiple of
+// 8, so a chunk lies wholly among the channels or wholly past them; the first
+// chunk past them holds the augmentation (its thread reads the whole row for
+// |x|^2), the rest are zero.  kCpr: chunks per output row when known at
+// compile time (the index split is then a multiply and shift), else 0.
 template <bool kBf16>
-__global__ void prep_rows_kernel(const uint16_t* src, int64_t bstride, int64_t rows, int nbatch,
-                                 int d, uint16_t* dst, int kpad, int form) {
-  const int cpr = kpad / 8, creal = d / 8;  // chunks per output row / per input row
-  const int64_t total = static_cast<int64_t>(nbatch) * rows * cpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += stride) {
-    const int64_t rr = i / cpr;  // row over all batches
-    const int c = static_cast<int>(i - rr * cpr);
-    const int64_t b = rr / rows, r = rr - b * rows;
-    const uint4* in = reinterpret_cast<const uint4*>(src + b * bstride + r * d);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (c < creal) {
-      v = __ldg(in + c);
-    } else if (c == creal && form != kFormPad) {
-      uint16_t aug[kAugCols];
-      if (form == kFormQuery) {
-        aug[0] = aug[1] = aug[2] = f_to_bits(1.0f, kBf16);
-      } else {
-        float n2 = 0.f;
-        for (int cc = 0; cc < creal; ++cc) {
-          const uint4 x = __ldg(in + cc);
-          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+__device__ __forceinline__ uint4 prep_chunk(const uint4* __restrict__ in, int c, int creal,
+                                            int form) {
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (c < creal) {
+    v = __ldg(in + c);
+  } else if (c == creal && form != kFormPad) {
+    uint16_t aug[kAugCols];
+    if (form == kFormQuery) {
+      aug[0] = aug[1] = aug[2] = f_to_bits(1.0f, kBf16);
+    } else {
+      float n2 = 0.f;
+      for (int cc = 0; cc < creal; ++cc) {
+        const uint4 x = __ldg(in + cc);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float lo = bits_to_f(static_cast<uint16_t>(w[e] & 0xFFFFu), kBf16);
-            const float hi = bits_to_f(static_cast<uint16_t>(w[e] >> 16), kBf16);
-            n2 = fmaf(lo, lo, n2);
-            n2 = fmaf(hi, hi, n2);
-          }
-        }
-        float rest = -0.5f * n2;
-#pragma unroll
-        for (int e = 0; e < kAugCols; ++e) {
-          aug[e] = f_to_bits(rest, kBf16);
-          rest -= bits_to_f(aug[e], kBf16);
+        for (int e = 0; e < 4; ++e) {
+          const float lo = bits_to_f(static_cast<uint16_t>(w[e] & 0xFFFFu), kBf16);
+          const float hi = bits_to_f(static_cast<uint16_t>(w[e] >> 16), kBf16);
+          n2 = fmaf(lo, lo, n2);
+          n2 = fmaf(hi, hi, n2);
         }
       }
-      v.x = static_cast<uint32_t>(aug[0]) | (static_cast<uint32_t>(aug[1]) << 16);
-      v.y = static_cast<uint32_t>(aug[2]);
+      float rest = -0.5f * n2;
+#pragma unroll
+      for (int e = 0; e < kAugCols; ++e) {
+        aug[e] = f_to_bits(rest, kBf16);
+        rest -= bits_to_f(aug[e], kBf16);
+      }
     }
-    reinterpret_cast<uint4*>(dst)[i] = v;
+    v.x = static_cast<uint32_t>(aug[0]) | (static_cast<uint32_t>(aug[1]) << 16);
+    v.y = static_cast<uint32_t>(aug[2]);
+  }
+  return v;
+}
+
+// One thread per 16-byte chunk of the output, so that reads and writes are
+// coalesced; map b of the batch is grid row blockIdx.y.  d is a multiple of
+// 8, so a chunk lies wholly among the channels or wholly past them; the first
+// chunk past them holds the augmentation (its thread reads the whole row for
+// |x|^2), the rest are zero.  kCpr: chunks per output row when known at
+// compile time (the index split is then a multiply and shift), else 0.  Each
+// thread handles two chunks a grid stride apart per step, both loads ahead of
+// both stores, for twice the reads in flight.
+template <bool kBf16, int kCpr>
+__global__ void prep_rows_kernel(const uint16_t* __restrict__ src, int64_t bstride,
+                                 int64_t rows, int d, uint16_t* __restrict__ dst, int kpad,
+                                 int form) {
+  const int cpr = kCpr ? kCpr : kpad / 8, creal = d / 8;  // chunks per output / input row
+  const int64_t b = blockIdx.y;
+  const int64_t total = rows * cpr;  // chunks of map b
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const uint16_t* __restrict__ sb = src + b * bstride;
+  uint4* __restrict__ db = reinterpret_cast<uint4*>(dst) + b * total;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += 2 * stride) {
+    const int64_t i2 = i + stride;
+    const int64_t r = i / cpr, r2 = i2 / cpr;
+    const uint4 v = prep_chunk<kBf16>(reinterpret_cast<const uint4*>(sb + r * d),
+                                      static_cast<int>(i - r * cpr), creal, form);
+    uint4 v2 = make_uint4(0, 0, 0, 0);
+    if (i2 < total)
+      v2 = prep_chunk<kBf16>(reinterpret_cast<const uint4*>(sb + r2 * d),
+                             static_cast<int>(i2 - r2 * cpr), creal, form);
+    db[i] = v;
+    if (i2 < total) db[i2] = v2;
   }
 }
 
@@ -1047,14 +1072,27 @@ static int64_t num_seeds(int H, int W, int S) {
 static rnn_status prep_rows(const void* src, int64_t bstride, int64_t rows, int nbatch, int d,
                             uint16_t* dst, int kpad, int form, rnn_dtype dt, DeviceInfo* di,
                             cudaStream_t s) {
-  const int grid = grid_for(static_cast<int64_t>(nbatch) * rows * (kpad / 8), di->sms);
+  // the same number of threads as one 1-D grid over all maps, split evenly
+  const int64_t per = rows * (kpad / 8);
+  const int g1 = grid_for(per * nbatch, di->sms);
+  const dim3 grid(static_cast<unsigned>(std::max<int64_t>(
+                      1, std::min<int64_t>((g1 + nbatch - 1) / nbatch,
+                                           (per + kSmallThreads - 1) / kSmallThreads))),
+                  static_cast<unsigned>(nbatch));
   const uint16_t* in = static_cast<const uint16_t*>(src);
-  if (dt == RNN_BF16)
-    prep_rows_kernel<true><<<grid, kSmallThreads, 0, s>>>(in, bstride, rows, nbatch, d, dst,
-                                                         kpad, form);
-  else
-    prep_rows_kernel<false><<<grid, kSmallThreads, 0, s>>>(in, bstride, rows, nbatch, d, dst,
-                                                          kpad, form);
+  auto go = [&](auto kernel) {
+    kernel<<<grid, kSmallThreads, 0, s>>>(in, bstride, rows, d, dst, kpad, form);
+  };
+  const int cpr = kpad / 8;
+  if (dt == RNN_BF16) {
+    if (cpr == 4) go(prep_rows_kernel<true, 4>);
+    else if (cpr == 8) go(prep_rows_kernel<true, 8>);
+    else go(prep_rows_kernel<true, 0>);
+  } else {
+    if (cpr == 4) go(prep_rows_kernel<false, 4>);
+    else if (cpr == 8) go(prep_rows_kernel<false, 8>);
+    else go(prep_rows_kernel<false, 0>);
+  }
   return launched();
 }
 
