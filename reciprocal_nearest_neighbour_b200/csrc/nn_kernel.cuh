@@ -251,8 +251,11 @@ __device__ __forceinline__ float max32(const float (&v)[32]) {
 // kEpiWarps: epilogue warps (8 or 16); kChunks: 32-column chunks of each
 // tile read by one of them; kBatch: chunks per copy from tensor memory to
 // registers; kOneGroup: all epilogue warps take every tile (each a column
-// part of it) instead of one group per accumulator.
-template <int kEpiWarps, int kChunks, int kBatch, bool kOneGroup = false>
+// part of it) instead of one group per accumulator; kPdl: launched as a
+// programmatic dependent of the previous kernel (the FRM chain), so it waits
+// for that kernel before reading the query counts.  The wait is compiled only
+// into that form: a kernel that holds it costs more to launch plainly.
+template <int kEpiWarps, int kChunks, int kBatch, bool kOneGroup = false, bool kPdl = false>
 __global__ void __launch_bounds__((kEpiWarp0 + kEpiWarps) * 32, 1)
 nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUtensorMap tmap0,
                  const __grid_constant__ CUtensorMap tmap1,
@@ -315,6 +318,8 @@ nn_argmax_kernel(const __grid_constant__ NNParams p, const __grid_constant__ CUt
     if (p.fam[0].q_tma) tma_prefetch_desc(&qmap0);
     if (p.nfam > 1 && p.fam[1].q_tma) tma_prefetch_desc(&qmap1);
   }
+  // everything below reads the previous kernel's output (query counts, lists)
+  if constexpr (kPdl) pdl_wait();
   // unit table
   for (int f = 0; f < 2; ++f) {
     if (f < p.nfam) {

@@ -243,6 +243,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
       : "memory");
 }
 
+// Programmatic dependent launch.  pdl_wait: block until the grid this one
+// depends on has completed and its writes are visible (returns at once when
+// the launch had no programmatic dependency); every read of the previous
+// kernel's output comes after it.  pdl_trigger: let the next grid in the
+// stream be launched now (it still waits for this grid in its pdl_wait).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Three-input maximum (sm_100 and later).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

@@ -30,6 +30,9 @@ constexpr int kSmallThreads = 1024;
 constexpr int kMnnChunk = 4096;  // rows per block in the mutual test (4 per thread)
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per bounded wait
 constexpr int kMaxGraphIters = 64;  // max_iter of a graph plan
+#ifndef RNN_PDL
+#define RNN_PDL 1  // programmatic dependent launch along the FRM chain
+#endif
 
 static size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -210,9 +213,33 @@ static rnn_status launched() {
   return RNN_OK;
 }
 
+// Launch with, when `pdl` is set, programmatic stream serialization: the
+// grid may be launched while the previous kernel of the stream finishes, and
+// waits for it in pdl_wait before reading its output.
+template <typename... KArgs, typename... Args>
+static void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, bool pdl, Args&&... args) {
+  if (!pdl) {  // the plain launch costs the host less
+    kernel<<<grid, block, smem, s>>>(std::forward<Args>(args)...);
+    return;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const CUtensorMap& m1,
                             const CUtensorMap& q0, const CUtensorMap& q1, const Geometry& g,
-                            DeviceInfo* di, cudaStream_t s) {
+                            DeviceInfo* di, cudaStream_t s, bool pdl = false) {
   NNParams p = p_in;
   p.kb = g.kb;
   p.nkb = g.nkb;
@@ -236,7 +263,11 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
       const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
       if (cudaFuncSetAttribute(nn_argmax_kernel<16, 4, 2>, attr, sm) != cudaSuccess ||
           cudaFuncSetAttribute(nn_argmax_kernel<8, 4, 4>, attr, sm) != cudaSuccess ||
-          cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2, true>, attr, sm) != cudaSuccess)
+          cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2, true>, attr, sm) != cudaSuccess ||
+          cudaFuncSetAttribute(nn_argmax_kernel<16, 4, 2, false, true>, attr, sm) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(nn_argmax_kernel<8, 4, 4, false, true>, attr, sm) != cudaSuccess ||
+          cudaFuncSetAttribute(nn_argmax_kernel<16, 2, 2, true, true>, attr, sm) != cudaSuccess)
         return RNN_ECUDA;
       di->smem_set = true;
     }
@@ -257,13 +288,30 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
   // follows its release.  Two 128-column accumulators: eight warps, one group
   // per accumulator.  Four: sixteen warps copying 64, one group per
   // accumulator.
-  if (g.nacc == 2 && g.block_n == 256)
-    nn_argmax_kernel<16, 2, 2, true><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0,
-                                                                                    q1);
-  else if (g.nacc == 2)
-    nn_argmax_kernel<8, 4, 4><<<di->sms, (kEpiWarp0 + 8) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
-  else
-    nn_argmax_kernel<16, 4, 2><<<di->sms, (kEpiWarp0 + 16) * 32, g.smem, s>>>(p, m0, m1, q0, q1);
+  const dim3 grid(di->sms);
+  if (g.nacc == 2 && g.block_n == 256) {
+    const dim3 block((kEpiWarp0 + 16) * 32);
+    if (pdl)
+      launch_k(nn_argmax_kernel<16, 2, 2, true, true>, grid, block, g.smem, s, true, p, m0, m1,
+               q0, q1);
+    else
+      launch_k(nn_argmax_kernel<16, 2, 2, true>, grid, block, g.smem, s, false, p, m0, m1, q0,
+               q1);
+  } else if (g.nacc == 2) {
+    const dim3 block((kEpiWarp0 + 8) * 32);
+    if (pdl)
+      launch_k(nn_argmax_kernel<8, 4, 4, false, true>, grid, block, g.smem, s, true, p, m0, m1,
+               q0, q1);
+    else
+      launch_k(nn_argmax_kernel<8, 4, 4>, grid, block, g.smem, s, false, p, m0, m1, q0, q1);
+  } else {
+    const dim3 block((kEpiWarp0 + 16) * 32);
+    if (pdl)
+      launch_k(nn_argmax_kernel<16, 4, 2, false, true>, grid, block, g.smem, s, true, p, m0, m1,
+               q0, q1);
+    else
+      launch_k(nn_argmax_kernel<16, 4, 2>, grid, block, g.smem, s, false, p, m0, m1, q0, q1);
+  }
   const rnn_status r = launched();
   if (r == RNN_OK && slot >= 0 &&
       cudaEventRecord(static_cast<cudaEvent_t>(g_timer_stop[slot]), s) != cudaSuccess)
@@ -923,6 +971,8 @@ __device__ __forceinline__ void frm_apply(const FrmState& st, int b, int64_t bas
 template <bool kBf16>
 __global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter,
                                 cudaGraphConditionalHandle next) {
+  pdl_wait();
+  pdl_trigger();
   const int32_t* cnt_in = st.cnt[h % 3];
   int32_t* cnt_out = st.cnt[(h + 1) % 3];
   const int32_t* list_in = st.list[h % 2];
@@ -977,6 +1027,7 @@ __global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter,
 // so a bitmap over image 1 de-duplicates and sorts.
 __global__ void frm_merge_kernel(FrmState st, int W1, int32_t* pairs, int64_t cap,
                                  int32_t* count_out, int32_t* seed_state) {
+  pdl_wait();
   const int b = blockIdx.x;
   const int64_t base = static_cast<int64_t>(b) * st.k;
   const int ns = st.nseeds[b];
@@ -1053,11 +1104,13 @@ static int grid_for(int64_t n, int sms) {
 
 static rnn_status frm_step(const FrmState& st, int h, int nn2_half, int last_iter,
                            rnn_dtype dt, int grid, cudaStream_t s,
-                           cudaGraphConditionalHandle next = 0) {
+                           cudaGraphConditionalHandle next = 0, bool pdl = false) {
   if (dt == RNN_BF16)
-    frm_step_kernel<true><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter, next);
+    launch_k(frm_step_kernel<true>, dim3(grid), dim3(kSmallThreads), 0, s, pdl, st, h, nn2_half,
+             last_iter, next);
   else
-    frm_step_kernel<false><<<grid, kSmallThreads, 0, s>>>(st, h, nn2_half, last_iter, next);
+    launch_k(frm_step_kernel<false>, dim3(grid), dim3(kSmallThreads), 0, s, pdl, st, h, nn2_half,
+             last_iter, next);
   return launched();
 }
 
@@ -1134,6 +1187,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   // A call that the caller captures into a graph does the same on this
   // thread's body stream, when it has one.
   NvtxRange nvtx_range("rnn_frm_match");
+  const bool own_plan = body_stream != nullptr;
   if (B < 1) return RNN_EINVAL;
   if (B > RNN_MAX_BATCH) return RNN_EUNSUPPORTED;
   if (H1 <= 0 || W1 <= 0 || H2 <= 0 || W2 <= 0 || max_iter < 1) return RNN_EINVAL;
@@ -1188,6 +1242,10 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
       if (on) t_capturing = prev;
     }
   } capture_flag(caller_capture);
+  // programmatic dependent launches along the chain of FRM kernels, on a
+  // stream or recorded into a graph plan (a caller's capture records plain
+  // launches)
+  const bool pdl = RNN_PDL && (own_plan || !t_capturing);
 
   FrmState st;
   FrmCopies cp;
@@ -1260,8 +1318,8 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_bstride = st.s1;
     F.q_index = st.U;
     F.n_cand = static_cast<int32_t>(N2);
-    if ((e = launch_nn(p, map2, map2, map2, map2, g, di, q)) != RNN_OK) return e;
-    if ((e = frm_step(st, h, 1, 0, dt, lgrid, q)) != RNN_OK) return e;
+    if ((e = launch_nn(p, map2, map2, map2, map2, g, di, q, pdl)) != RNN_OK) return e;
+    if ((e = frm_step(st, h, 1, 0, dt, lgrid, q, 0, pdl)) != RNN_OK) return e;
     // half-step 2: U = NN1(V)
     F.q_list = st.list[(h + 1) % 2];
     F.q_count_dev = st.cnt[(h + 1) % 3];
@@ -1269,8 +1327,8 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
     F.q_bstride = st.s2;
     F.q_index = st.V;
     F.n_cand = static_cast<int32_t>(N1);
-    if ((e = launch_nn(p, map1, map1, map1, map1, g, di, q)) != RNN_OK) return e;
-    return frm_step(st, h + 1, 0, it == max_iter ? 1 : 0, dt, lgrid, q, next);
+    if ((e = launch_nn(p, map1, map1, map1, map1, g, di, q, pdl)) != RNN_OK) return e;
+    return frm_step(st, h + 1, 0, it == max_iter ? 1 : 0, dt, lgrid, q, next, pdl);
   };
   if (!body_stream) {
     for (int it = 1; it <= max_iter; ++it)
@@ -1316,7 +1374,8 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
       if (ce != cudaSuccess) return RNN_ECUDA;
     }
   }
-  frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, W1, pairs, cap, count_out, seed_state);
+  launch_k(frm_merge_kernel, dim3(B), dim3(kSmallThreads), 0, s, pdl, st, W1, pairs, cap,
+           count_out, seed_state);
   return launched();
 }
 
