@@ -985,10 +985,38 @@ __global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter,
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int n_cand = nn2_half ? st.N2 : st.N1;
   const int32_t* rows = nn2_half ? st.U : st.V;
-  for (int64_t x = w0; x < static_cast<int64_t>(st.B) * st.k; x += nw) {
-    const int b = static_cast<int>(x / st.k);
-    const int i = static_cast<int>(x - static_cast<int64_t>(b) * st.k);
-    if (i >= cnt_in[b]) continue;
+  // The active seeds of all pairs as one range: prefix of the counts over
+  // the pairs (one per thread; B <= blockDim.x), so that the warps visit only
+  // active seeds and a launch with none ends after the scan.  Above 2^31 slots
+  // in all, the warps visit every slot instead.
+  __shared__ int s_pref[kSmallThreads + 1];
+  const bool compact = static_cast<int64_t>(st.B) * st.k < INT32_MAX;
+  int64_t n_items = static_cast<int64_t>(st.B) * st.k;
+  if (compact) {
+    int total;
+    const int c = static_cast<int>(threadIdx.x) < st.B ? cnt_in[threadIdx.x] : 0;
+    const int ex = block_exclusive_scan(c, &total);
+    if (static_cast<int>(threadIdx.x) < st.B) s_pref[threadIdx.x] = ex;
+    if (threadIdx.x == 0) s_pref[st.B] = total;
+    __syncthreads();
+    n_items = total;
+  }
+  for (int64_t x = w0; x < n_items; x += nw) {
+    int b, i;
+    if (compact) {
+      // the last pair whose first active seed is at or before x
+      int lo = 0, hi = st.B;  // s_pref[lo] <= x < s_pref[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_pref[mid] <= x) lo = mid; else hi = mid;
+      }
+      b = lo;
+      i = static_cast<int>(x - s_pref[lo]);
+    } else {
+      b = static_cast<int>(x / st.k);
+      i = static_cast<int>(x - static_cast<int64_t>(b) * st.k);
+      if (i >= cnt_in[b]) continue;
+    }
     const int64_t base = static_cast<int64_t>(b) * st.k;
     const uint16_t* Dq = nn2_half ? st.Q1 + b * st.s1 : st.Q2 + b * st.s2;
     const uint16_t* Dx = nn2_half ? st.X2 + b * st.s2 : st.X1 + b * st.s1;
@@ -1293,7 +1321,8 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
   if ((r = make_map(&map2, st.X2, st.ld, N2, B, st.s2, g)) != RNN_OK) return r;
 
   if ((r = frm_seed(st, init, n_init, W1, S, di, s)) != RNN_OK) return r;
-  const int lgrid = grid_for(static_cast<int64_t>(B) * k * 32, di->sms);
+  // the step kernels: one resident wave (two blocks of 1024 a SM) at most
+  const int lgrid = std::min(grid_for(static_cast<int64_t>(B) * k * 32, di->sms), 2 * di->sms);
 
   NNParams p;
   std::memset(&p, 0, sizeof(p));
