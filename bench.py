@@ -33,8 +33,8 @@ import time
 # the fused kernel in the bench step, from one ncu capture of the step's
 # first FRM call (20 launches averaged).  It belongs to the kernel sources it
 # was taken on: with any other sources the bench reports traffic as null.
-TRAFFIC = {"sources_sha256": "f2095a701836ddbcf4733e0ee53f47136f5f6dd9f4f1d05427b2d3bb71d15ceb",
-           "frm_nn_bytes_per_launch": 37.28e6}
+TRAFFIC = {"sources_sha256": "484732799122cc22fd04085a024d82f3299be8264274d91f7661eef68193e127",
+           "frm_nn_bytes_per_launch": 37.29e6}
 
 
 def _kernel_sources_sha256() -> str:
