@@ -320,3 +320,17 @@ def test_frm_graph_host_checks(lib):
     assert not h.value
     assert lib.rnn_frm_graph_launch(None, None) == EINVAL
     lib.rnn_frm_graph_destroy(None)
+
+
+def test_frm_graph_binding_rejects_bad_maps(lib):
+    # the binding checks its arguments before the library is asked for a plan
+    import torch
+    import reciprocal_nearest_neighbour_b200 as rnn
+    cpu = torch.zeros((8, 8, 24), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        rnn.FRMGraph(cpu, cpu)
+    g = rnn.FRMGraph.__new__(rnn.FRMGraph)   # a plan whose creation never ran
+    g._handle = ctypes.c_void_p()
+    with pytest.raises(RuntimeError):
+        g.launch()
+    g.close()                                 # closing it is a no-op
