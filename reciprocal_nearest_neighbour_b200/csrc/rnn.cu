@@ -756,8 +756,13 @@ struct FrmState {
   float pixel_tol;  // > 0: converged when the move from U_old is below it
   int starts;       // 1: the seeds were given (output U_old with pixel_tol)
   const int32_t* pair_on;  // [B] or null: grid seeds only for the pairs marked 1
-  int B, k, N1, N2, nwords;
+  int32_t* mcounts; // [B][mblocks] output pixels per bitmap block (merge)
+  int B, k, N1, N2, nwords, mblocks;
 };
+
+// Merge: threads of its kernels, and bitmap words per block of its count and
+// emit kernels (one word per thread).
+constexpr int kMergeThreads = 256;
 
 // Row-form copies a call needs: none, one padded copy per map (dot metric,
 // d short of the K-block layout), or a query and a candidate form per map
@@ -798,6 +803,8 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int
   const int64_t nwords = (N1 + 31) / 32;
   st->bitmap = c.take<uint32_t>(B * nwords);
   st->partner = c.take<int32_t>(B * N1);
+  const int64_t mblocks = (nwords + kMergeThreads - 1) / kMergeThreads;
+  st->mcounts = c.take<int32_t>(B * mblocks);
   const int mode = d > 0 ? copies_for(d, metric) : kCopiesNone;  // d = 0: point maps
   cp->q1 = cp->x1 = cp->q2 = cp->x2 = nullptr;
   if (mode != kCopiesNone) {
@@ -816,6 +823,7 @@ static size_t frm_layout(void* ws, int B, int64_t k, int64_t N1, int64_t N2, int
   st->N1 = static_cast<int>(N1);
   st->N2 = static_cast<int>(N2);
   st->nwords = static_cast<int>(nwords);
+  st->mblocks = static_cast<int>(mblocks);
   st->basin = nullptr;
   st->pair_on = nullptr;
   return c.off;
@@ -1047,71 +1055,91 @@ __global__ void frm_step_kernel(FrmState st, int h, int nn2_half, int last_iter,
   }
 }
 
-// Unique output pairs of pair blockIdx.x, sorted by the image-1 pixel.  A
-// seed is in the output when it is no longer active, or, with a pixel
-// tolerance, when its last move (U_old -> U) is shorter than the tolerance;
-// the pair is (U, V), or (U_old, V) with a tolerance and given starts.  An
-// output pixel determines its partner (a mutual pair, or a start's match),
-// so a bitmap over image 1 de-duplicates and sorts.
-__global__ void frm_merge_kernel(FrmState st, int W1, int32_t* pairs, int64_t cap,
-                                 int32_t* count_out, int32_t* seed_state) {
+// Unique output pairs of every pair, sorted by the image-1 pixel, in three
+// kernels over many blocks (the pairs on grid.y).  A seed is in the output
+// when it is no longer active, or, with a pixel tolerance, when its last move
+// (U_old -> U) is shorter than the tolerance; the pair is (U, V), or
+// (U_old, V) with a tolerance and given starts.  An output pixel determines
+// its partner (a mutual pair, or a start's match), so a bitmap over image 1
+// de-duplicates and sorts.
+//
+// Mark: one thread per seed slot marks its output pixel in the bitmap,
+// writes the partner, and fills the seed state.
+__global__ void frm_mark_kernel(FrmState st, int W1, int32_t* seed_state) {
   pdl_wait();
-  const int b = blockIdx.x;
+  pdl_trigger();
+  const int b = blockIdx.y;
+  const int s = blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= st.k) return;
   const int64_t base = static_cast<int64_t>(b) * st.k;
   const int ns = st.nseeds[b];
-  uint32_t* bm = st.bitmap + static_cast<int64_t>(b) * st.nwords;
-  int32_t* partner = st.partner + static_cast<int64_t>(b) * st.N1;
-  for (int s = threadIdx.x; s < st.k; s += blockDim.x) {
-    int conv = 0;
-    int32_t u = -1, v = -1;
-    if (s < ns) {
-      u = st.U[base + s];
-      v = st.V[base + s];
-      int32_t uo = u;
-      if (st.pixel_tol > 0.f) {
-        const int32_t u0 = st.Uold[base + s];
-        // in double, as the distance is written down
-        const double dy = static_cast<double>(u0 / W1 - u / W1);
-        const double dx = static_cast<double>(u0 % W1 - u % W1);
-        conv = sqrt(dy * dy + dx * dx) < static_cast<double>(st.pixel_tol);
-        if (st.starts) uo = u0;
-      } else {
-        conv = st.act[base + s] == 0;
-      }
-      if (conv) {
-        atomicOr(bm + (uo >> 5), 1u << (uo & 31));
-        partner[uo] = v;
-      }
+  int conv = 0;
+  int32_t u = -1, v = -1;
+  if (s < ns) {
+    u = st.U[base + s];
+    v = st.V[base + s];
+    int32_t uo = u;
+    if (st.pixel_tol > 0.f) {
+      const int32_t u0 = st.Uold[base + s];
+      // in double, as the distance is written down
+      const double dy = static_cast<double>(u0 / W1 - u / W1);
+      const double dx = static_cast<double>(u0 % W1 - u % W1);
+      conv = sqrt(dy * dy + dx * dx) < static_cast<double>(st.pixel_tol);
+      if (st.starts) uo = u0;
+    } else {
+      conv = st.act[base + s] == 0;
     }
-    if (seed_state) {
-      int32_t* o = seed_state + (base + s) * 4;
-      o[0] = u;
-      o[1] = v;
-      o[2] = s < ns ? st.nq[base + s] : 0;
-      o[3] = conv;
+    if (conv) {
+      atomicOr(st.bitmap + static_cast<int64_t>(b) * st.nwords + (uo >> 5), 1u << (uo & 31));
+      st.partner[static_cast<int64_t>(b) * st.N1 + uo] = v;
     }
   }
-  __syncthreads();
-  const int per = (st.nwords + blockDim.x - 1) / blockDim.x;
-  const int w0 = threadIdx.x * per;
-  const int w1 = min(st.nwords, w0 + per);
-  int c = 0;
-  for (int w = w0; w < w1; ++w) c += __popc(__ldcg(bm + w));
+  if (seed_state) {
+    int32_t* o = seed_state + (base + s) * 4;
+    o[0] = u;
+    o[1] = v;
+    o[2] = s < ns ? st.nq[base + s] : 0;
+    o[3] = conv;
+  }
+}
+
+// Count: output pixels in each block of kMergeThreads bitmap words.
+__global__ void frm_count_kernel(FrmState st) {
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.y;
+  const int w = blockIdx.x * kMergeThreads + threadIdx.x;
+  const int c = w < st.nwords ? __popc(st.bitmap[static_cast<int64_t>(b) * st.nwords + w]) : 0;
   int tot;
-  int pos = block_exclusive_scan(c, &tot);
+  (void)block_exclusive_scan(c, &tot);
+  if (threadIdx.x == 0) st.mcounts[static_cast<int64_t>(b) * st.mblocks + blockIdx.x] = tot;
+}
+
+// Emit: each block writes (pixel, partner) for its words from its offset in
+// the pair's output; the last block of a pair writes the pair's count.
+__global__ void frm_emit_kernel(FrmState st, int32_t* pairs, int64_t cap, int32_t* count_out) {
+  pdl_wait();
+  const int b = blockIdx.y;
+  const int32_t* mc = st.mcounts + static_cast<int64_t>(b) * st.mblocks;
+  int part = 0;
+  for (int j = threadIdx.x; j < static_cast<int>(blockIdx.x); j += kMergeThreads) part += mc[j];
+  int off;
+  (void)block_exclusive_scan(part, &off);
+  const int w = blockIdx.x * kMergeThreads + threadIdx.x;
+  uint32_t bits = w < st.nwords ? st.bitmap[static_cast<int64_t>(b) * st.nwords + w] : 0u;
+  int btot;
+  int pos = off + block_exclusive_scan(__popc(bits), &btot);
   int32_t* out = pairs + static_cast<int64_t>(b) * cap * 2;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t bits = __ldcg(bm + w);
-    while (bits) {
-      const int bit = __ffs(bits) - 1;
-      bits &= bits - 1;
-      const int u = w * 32 + bit;
-      out[2 * static_cast<int64_t>(pos)] = u;
-      out[2 * static_cast<int64_t>(pos) + 1] = __ldcg(partner + u);
-      ++pos;
-    }
+  const int32_t* partner = st.partner + static_cast<int64_t>(b) * st.N1;
+  while (bits) {
+    const int bit = __ffs(bits) - 1;
+    bits &= bits - 1;
+    const int u = w * 32 + bit;
+    out[2 * static_cast<int64_t>(pos)] = u;
+    out[2 * static_cast<int64_t>(pos) + 1] = partner[u];
+    ++pos;
   }
-  if (threadIdx.x == 0) count_out[b] = tot;
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) count_out[b] = off + btot;
 }
 
 }  // namespace rnn
@@ -1128,6 +1156,21 @@ static int grid_for(int64_t n, int sms) {
   if (g > 4LL * sms) g = 4LL * sms;
   if (g < 1) g = 1;
   return static_cast<int>(g);
+}
+
+// The three merge launches (mark, count, emit) of a batched FRM call.
+static rnn_status frm_merge(const FrmState& st, int W1, int32_t* pairs, int64_t cap,
+                            int32_t* count_out, int32_t* seed_state, cudaStream_t s, bool pdl) {
+  const unsigned B = static_cast<unsigned>(st.B);
+  const dim3 blk(kMergeThreads);
+  launch_k(frm_mark_kernel, dim3((st.k + kMergeThreads - 1) / kMergeThreads, B), blk, 0, s, pdl,
+           st, W1, seed_state);
+  rnn_status r = launched();
+  if (r != RNN_OK) return r;
+  launch_k(frm_count_kernel, dim3(st.mblocks, B), blk, 0, s, pdl, st);
+  if ((r = launched()) != RNN_OK) return r;
+  launch_k(frm_emit_kernel, dim3(st.mblocks, B), blk, 0, s, pdl, st, pairs, cap, count_out);
+  return launched();
 }
 
 static rnn_status frm_step(const FrmState& st, int h, int nn2_half, int last_iter,
@@ -1403,9 +1446,7 @@ static rnn_status frm_run(int B, const void* D1, int64_t bs1, const void* D2, in
       if (ce != cudaSuccess) return RNN_ECUDA;
     }
   }
-  launch_k(frm_merge_kernel, dim3(B), dim3(kSmallThreads), 0, s, pdl, st, W1, pairs, cap,
-           count_out, seed_state);
-  return launched();
+  return frm_merge(st, W1, pairs, cap, count_out, seed_state, s, pdl);
 }
 
 // ------------------------------------------------------------- 3-D points
@@ -1571,8 +1612,7 @@ static rnn_status frm_run_pts(int B, const float* P1, int64_t bs1, const float* 
                                                    it == max_iter ? 1 : 0);
     if ((r = launched()) != RNN_OK) return r;
   }
-  frm_merge_kernel<<<B, kSmallThreads, 0, s>>>(st, W1, pairs, cap, count_out, seed_state);
-  return launched();
+  return frm_merge(st, W1, pairs, cap, count_out, seed_state, s, false);
 }
 
 }  // namespace rnn
