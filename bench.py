@@ -31,22 +31,35 @@ import time
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
 # the fused kernel in the bench step, from one ncu capture of the step's
-# first FRM call (20 launches averaged).  It belongs to the kernel sources it
-# was taken on: with any other sources the bench reports traffic as null.
-TRAFFIC = {"sources_sha256": "484732799122cc22fd04085a024d82f3299be8264274d91f7661eef68193e127",
+# first FRM call (20 launches averaged).  It belongs to the sources that
+# determine that kernel's memory traffic (see _kernel_sources_sha256): with any
+# other sources the bench reports traffic as null.
+TRAFFIC = {"sources_sha256": "767ed186debf1de4f731e048633419dda6a9f9fc05f4c22264d6df1b7bf11585",
            "frm_nn_bytes_per_launch": 37.29e6}
+
+# What fixes the fused kernel's traffic: its own code and the PTX helpers,
+# and in the ABI source the functions that size its tiles, launch it, build
+# its tensor maps and write the zero-padded rows it reads.
+_TRAFFIC_FILES = ("nn_kernel.cuh", "ptx.cuh")
+_TRAFFIC_FUNCS = ("static Geometry geometry(", "static rnn_status launch_nn(",
+                  "static rnn_status make_map(", "__device__ __forceinline__ uint4 prep_chunk(",
+                  "__global__ void prep_rows_kernel(")
 
 
 def _kernel_sources_sha256() -> str:
-    import glob
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)),
                         "reciprocal_nearest_neighbour_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(csrc, "*.cu*"))):
-        h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
+    for f in _TRAFFIC_FILES:
+        h.update(f.encode())
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
+    with open(os.path.join(csrc, "rnn.cu")) as fh:
+        text = fh.read()
+    for sig in _TRAFFIC_FUNCS:
+        i = text.index(sig)
+        h.update(text[i:text.index("\n}\n", i)].encode())
     return h.hexdigest()
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
