@@ -145,7 +145,7 @@ rnn_status rnn_mnn_exhaustive(const void *D1, int H1, int W1, const void *D2, in
  *   output the (U, V) of the seeds that are no longer active, unique, sorted
  *          by U.  Every output pair is in M.
  *
- * The whole loop runs on the device: 4*max_iter + 2 kernel launches (2 more
+ * The whole loop runs on the device: 4*max_iter + 4 kernel launches (2 more
  * when d needs padded copies), no host synchronisation.
  *
  *   seed_stride >= 1, max_iter >= 1 (RNN_EINVAL otherwise).
@@ -217,7 +217,7 @@ rnn_status rnn_frm_match_batched(int B, const void *D1, int64_t d1_batch_stride,
  *                hold -1, -1, 0, 0.
  * rnn_frm_workspace_size_ex takes n_init = the starts per pair, or -1 for the
  * grid of stride seed_stride.
- * 2 + 4*max_iter kernel launches, plus 2 (padded copies, dot metric with
+ * 4 + 4*max_iter kernel launches, plus 2 (padded copies, dot metric with
  * d = 8, 24, 40, ...) or 4 (Euclidean metric) for the row copies, plus 2 with
  * given starts.
  */
@@ -331,7 +331,7 @@ rnn_status rnn_mnn_mutual(const int32_t *rowarg, int64_t n1, const int32_t *cola
  * All four maps share dtype; C1/C2 and F1/F2 follow the descriptor rules
  * (16-byte aligned, dc and d multiples of 8).  rnn_workspace_status() on the
  * workspace reports a timed-out wait of any part.  No host synchronisation;
- * 13 + 4*max_iter kernel launches, plus the row copies: 2 when dc needs
+ * 15 + 4*max_iter kernel launches, plus the row copies: 2 when dc needs
  * padding (dc = 8, 24, 40, ...), and with RNN_L2 4 for the coarse and 4 for
  * the fine Euclidean forms.
  */
@@ -382,7 +382,7 @@ rnn_status rnn_c2f_match(const void *C1, int Hc1, int Wc1, const void *C2, int H
  *   rnn_frm_match_ex (batch strides in floats, at least 3*H*W; init_xy1,
  *   n_init, pixel_tol, basin_out, cap and seed_state_out as there).
  *   rnn_pts_frm_workspace_size takes n_init = starts per pair, or -1 for the
- *   grid of stride seed_stride.  8 + 2*max_iter kernel launches (2 more with
+ *   grid of stride seed_stride.  10 + 2*max_iter kernel launches (2 more with
  *   given starts).
  */
 size_t rnn_pts_nn_workspace_size(int64_t nq, int64_t nx);
