@@ -1,0 +1,503 @@
+// One-pass fused kernel for the exhaustive reciprocal set.
+//
+// M = {(i,j) | j = NN2(D1_i) and i = NN1(D2_j)} (cv-learn.com "MASt3R" note,
+// paragraph "Fast reciprocal matching (FRM)") needs the largest score of
+// every row AND of every column of S = D1 * D2^T.  The two-sweep form
+// (nn_kernel.cuh with both families) computes every score twice on the
+// tensor cores.  This kernel computes each 128 x 256 tile of S once
+// (tcgen05.mma, fp32 in tensor memory) and reduces it in both directions.
+//
+// Tensor-memory reads.  Each epilogue warp owns a quadrant q of the 128
+// lanes (rows) and a 64-column part p of the tile.  It reads its 32 x 64
+// block with two tcgen05.ld.16x256b.x8, which gives every thread 4 rows x 16
+// columns (rows g, g+8, g+16, g+24 with g = lane/4; columns 8j + 2s + e with
+// s = lane%4).  So a thread holds 4 rows of each of its columns, and each
+// column needs only a cross-lane step over 8 lanes, each row over 4 lanes.
+//
+// Loop order.  A work unit is bm m-tiles (image-1 rows) x bn n-tiles (image-2
+// rows).  For each n-tile, the m-tiles go by in the inner loop, so every
+// thread keeps the running maximum of its 16 columns in registers over the
+// whole inner loop (two three-input maxima per column and tile) and merges
+// across lanes and quadrants once per n-tile.  Row partials (one per row and
+// 64-column part, after a two-step shuffle across 4 lanes) go to shared
+// memory, where each (m-tile, row, part) slot keeps the best over the n-tiles
+// with the first n-tile that reached it; they are merged and written once
+// per unit.
+//
+// Ragged edges.  The maps are read from copies whose rows past the last
+// pixel (up to a whole unit) are NaN, so every score there is NaN, and the
+// three-input maximum (like fmaxf) returns the other operands when one is
+// NaN: those rows and columns never take part, with no masks in the loop.  A
+// part or quadrant wholly past the end reduces to NaN and is skipped when
+// written.
+//
+// Chunks and the exact index.  As in the row-only kernel, the fold keeps the
+// maximum and the first chunk reaching it; a locate pass afterwards resolves
+// the lowest index inside the chunk.  Row chunks are the 64-column parts.
+// For columns, the quadrant is the finest piece a lane-group merge can name,
+// so the query tile of m-tile l of m-block mb is gathered as four 32-row
+// slices: quadrant q holds rows mb*128*bm + 32*(bm*q + l) + [0, 32).  Then
+// quadrant q over the bm m-tiles of the block is the contiguous range
+// [mb*128*bm + 32*bm*q, +32*bm): the column chunk.  Chunks compare by their
+// maxima with a strict '>' in increasing order, so the kept chunk is the
+// first that holds the maximum.
+//
+// Warp roles (18 warps):
+//   warp 0       TMA producer: the bm query tiles of a unit (four 32-row
+//                boxes each) once per unit, the candidate tile once per n-tile
+//   warp 1       MMA issuer (one warp: every commit then covers every MMA
+//                that read a shared-memory slot before it is refilled)
+//   warps 2..17  epilogue, quadrant q = warp % 4, part p = (warp - 2) / 4
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include "nn_kernel.cuh"
+#include "ptx.cuh"
+
+#ifndef RNN_OP_PIPE
+#define RNN_OP_PIPE 0
+#endif
+
+namespace rnn {
+
+constexpr int kOpEpiWarp0 = 2;
+constexpr int kOpEpiWarps = 16;
+constexpr int kOpThreads = (kOpEpiWarp0 + kOpEpiWarps) * 32;  // 576
+constexpr int kOpBlockN = 256;
+constexpr int kOpMaxBm = 16;      // query tiles a unit holds in shared memory
+constexpr int kOpMaxBn = 8;       // candidate tiles per unit (row chunk ids are bytes)
+constexpr int kOpRowChunk = 64;   // columns of a row chunk (one epilogue warp's part)
+
+struct OnePassParams {
+  int n1, n2;            // image-1 rows (tensor-memory lanes), image-2 rows (columns)
+  int kpad;              // K of the tiles: 16, 32 or 64 (one K-block, swizzle 2*kpad bytes)
+  int bm, bn;            // m-tiles and n-tiles of a unit
+  int mblocks, nblocks;  // units = mblocks * nblocks; unit u -> (u % mblocks, u / mblocks)
+  uint32_t idesc;
+  unsigned long long* rowk;  // [n1] (score, first column of the row chunk), atomicMax
+  unsigned long long* colk;  // [n2] (score, first row of the column chunk), atomicMax
+  int* err;
+  unsigned long long wait_limit_ns;
+  int stall_loads;       // failure-detection test: load nothing, so the MMA warp's wait runs out
+};
+
+// Shared-memory layout, offsets from the 1024-byte aligned base.
+struct OnePassSmem {
+  uint32_t a_off, b_off, rbest_off, rchunk_off, colred_off, bar_off, misc_off, total;
+};
+
+__host__ __device__ inline OnePassSmem onepass_smem(int kpad, int bm) {
+  OnePassSmem s;
+  const uint32_t a_bytes = 128u * static_cast<uint32_t>(kpad) * 2u;
+  const uint32_t b_bytes = 256u * static_cast<uint32_t>(kpad) * 2u;
+  s.a_off = 0;
+  s.b_off = s.a_off + static_cast<uint32_t>(bm) * a_bytes;
+  s.rbest_off = s.b_off + 2u * b_bytes;                             // float [bm][4][128]
+  s.rchunk_off = s.rbest_off + static_cast<uint32_t>(bm) * 4u * 128u * 4u;  // u8 [bm][4][128]
+  s.colred_off = (s.rchunk_off + static_cast<uint32_t>(bm) * 4u * 128u + 15u) & ~15u;
+  s.bar_off = s.colred_off + 2u * 4u * 256u * 4u;                   // float [2][4][256]
+  // a_full[16], a_empty[16], b_full[2], b_empty[2], acc_full[2], acc_empty[2],
+  // colbar[4], rowbar, drain
+  s.misc_off = s.bar_off + (2u * kOpMaxBm + 14u) * 8u;
+  s.total = s.misc_off + 16u;
+  return s;
+}
+
+// Keep one of two values and send the other to the partner lane `mask`
+// away; the lane whose bit is set keeps `hi`.  Returns the larger of the
+// kept value and the partner's.
+__device__ __forceinline__ float swap_max(float lo, float hi, bool bit, int mask) {
+  const float send = bit ? lo : hi;
+  const float keep = bit ? hi : lo;
+  return fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, mask));
+}
+
+__global__ void __launch_bounds__(kOpThreads, 1)
+mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
+                   const __grid_constant__ CUtensorMap amap,   // image-1 rows, 32-row boxes
+                   const __grid_constant__ CUtensorMap bmap) { // image-2 rows, 256-row boxes
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const OnePassSmem L = onepass_smem(p.kpad, p.bm);
+  uint8_t* a_tiles = smem + L.a_off;
+  uint8_t* b_tiles = smem + L.b_off;
+  float* rbest = reinterpret_cast<float*>(smem + L.rbest_off);
+  uint8_t* rchunk = smem + L.rchunk_off;
+  float* colred = reinterpret_cast<float*>(smem + L.colred_off);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = bars + kOpMaxBm;
+  uint64_t* b_full = bars + 2 * kOpMaxBm;
+  uint64_t* b_empty = b_full + 2;
+  uint64_t* acc_full = b_empty + 2;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* colbar = acc_empty + 2;
+  uint64_t* rowbar = colbar + 4;
+  uint64_t* drain_bar = rowbar + 1;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L.misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t a_bytes = 128u * static_cast<uint32_t>(p.kpad) * 2u;
+  const uint32_t b_bytes = 256u * static_cast<uint32_t>(p.kpad) * 2u;
+  const int units = p.mblocks * p.nblocks;
+  const int bm = p.bm, bn = p.bn;
+
+  if (threadIdx.x == 0) {
+    for (int l = 0; l < bm; ++l) {
+      mbar_init(smem_u32(&a_full[l]), 1);
+      mbar_init(smem_u32(&a_empty[l]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&b_full[i]), 1);
+      mbar_init(smem_u32(&b_empty[i]), 1);
+      mbar_init(smem_u32(&acc_full[i]), 1);
+      mbar_init(smem_u32(&acc_empty[i]), kOpEpiWarps);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&colbar[i]), 4);
+    mbar_init(smem_u32(rowbar), kOpEpiWarps);
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&bmap);
+  }
+  __syncthreads();
+  if (static_cast<int>(blockIdx.x) >= units) return;
+  if (warp == 1) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+  const uint64_t lim = p.wait_limit_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int a_it = 0;         // unit iterations: each query slot is loaded once per unit
+      long long b_cnt = 0;  // candidate tiles loaded
+      // parity of the phase the last load issued into each candidate slot
+      // completes (-1: none); query slots 0..a_n-1 were last loaded in unit
+      // iteration a_last, the others in a_last - 1
+      int b_par0 = -1, b_par1 = -1, a_last = -1, a_n = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++a_it) {
+        const int mb = u % p.mblocks, nb = u / p.mblocks;
+        for (int n = 0; n < bn && ok; ++n) {
+          const int bs = static_cast<int>(b_cnt & 1);
+          const uint32_t use = static_cast<uint32_t>((b_cnt >> 1) & 1);  // phase of this use
+          if (!mbar_wait_sleep(smem_u32(&b_empty[bs]), use ^ 1u, abort_flag, p.err,
+                               kErrWaitProducer, lim)) {
+            ok = false;
+            break;
+          }
+          if (!p.stall_loads) {
+            const uint32_t fb = smem_u32(&b_full[bs]);
+            mbar_arrive_expect_tx(fb, b_bytes);
+            tma_load_3d(smem_u32(b_tiles + bs * b_bytes), &bmap, fb, 0, (nb * bn + n) * kOpBlockN,
+                        0);
+            if (bs == 0) b_par0 = static_cast<int>(use); else b_par1 = static_cast<int>(use);
+          }
+          ++b_cnt;
+          if (n != 0) continue;
+          for (int l = 0; l < bm; ++l) {
+            if (!mbar_wait_sleep(smem_u32(&a_empty[l]), static_cast<uint32_t>(a_it & 1) ^ 1u,
+                                 abort_flag, p.err, kErrWaitProducer, lim)) {
+              ok = false;
+              break;
+            }
+            if (!p.stall_loads) {
+              const uint32_t fa = smem_u32(&a_full[l]);
+              mbar_arrive_expect_tx(fa, a_bytes);
+              const uint32_t dst = smem_u32(a_tiles + l * a_bytes);
+              for (int q = 0; q < 4; ++q)
+                tma_load_3d(dst + q * (a_bytes / 4), &amap, fa, 0,
+                            mb * 128 * bm + 32 * (bm * q + l), 0);
+              a_last = a_it;
+              a_n = l + 1;
+            }
+          }
+        }
+      }
+      if (!ok) {
+        // wait (bounded) for the loads still in flight before the CTA exits
+        const uint64_t t0 = globaltimer_ns();
+        for (int i = 0; i < 2 + bm; ++i) {
+          const int al = i - 2 < a_n ? a_last : a_last - 1;
+          const int par = i == 0 ? b_par0 : i == 1 ? b_par1 : (al < 0 ? -1 : (al & 1));
+          if (par < 0) continue;
+          const uint32_t bar = smem_u32(i < 2 ? &b_full[i] : &a_full[i - 2]);
+          while (!mbar_try_wait(bar, static_cast<uint32_t>(par))) {
+            if (globaltimer_ns() - t0 > lim) {
+              atomicOr(p.err, kErrDrain);
+              break;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    long long T = 0, b_cnt = 0;
+    int a_it = 0;
+    bool ok = true, any = false;
+    const uint64_t a_desc0 = make_sdesc(smem_u32(a_tiles), p.kpad);
+    const uint64_t b_desc0 = make_sdesc(smem_u32(b_tiles), p.kpad);
+    const uint32_t a_step = a_bytes >> 4, b_step = b_bytes >> 4;
+    const int ksteps = p.kpad / 16;
+    const uint32_t idesc = p.idesc;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++a_it) {
+      for (int n = 0; n < bn && ok; ++n, ++b_cnt) {
+        const int bs = static_cast<int>(b_cnt & 1);
+        const uint32_t bpar = static_cast<uint32_t>((b_cnt >> 1) & 1);
+        for (int l = 0; l < bm; ++l, ++T) {
+          const int acc = static_cast<int>(T & 1);
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(smem_u32(&a_full[l]), static_cast<uint32_t>(a_it & 1),
+                                    abort_flag, p.err, kErrWaitMma, lim) &&
+                              mbar_wait(smem_u32(&b_full[bs]), bpar, abort_flag, p.err,
+                                        kErrWaitMma, lim) &&
+                              mbar_wait_sleep(smem_u32(&acc_empty[acc]),
+                                              static_cast<uint32_t>((T >> 1) & 1) ^ 1u,
+                                              abort_flag, p.err, kErrWaitMma, lim));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kOpBlockN);
+          const uint64_t a = a_desc0 + static_cast<uint64_t>(l) * a_step;
+          const uint64_t b = b_desc0 + static_cast<uint64_t>(bs) * b_step;
+          for (int k = 0; k < ksteps; ++k)
+            umma_f16_warp(d_tmem, a + 2 * k, b + 2 * k, idesc, k > 0 ? 1u : 0u);
+          umma_commit_warp(smem_u32(&acc_full[acc]));
+          if (n == bn - 1) umma_commit_warp(smem_u32(&a_empty[l]));  // last read of slot l
+          if (l == bm - 1) umma_commit_warp(smem_u32(&b_empty[bs]));  // last read of slot bs
+          __syncwarp();
+          any = true;
+        }
+      }
+    }
+    if (!ok && any) {
+      // let every MMA issued finish before tensor memory is released
+      umma_commit_warp(smem_u32(drain_bar));
+      __syncwarp();
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(drain_bar), 0)) {
+        if (globaltimer_ns() - t0 > lim) {
+          if (lane == 0) atomicOr(p.err, kErrDrain);
+          break;
+        }
+      }
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int e = warp - kOpEpiWarp0;
+    const int q = warp & 3;        // tensor-memory lane quadrant this warp may read
+    const int part = e >> 2;       // 64-column part of the tile
+    const int g = lane >> 2, s = lane & 3;
+    const bool s0 = (lane & 1) != 0, s1 = (lane & 2) != 0;
+    const bool g0 = (lane & 4) != 0, g1 = (lane & 8) != 0, g2 = (lane & 16) != 0;
+    const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                        static_cast<uint32_t>(64 * part);
+    // this lane's row-state slot: row 32q + g + 8s of part `part`, per m-tile l
+    const int rslot = part * 128 + 32 * q + g + 8 * s;
+    const uint32_t rb_s = smem_u32(rbest) + 4u * rslot, rc_s = smem_u32(rchunk) + rslot;
+    const uint32_t cr_s = smem_u32(colred);
+    const float ninf = -__int_as_float(0x7f800000);
+    uint32_t T = 0;  // tile sequence of this CTA (only its two low bits are used)
+    int flushes = 0, rowphase = 0;
+    bool ok = true;
+    // Software pipeline over the tiles of this CTA: each tile is read in two
+    // halves (rows g, g+8 into va; rows g+16, g+24 into vb).  The read of vb
+    // runs while va is folded, and the read of the next tile's va runs while
+    // vb is folded, so the tensor-memory latency hides behind the folds with
+    // 64 value registers.  `pend`: va's read for tile T is already issued.
+    float va[32], vb[32];
+    bool pend = false;
+#if !RNN_OP_PIPE
+    constexpr bool kPipe = false;
+#else
+    constexpr bool kPipe = true;
+#endif
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const int mb = u % p.mblocks, nb = u / p.mblocks;
+      const int row_base = mb * 128 * bm;
+      for (int n = 0; n < bn && ok; ++n) {
+        const int col0 = (nb * bn + n) * kOpBlockN + 64 * part;  // first column of this part
+        float pm[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pm[c] = ninf;
+        for (int l = 0; l < bm; ++l, ++T) {
+          const uint32_t ta = tq + static_cast<uint32_t>((T & 1u) * kOpBlockN);
+          if (!pend) {
+            if (!mbar_wait_sleep(smem_u32(&acc_full[T & 1u]), (T >> 1) & 1u, abort_flag, p.err,
+                                 kErrWaitEpilogue, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            tmem_ld16x256_x8(ta, va);
+          }
+          if (!kPipe) tmem_ld16x256_x8(ta + (16u << 16), vb);
+          tmem_wait_ld_regs(va);
+          if (!kPipe) {
+            reg_fence(vb);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[T & 1u]));
+          } else {
+            tmem_ld16x256_x8(ta + (16u << 16), vb);
+          }
+          reg_fence(va);
+          // first half: columns over rows g, g+8; rows g and g+8 over this thread's 16 columns
+          // (column by column, so that each group of four values dies early)
+          float r0 = fmaxf(va[0], va[1]), r1 = fmaxf(va[2], va[3]);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              pm[2 * j + h] = fmax3(pm[2 * j + h], va[4 * j + h], va[4 * j + 2 + h]);
+            if (j > 0) {
+              r0 = fmax3(r0, va[4 * j], va[4 * j + 1]);
+              r1 = fmax3(r1, va[4 * j + 2], va[4 * j + 3]);
+            }
+          }
+          // the first half's folds before the wait for the second half
+#pragma unroll
+          for (int c = 0; c < 16; ++c) keep_order(pm[c]);
+          keep_order(r0);
+          keep_order(r1);
+          if (kPipe) {
+            tmem_wait_ld_regs(vb);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[T & 1u]));
+          }
+          // the next tile's first half, read during this tile's second fold
+          // (within the candidate tile: its column flush comes first)
+          pend = false;
+          if (kPipe && l != bm - 1) {
+            const uint32_t T1 = T + 1u;
+            if (!mbar_wait_sleep(smem_u32(&acc_full[T1 & 1u]), (T1 >> 1) & 1u, abort_flag, p.err,
+                                 kErrWaitEpilogue, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            tmem_ld16x256_x8(tq + static_cast<uint32_t>((T1 & 1u) * kOpBlockN), va);
+            pend = true;
+          }
+          reg_fence(vb);
+          // second half: rows g+16, g+24
+          float r2 = fmaxf(vb[0], vb[1]), r3 = fmaxf(vb[2], vb[3]);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              pm[2 * j + h] = fmax3(pm[2 * j + h], vb[4 * j + h], vb[4 * j + 2 + h]);
+            if (j > 0) {
+              r2 = fmax3(r2, vb[4 * j], vb[4 * j + 1]);
+              r3 = fmax3(r3, vb[4 * j + 2], vb[4 * j + 3]);
+            }
+          }
+          // across the 4 lanes holding the same rows: lane s ends with row g + 8s
+          const float x0 = swap_max(r0, r1, s0, 1);  // row (s & 1)
+          const float x1 = swap_max(r2, r3, s0, 1);  // row 2 + (s & 1)
+          const float y = swap_max(x0, x1, s1, 2);   // row s
+          const uint32_t slot = rb_s + 2048u * l, cslot = rc_s + 512u * l;
+          if (n == 0) {
+            sts_f32(slot, y);
+            sts_u8(cslot, 0u);
+          } else if (y > lds_f32(slot)) {
+            sts_f32(slot, y);
+            sts_u8(cslot, static_cast<uint32_t>(n));
+          }
+        }
+        if (!ok) break;
+        // ---- column flush: over the 8 lanes of this quadrant holding the same columns
+        float x[8], y4[4], z[2];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = swap_max(pm[i], pm[i + 8], g2, 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y4[i] = swap_max(x[i], x[i + 4], g1, 8);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) z[i] = swap_max(y4[i], y4[i + 2], g0, 4);
+        // z[h]: column 8g + 2s + h of this part, over the quadrant's 32*bm rows
+        const uint32_t cr = cr_s + 4096u * (flushes & 1);
+        sts_v2f32(cr + 4u * (q * 256 + 64 * part + 8 * g + 2 * s), z[0], z[1]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&colbar[part]));
+        if (!mbar_wait(smem_u32(&colbar[part]), static_cast<uint32_t>(flushes & 1), abort_flag,
+                       p.err, kErrWaitEpilogue, lim)) {
+          ok = false;
+          break;
+        }
+        if (lane < 16) {
+          const int c = 16 * q + lane;  // this warp's share of the part's columns
+          float best = lds_f32(cr + 4u * (64 * part + c));
+          int bq = 0;
+#pragma unroll
+          for (int qq = 1; qq < 4; ++qq) {
+            const float v = lds_f32(cr + 4u * (qq * 256 + 64 * part + c));
+            if (v > best) {
+              best = v;
+              bq = qq;
+            }
+          }
+          if (col0 + c < p.n2)
+            atomicMax(p.colk + col0 + c, pack_key(best, row_base + 32 * bm * bq));
+        }
+        ++flushes;
+      }
+      if (!ok) break;
+      // ---- row flush: every epilogue warp has written its slots for this unit
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(rowbar));
+      if (!mbar_wait(smem_u32(rowbar), static_cast<uint32_t>(rowphase & 1), abort_flag, p.err,
+                     kErrWaitEpilogue, lim)) {
+        ok = false;
+        break;
+      }
+      ++rowphase;
+      for (int r = e * 32 + lane; r < bm * 128; r += kOpEpiWarps * 32) {
+        const int l = r >> 7, rl = r & 127;
+        unsigned long long best = 0;
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          const float v = lds_f32(smem_u32(rbest) + 4u * (l * 512 + pp * 128 + rl));
+          const int nn = static_cast<int>(lds_u8(smem_u32(rchunk) + l * 512 + pp * 128 + rl));
+          // a part wholly past the last image-2 row holds NaN
+          const unsigned long long k =
+              v == v ? pack_key(v, (nb * bn + nn) * kOpBlockN + 64 * pp) : 0ull;
+          best = k > best ? k : best;
+        }
+        const int grow = row_base + 32 * (bm * (rl >> 5) + l) + (rl & 31);
+        if (grow < p.n1) atomicMax(p.rowk + grow, best);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(rowbar));
+      if (!mbar_wait(smem_u32(rowbar), static_cast<uint32_t>(rowphase & 1), abort_flag, p.err,
+                     kErrWaitEpilogue, lim)) {
+        ok = false;
+        break;
+      }
+      ++rowphase;
+    }
+    // an abort after the next tile's read was issued: let it land before the
+    // tensor memory is released
+    if (pend) tmem_wait_ld();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace rnn

@@ -19,6 +19,7 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include "mnn_kernel.cuh"
 #include "nn_kernel.cuh"
 #include "rnn.h"
 
@@ -61,6 +62,7 @@ struct DeviceInfo {
   int sms = 0;
   bool sm100 = false;
   bool smem_set = false;
+  bool op_smem_set = false;  // one-pass exhaustive-set kernels
 };
 
 static std::mutex g_mu;
@@ -150,6 +152,17 @@ static Geometry geometry(int d) {
   return g;
 }
 
+// The one-pass kernel for the exhaustive set covers one K-block of 16, 32 or
+// 64 (d <= 32 or d = 64) with the dot metric; other shapes take the
+// two-sweep form.  Its copies of the maps carry kOpPadRows NaN rows past the
+// last pixel: enough for the last unit (bm*128 <= 2048 query rows, 8*256
+// candidate rows) to read nothing but NaN beyond the end.
+constexpr int64_t kOpPadRows = 2048;
+static bool onepass_fits(const Geometry& g, rnn_metric metric) {
+  return metric == RNN_DOT && g.nkb == 1 && g.block_n == kOpBlockN &&
+         (g.kpad == 16 || g.kpad == 32 || g.kpad == 64);
+}
+
 // Depth K of the tensor-core tiles for d channels (d rounded up to the
 // K-block layout the geometry picks).
 static int padded_depth(int d) { return geometry(d).kpad; }
@@ -237,6 +250,24 @@ static void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
   (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Benchmark timer (rnn_set_kernel_timer): events around the fused kernels.
+static rnn_status timer_begin(cudaStream_t s, int* slot) {
+  *slot = -1;
+  if (t_capturing || !g_timer_count || !g_timer_start || !g_timer_stop) return RNN_OK;
+  const int k = (*g_timer_count)++;
+  if (k >= g_timer_cap) return RNN_OK;
+  if (cudaEventRecord(static_cast<cudaEvent_t>(g_timer_start[k]), s) != cudaSuccess)
+    return RNN_ECUDA;
+  *slot = k;
+  return RNN_OK;
+}
+
+static rnn_status timer_end(cudaStream_t s, int slot) {
+  if (slot >= 0 && cudaEventRecord(static_cast<cudaEvent_t>(g_timer_stop[slot]), s) != cudaSuccess)
+    return RNN_ECUDA;
+  return RNN_OK;
+}
+
 static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const CUtensorMap& m1,
                             const CUtensorMap& q0, const CUtensorMap& q1, const Geometry& g,
                             DeviceInfo* di, cudaStream_t s, bool pdl = false) {
@@ -273,14 +304,9 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
     }
   }
   int slot = -1;
-  if (!t_capturing && g_timer_count && g_timer_start && g_timer_stop) {
-    slot = (*g_timer_count)++;
-    if (slot < g_timer_cap) {
-      if (cudaEventRecord(static_cast<cudaEvent_t>(g_timer_start[slot]), s) != cudaSuccess)
-        return RNN_ECUDA;
-    } else {
-      slot = -1;
-    }
+  {
+    const rnn_status tr = timer_begin(s, &slot);
+    if (tr != RNN_OK) return tr;
   }
   // Epilogue layout.  Two 256-column accumulators: sixteen warps, all on
   // every tile, each 64 columns of its lane quadrant in one copy, so an
@@ -313,10 +339,7 @@ static rnn_status launch_nn(const NNParams& p_in, const CUtensorMap& m0, const C
       launch_k(nn_argmax_kernel<16, 4, 2>, grid, block, g.smem, s, false, p, m0, m1, q0, q1);
   }
   const rnn_status r = launched();
-  if (r == RNN_OK && slot >= 0 &&
-      cudaEventRecord(static_cast<cudaEvent_t>(g_timer_stop[slot]), s) != cudaSuccess)
-    return RNN_ECUDA;
-  return r;
+  return r == RNN_OK ? timer_end(s, slot) : r;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -717,6 +740,197 @@ __global__ void mutual_write_kernel(const int32_t* rowarg, int64_t n1, const int
     }
   }
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) *count_out = off + btot;
+}
+
+// ------------------------------------------- grouped locate (one-pass M)
+// The one-pass kernel leaves row keys whose chunk is kOpRowChunk candidates
+// of image 2, and column keys whose chunk is 32*bm candidates of image 1.
+// The exact lowest index inside a chunk comes from recomputing the chunk's
+// scores (fp32 fused multiply-adds over the channels in order, as in
+// locate_chunk).  A column chunk is hundreds of rows, so the queries are
+// grouped by chunk first: each chunk's candidates are then read once into
+// shared memory and serve all of its queries.  Four launches: count per
+// chunk, scan, scatter of the query ids, and the resolve over items of at
+// most kLocItem queries of one chunk.
+constexpr int kLocItem = 256;
+
+struct LocParams {
+  unsigned long long* rowk;  // [n1] row keys, chunks of lr columns (image 2)
+  unsigned long long* colk;  // [n2] column keys, chunks of lc rows (image 1)
+  int64_t n1, n2;
+  int lr, lc;
+  int nch_r, nch;            // row chunks; all chunks (row chunks first)
+  int* cnt;                  // [nch] queries per chunk
+  int* start;                // [nch + 1] first list position of each chunk
+  int* items;                // [nch + 1] first item of each chunk
+  int* cursor;               // [nch] fill counters of the scatter
+  uint32_t* list;            // [n1 + n2] query ids: image-1 row i, or n1 + image-2 row j
+  const uint16_t* X1;        // rows of image 1 and image 2, ld elements apart
+  const uint16_t* X2;
+  int ld;
+};
+
+__device__ __forceinline__ int loc_chunk(const LocParams& P, int64_t i) {
+  if (i < P.n1) {
+    int c0 = key_index(P.rowk[i]);
+    if (c0 < 0 || c0 >= P.n2) c0 = 0;  // a key no candidate reached (after an abort)
+    return c0 / P.lr;
+  }
+  int c0 = key_index(P.colk[i - P.n1]);
+  if (c0 < 0 || c0 >= P.n1) c0 = 0;
+  return P.nch_r + c0 / P.lc;
+}
+
+__global__ void zero_words_kernel(int* a, int64_t n) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += stride)
+    a[i] = 0;
+}
+
+// The one-pass kernel's copy of a map: rows of kpad elements, the d channels
+// then zeros, and NaN rows from row n to ntot.  One thread per 16-byte chunk
+// of the output.
+__global__ void op_copy_kernel(const uint16_t* __restrict__ src, int64_t n, int d,
+                               uint16_t* __restrict__ dst, int kpad, int64_t ntot, int bf16) {
+  const int cpr = kpad / 8, creal = d / 8;
+  const uint16_t nan16 = bf16 ? 0x7FC0u : 0x7E00u;
+  const uint32_t nan2 = static_cast<uint32_t>(nan16) * 0x10001u;
+  const int64_t total = ntot * cpr, stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += stride) {
+    const int64_t r = i / cpr;
+    const int c = static_cast<int>(i - r * cpr);
+    uint4 v;
+    if (r >= n)
+      v = make_uint4(nan2, nan2, nan2, nan2);
+    else if (c < creal)
+      v = __ldg(reinterpret_cast<const uint4*>(src + r * d) + c);
+    else
+      v = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(dst)[i] = v;
+  }
+}
+
+__global__ void loc_count_kernel(LocParams P) {
+  const int64_t n = P.n1 + P.n2, stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += stride) {
+    const int c = loc_chunk(P, i);
+    const unsigned m = __match_any_sync(__activemask(), c);
+    if ((threadIdx.x & 31) == __ffs(m) - 1) atomicAdd(P.cnt + c, __popc(m));
+  }
+}
+
+// One block: exclusive scans of the counts and of the items per chunk.
+__global__ void loc_scan_kernel(LocParams P) {
+  const int n = P.nch;
+  const int per = (n + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x);
+  const int b0 = threadIdx.x * per;
+  int sc = 0, si = 0;
+  for (int k = 0; k < per; ++k) {
+    const int c = b0 + k;
+    if (c < n) {
+      sc += P.cnt[c];
+      si += (P.cnt[c] + kLocItem - 1) / kLocItem;
+    }
+  }
+  int tc, ti;
+  int oc = block_exclusive_scan(sc, &tc);
+  int oi = block_exclusive_scan(si, &ti);
+  for (int k = 0; k < per; ++k) {
+    const int c = b0 + k;
+    if (c < n) {
+      P.start[c] = oc;
+      P.items[c] = oi;
+      P.cursor[c] = 0;
+      oc += P.cnt[c];
+      oi += (P.cnt[c] + kLocItem - 1) / kLocItem;
+    }
+  }
+  if (threadIdx.x == 0) {
+    P.start[n] = tc;
+    P.items[n] = ti;
+  }
+}
+
+__global__ void loc_scatter_kernel(LocParams P) {
+  const int64_t n = P.n1 + P.n2, stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int lane = threadIdx.x & 31;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += stride) {
+    const int c = loc_chunk(P, i);
+    const unsigned m = __match_any_sync(__activemask(), c);
+    const int leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(P.cursor + c, __popc(m));
+    base = __shfl_sync(m, base, leader);
+    const int rank = __popc(m & ((1u << lane) - 1u));
+    P.list[P.start[c] + base + rank] = static_cast<uint32_t>(i);
+  }
+}
+
+// Items are slices of at most kLocItem queries of one chunk.  The block
+// stages the chunk's candidates as fp32 [len][kD] in shared memory; each
+// thread takes one query and scans them in increasing index with a strict
+// '>', so it keeps the lowest index reaching the largest recomputed score.
+// The key keeps the tensor cores' maximum as its score.
+template <bool kBf16, int kD>
+__global__ void __launch_bounds__(kLocItem) loc_resolve_kernel(LocParams P) {
+  extern __shared__ float cand[];
+  const int total = P.items[P.nch];
+  for (int it = blockIdx.x; it < total; it += gridDim.x) {
+    int lo = 0, hi = P.nch;  // items[lo] <= it < items[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (P.items[mid] <= it) lo = mid; else hi = mid;
+    }
+    const int c = lo;
+    const bool rows = c < P.nch_r;
+    const int L = rows ? P.lr : P.lc;
+    const int64_t ncand = rows ? P.n2 : P.n1;
+    const int64_t c0 = static_cast<int64_t>(rows ? c : c - P.nch_r) * L;
+    const int len = static_cast<int>(ncand - c0 < L ? ncand - c0 : L);
+    const uint16_t* X = rows ? P.X2 : P.X1;
+    __syncthreads();  // the previous item's readers are done with `cand`
+    for (int e = threadIdx.x; e < len * kD; e += blockDim.x) {
+      const int r = e / kD, ch = e - r * kD;
+      cand[e] = h2f(X[(c0 + r) * P.ld + ch], kBf16);
+    }
+    __syncthreads();
+    const int q0 = P.start[c] + (it - P.items[c]) * kLocItem;
+    const int qend = P.start[c] + P.cnt[c];
+    if (q0 + static_cast<int>(threadIdx.x) < qend) {
+      const uint32_t id = P.list[q0 + threadIdx.x];
+      const int64_t qi = rows ? static_cast<int64_t>(id) : static_cast<int64_t>(id) - P.n1;
+      const uint16_t* qr = (rows ? P.X1 : P.X2) + qi * P.ld;
+      float qv[kD];
+#pragma unroll
+      for (int ch = 0; ch < kD; ch += 8) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qr + ch));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          qv[ch + 2 * k] = h2f(static_cast<uint16_t>(ws[k] & 0xFFFFu), kBf16);
+          qv[ch + 2 * k + 1] = h2f(static_cast<uint16_t>(ws[k] >> 16), kBf16);
+        }
+      }
+      float best = -__int_as_float(0x7f800000);
+      int bk = 0;
+      for (int k = 0; k < len; ++k) {
+        const float* cr = cand + k * kD;
+        float acc = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < kD; ++ch) acc = fmaf(qv[ch], cr[ch], acc);
+        if (acc > best) {
+          best = acc;
+          bk = k;
+        }
+      }
+      unsigned long long* kp = rows ? P.rowk + qi : P.colk + qi;
+      *kp = pack_key(key_score(*kp), static_cast<int>(c0 + bk));
+    }
+  }
 }
 
 // ------------------------------------------------------------------- FRM
@@ -1774,6 +1988,11 @@ struct MnnWs {
   unsigned long long *rowk, *colk;
   int* counts;
   uint16_t *q1, *x1, *q2, *x2;
+  // grouped locate of the one-pass path (chunks: at most n2/64 row chunks and
+  // n1/32 column chunks)
+  int64_t nch_max;
+  int *loc_cnt, *loc_start, *loc_items, *loc_cursor;
+  uint32_t* loc_list;
 };
 
 static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, rnn_metric metric, MnnWs* w) {
@@ -1782,9 +2001,20 @@ static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, rnn_metric met
   w->rowk = c.take<unsigned long long>(n1 > 0 ? n1 : 1);
   w->colk = c.take<unsigned long long>(n2 > 0 ? n2 : 1);
   w->counts = c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
+  w->nch_max = (n2 + kOpRowChunk - 1) / kOpRowChunk + (n1 + 31) / 32;
+  w->loc_cnt = c.take<int>(w->nch_max + 1);
+  w->loc_cursor = c.take<int>(w->nch_max + 1);
+  w->loc_start = c.take<int>(w->nch_max + 1);
+  w->loc_items = c.take<int>(w->nch_max + 1);
+  w->loc_list = c.take<uint32_t>(n1 + n2 > 0 ? n1 + n2 : 1);
   w->q1 = w->x1 = w->q2 = w->x2 = nullptr;
   const int mode = d > 0 ? copies_for(d, metric) : kCopiesNone;
-  if (mode != kCopiesNone) {
+  if (d > 0 && onepass_fits(geometry(d), metric)) {
+    // one-pass form: padded rows, then kOpPadRows NaN rows
+    const int kpad = geometry(d).kpad;
+    w->q1 = w->x1 = c.take<uint16_t>((n1 + kOpPadRows) * kpad);
+    w->q2 = w->x2 = c.take<uint16_t>((n2 + kOpPadRows) * kpad);
+  } else if (mode != kCopiesNone) {
     const int kpad = tile_depth(d, metric);
     w->q1 = c.take<uint16_t>(n1 * kpad);
     w->q2 = c.take<uint16_t>(n2 * kpad);
@@ -1808,6 +2038,137 @@ size_t rnn_mnn_workspace_size_ex(int H1, int W1, int H2, int W2, int d, rnn_metr
 size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2, int d) {
   return rnn_mnn_workspace_size_ex(H1, W1, H2, W2, d, RNN_DOT);
 }
+
+}  // extern "C"
+
+// ---------------------------------------------------- one-pass exhaustive M
+struct OnePassPlan {
+  int bm, bn, mblocks, nblocks;
+};
+
+// Unit shape: the largest that shared memory holds (bm query tiles of
+// 128 x kpad, 8 candidate tiles), halved along the longer side until there
+// are at least two units per SM.
+static OnePassPlan onepass_plan(int64_t n1, int64_t n2, int kpad, int sms) {
+  const int mt = static_cast<int>((n1 + 127) / 128);
+  const int nt = static_cast<int>((n2 + kOpBlockN - 1) / kOpBlockN);
+  auto blocks = [](int t, int b) { return (t + b - 1) / b; };
+  int bm = std::min(kpad == 64 ? 8 : kOpMaxBm, mt), bn = std::min(kOpMaxBn, nt);
+  while (static_cast<int64_t>(blocks(mt, bm)) * blocks(nt, bn) < 2LL * sms && (bm > 1 || bn > 1)) {
+    if (bn >= bm && bn > 1)
+      bn = (bn + 1) / 2;
+    else
+      bm = (bm + 1) / 2;
+  }
+  return {bm, bn, blocks(mt, bm), blocks(nt, bn)};
+}
+
+template <bool kBf16>
+static rnn_status loc_resolve_launch(int d, const LocParams& P, int grid, size_t smem,
+                                     cudaStream_t s) {
+  switch (d) {
+    case 8: loc_resolve_kernel<kBf16, 8><<<grid, kLocItem, smem, s>>>(P); break;
+    case 16: loc_resolve_kernel<kBf16, 16><<<grid, kLocItem, smem, s>>>(P); break;
+    case 24: loc_resolve_kernel<kBf16, 24><<<grid, kLocItem, smem, s>>>(P); break;
+    case 32: loc_resolve_kernel<kBf16, 32><<<grid, kLocItem, smem, s>>>(P); break;
+    case 64: loc_resolve_kernel<kBf16, 64><<<grid, kLocItem, smem, s>>>(P); break;
+    default: return RNN_EUNSUPPORTED;
+  }
+  return launched();
+}
+
+template <bool kBf16>
+static cudaError_t loc_resolve_attr(int smem) {
+  const auto a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(loc_resolve_kernel<kBf16, 8>, a, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(loc_resolve_kernel<kBf16, 16>, a, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(loc_resolve_kernel<kBf16, 24>, a, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(loc_resolve_kernel<kBf16, 32>, a, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(loc_resolve_kernel<kBf16, 64>, a, smem);
+  return e;
+}
+
+// Keys of both directions from one pass over the scores, then the grouped
+// locate.  X1, X2: the rows the tensor maps read (ld elements apart).
+static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2, int64_t n2,
+                              int ld, int d, rnn_dtype dtype, const Geometry& g, const MnnWs& w,
+                              DeviceInfo* di, cudaStream_t s) {
+  constexpr int kLocSmem = 64 * 1024;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!di->op_smem_set) {
+      if (cudaFuncSetAttribute(mnn_onepass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) != cudaSuccess ||
+          loc_resolve_attr<false>(kLocSmem) != cudaSuccess ||
+          loc_resolve_attr<true>(kLocSmem) != cudaSuccess)
+        return RNN_ECUDA;
+      di->op_smem_set = true;
+    }
+  }
+  const OnePassPlan pl = onepass_plan(n1, n2, g.kpad, di->sms);
+  CUtensorMap am, bm;
+  rnn_status r;
+  const int64_t r1 = n1 + kOpPadRows, r2 = n2 + kOpPadRows;  // rows with the NaN tail
+  if ((r = make_map(&am, X1, ld, r1, 1, r1 * ld, g, 32)) != RNN_OK) return r;
+  if ((r = make_map(&bm, X2, ld, r2, 1, r2 * ld, g, kOpBlockN)) != RNN_OK) return r;
+  OnePassParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.n1 = static_cast<int>(n1);
+  p.n2 = static_cast<int>(n2);
+  p.kpad = g.kpad;
+  p.bm = pl.bm;
+  p.bn = pl.bn;
+  p.mblocks = pl.mblocks;
+  p.nblocks = pl.nblocks;
+  p.idesc = make_idesc(dtype, kOpBlockN);
+  p.rowk = w.rowk;
+  p.colk = w.colk;
+  p.err = w.err;
+  p.stall_loads = g_stall_loads.load(std::memory_order_relaxed);
+  p.wait_limit_ns = p.stall_loads ? g_stall_limit_ns.load(std::memory_order_relaxed)
+                                  : kWaitLimitNs;
+  const size_t smem = onepass_smem(g.kpad, pl.bm).total + 1024;
+  const int units = pl.mblocks * pl.nblocks;
+  int slot = -1;
+  if ((r = timer_begin(s, &slot)) != RNN_OK) return r;
+  mnn_onepass_kernel<<<std::min(units, di->sms), kOpThreads, smem, s>>>(p, am, bm);
+  if ((r = launched()) != RNN_OK) return r;
+  if ((r = timer_end(s, slot)) != RNN_OK) return r;
+
+  LocParams P;
+  P.rowk = w.rowk;
+  P.colk = w.colk;
+  P.n1 = n1;
+  P.n2 = n2;
+  P.lr = kOpRowChunk;
+  P.lc = 32 * pl.bm;
+  P.nch_r = static_cast<int>((n2 + P.lr - 1) / P.lr);
+  P.nch = P.nch_r + static_cast<int>((n1 + P.lc - 1) / P.lc);
+  P.cnt = w.loc_cnt;
+  P.start = w.loc_start;
+  P.items = w.loc_items;
+  P.cursor = w.loc_cursor;
+  P.list = w.loc_list;
+  P.X1 = X1;
+  P.X2 = X2;
+  P.ld = ld;
+  zero_words_kernel<<<grid_for(P.nch, di->sms), kSmallThreads, 0, s>>>(P.cnt, P.nch);
+  if ((r = launched()) != RNN_OK) return r;
+  loc_count_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(P);
+  if ((r = launched()) != RNN_OK) return r;
+  loc_scan_kernel<<<1, kSmallThreads, 0, s>>>(P);
+  if ((r = launched()) != RNN_OK) return r;
+  loc_scatter_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(P);
+  if ((r = launched()) != RNN_OK) return r;
+  const int64_t max_items = P.nch + (n1 + n2) / kLocItem + 1;
+  const int rg = static_cast<int>(std::min<int64_t>(max_items, 4LL * di->sms));
+  const size_t lsm = static_cast<size_t>(std::max(P.lr, P.lc)) * d * sizeof(float);
+  return dtype == RNN_BF16 ? loc_resolve_launch<true>(d, P, rg, lsm, s)
+                           : loc_resolve_launch<false>(d, P, rg, lsm, s);
+}
+
+extern "C" {
 
 rnn_status rnn_mnn_exhaustive_ex(const void* D1, int H1, int W1, const void* D2, int H2, int W2,
                                  int d, rnn_dtype dtype, rnn_metric metric, int32_t* pairs_out,
@@ -1837,6 +2198,27 @@ rnn_status rnn_mnn_exhaustive_ex(const void* D1, int H1, int W1, const void* D2,
 
   const bool l2 = metric == RNN_L2;
   const Geometry g = geometry(d + (l2 ? kAugCols : 0));
+  const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
+  zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2,
+                                                                        w.err);
+  if ((r = launched()) != RNN_OK) return r;
+  if (onepass_fits(g, metric)) {
+    // every score once, reduced by rows and by columns
+    const int bf = dtype == RNN_BF16 ? 1 : 0;
+    op_copy_kernel<<<grid_for((n1 + kOpPadRows) * g.kpad / 8, di->sms), kSmallThreads, 0, s>>>(
+        static_cast<const uint16_t*>(D1), n1, d, w.q1, g.kpad, n1 + kOpPadRows, bf);
+    if ((r = launched()) != RNN_OK) return r;
+    op_copy_kernel<<<grid_for((n2 + kOpPadRows) * g.kpad / 8, di->sms), kSmallThreads, 0, s>>>(
+        static_cast<const uint16_t*>(D2), n2, d, w.q2, g.kpad, n2 + kOpPadRows, bf);
+    if ((r = launched()) != RNN_OK) return r;
+    if ((r = mnn_onepass(w.q1, n1, w.q2, n2, g.kpad, d, dtype, g, w, di, s)) != RNN_OK) return r;
+    mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2, w.counts, nblk1,
+                                                  rowarg_out, rowmax_out, colarg_out, colmax_out);
+    if ((r = launched()) != RNN_OK) return r;
+    mnn_write_kernel<<<nblk1, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, w.counts, nblk1,
+                                                     pairs_out, count_out);
+    return launched();
+  }
   // tensor maps and locate rows over the row forms, or over the inputs
   const uint16_t* Q1 = static_cast<const uint16_t*>(D1);
   const uint16_t* Q2 = static_cast<const uint16_t*>(D2);
@@ -1867,10 +2249,6 @@ rnn_status rnn_mnn_exhaustive_ex(const void* D1, int H1, int W1, const void* D2,
   if ((r = make_map(&m2, X2, ld, n2, 1, n2 * ld, g)) != RNN_OK) return r;
   if ((r = make_map(&q1, Q1, ld, n1, 1, n1 * ld, g, kBlockM)) != RNN_OK) return r;
   if ((r = make_map(&q2, Q2, ld, n2, 1, n2 * ld, g, kBlockM)) != RNN_OK) return r;
-
-  zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2,
-                                                                        w.err);
-  if ((r = launched()) != RNN_OK) return r;
   NNParams p;
   std::memset(&p, 0, sizeof(p));
   p.nfam = 2;
@@ -1901,7 +2279,6 @@ rnn_status rnn_mnn_exhaustive_ex(const void* D1, int H1, int W1, const void* D2,
                                                             X2, ld, d, l2);
     if ((r = launched()) != RNN_OK) return r;
   }
-  const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
   mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2, w.counts, nblk1,
                                                 rowarg_out, rowmax_out, colarg_out, colmax_out);
   if ((r = launched()) != RNN_OK) return r;
@@ -2399,18 +2776,25 @@ static __device__ __align__(256) unsigned char
 static std::mutex g_noalloc_mu;
 static void* g_noalloc_ptr[64];
 
-// Device address of the scratch array on the current device, looked up once
-// per device (host code only knows the array by a host-side stand-in name).
-static rnn_status noalloc_scratch(void** out) {
+// Device address of the scratch array on the current device (host code only
+// knows the array by a host-side stand-in name).  It is looked up with that
+// device current on every call whose stream is not being captured, so that a
+// context made anew after cudaDeviceReset gets its own address; a call on a
+// capturing stream uses the address the device's last such lookup found
+// (none yet: RNN_ECUDA).
+static rnn_status noalloc_scratch(cudaStream_t s, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RNN_ECUDA;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return RNN_ECUDA;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return RNN_ECUDA;
     g_noalloc_ptr[dev] = p;
   }
+  if (!g_noalloc_ptr[dev]) return RNN_ECUDA;
   *out = g_noalloc_ptr[dev];
   return RNN_OK;
 }
@@ -2423,10 +2807,27 @@ extern "C" rnn_status rnn_nn_argmax_noalloc(const void* Q, int64_t nq, const voi
   if (nq > RNN_NN_NOALLOC_MAX_QUERIES) return RNN_EUNSUPPORTED;
   if (nq < 0) return RNN_EINVAL;
   void* scratch = nullptr;
-  const rnn_status r = rnn::noalloc_scratch(&scratch);
+  const rnn_status r =
+      rnn::noalloc_scratch(reinterpret_cast<cudaStream_t>(stream), &scratch);
   if (r != RNN_OK) return r;
   static_assert(sizeof(rnn::g_noalloc_scratch) >= 256 + RNN_NN_NOALLOC_MAX_QUERIES * 8,
                 "scratch array too small");
   return rnn_nn_argmax(Q, nq, X, nx, d, dtype, idx_out, score_out, scratch,
                        sizeof(rnn::g_noalloc_scratch), stream);
+}
+
+// The status word of the shared scratch array (the first int, which every
+// call clears before its kernels run): RNN_ETIMEOUT when a bounded wait of the
+// last call ran out.  One 4-byte copy to the host and a synchronisation of
+// `stream`; nothing is allocated.
+extern "C" rnn_status rnn_nn_argmax_noalloc_status(rnn_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  rnn_status r = rnn::noalloc_scratch(s, &scratch);
+  if (r != RNN_OK) return r;
+  int err = 0;
+  if (cudaMemcpyAsync(&err, scratch, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return RNN_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RNN_ECUDA;
+  return err ? RNN_ETIMEOUT : RNN_OK;
 }

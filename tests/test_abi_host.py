@@ -59,9 +59,17 @@ def test_seed_counts_match_oracle(lib, H, W, S):
 def test_workspace_sizes(lib):
     assert lib.rnn_nn_workspace_size(1000) >= 1000 * 8
     assert lib.rnn_mnn_workspace_size(384, 512, 384, 512, 32) >= 2 * 384 * 512 * 8
-    # d = 24 is padded to 32: the workspace also holds both maps at 64 bytes a row
+    # d <= 32 (and d = 64) take the one-pass kernel, which reads copies of both
+    # maps padded to the K-block (d = 24 -> 32 channels, 64 bytes a row) with
+    # 2048 NaN rows past the last pixel
+    n = 384 * 512
     assert (lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24)
-            >= lib.rnn_mnn_workspace_size(384, 512, 384, 512, 32) + 2 * 384 * 512 * 64)
+            >= 2 * n * 8 + 2 * (n + 2048) * 64)
+    assert (lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24)
+            == lib.rnn_mnn_workspace_size(384, 512, 384, 512, 32))
+    # the Euclidean metric keeps the two-sweep form: a query and a candidate form per map
+    assert (lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, 1)
+            >= 2 * n * 8 + 4 * n * 64)
     one = lib.rnn_frm_workspace_size(1, 384, 512, 384, 512, 32, 8)
     many = lib.rnn_frm_workspace_size(64, 288, 512, 288, 512, 32, 8)
     assert one > 0 and many > 64 * 2304 * 8
@@ -140,9 +148,10 @@ def test_frm_argument_errors(lib):
 def test_ex_workspace_sizes(lib):
     dot = lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, _lib.RNN_DOT)
     assert dot == lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24)
-    # the Euclidean metric keeps a query and a candidate form of each map
+    # the Euclidean metric keeps a query and a candidate form of each map (the
+    # dot metric holds one padded copy of each, with a tail of 2048 rows)
     l2 = lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, _lib.RNN_L2)
-    assert l2 >= dot + 2 * 384 * 512 * 32 * 2
+    assert l2 >= dot + 2 * 384 * 512 * 32 * 2 - 2 * 2048 * 32 * 2
     assert lib.rnn_nn_workspace_size_ex(100, 5000, 24, _lib.RNN_DOT) == \
         lib.rnn_nn_workspace_size(100)
     assert lib.rnn_nn_workspace_size_ex(100, 5000, 24, _lib.RNN_L2) >= \
@@ -334,3 +343,16 @@ def test_frm_graph_binding_rejects_bad_maps(lib):
     with pytest.raises(RuntimeError):
         g.launch()
     g.close()                                 # closing it is a no-op
+
+
+def test_noalloc_scratch_holds_the_largest_call(lib):
+    """The no-allocation entry point passes its fixed array (256 + 8 *
+    RNN_NN_NOALLOC_MAX_QUERIES bytes) as the workspace of the ordinary call;
+    the workspace that call needs at the limit must fit in it.  Argument
+    errors come back before any device work."""
+    m = _lib.RNN_NN_NOALLOC_MAX_QUERIES
+    assert lib.rnn_nn_workspace_size(m) <= 256 + 8 * m
+    assert lib.rnn_nn_workspace_size_ex(m, 1 << 20, 64, _lib.RNN_DOT) <= 256 + 8 * m
+    call = lib.rnn_nn_argmax_noalloc
+    assert _lib.STATUS[call(FAKE, m + 1, FAKE, 4, 8, 0, FAKE, None, None)] == "RNN_EUNSUPPORTED"
+    assert _lib.STATUS[call(FAKE, -1, FAKE, 4, 8, 0, FAKE, None, None)] == "RNN_EINVAL"

@@ -67,3 +67,28 @@ def test_frm_wait_runs_out_and_is_reported():
     r = rnn.frm_match(dev(D1), dev(D2), 4, 3, workspace=ws)
     rnn.workspace_status(ws)
     assert np.array_equal(r.trimmed().cpu().numpy(), oracle.frm(D1, D2, 4, 3).pairs)
+
+
+def test_mnn_onepass_wait_runs_out_and_is_reported():
+    """The exhaustive set's one-pass kernel (d <= 32): its MMA warp's wait on
+    the first query tile runs out, every role of every CTA stops, and the
+    status reads RNN_ETIMEOUT; indices stay in range and the next call on the
+    same workspace is exact."""
+    rng = np.random.default_rng(202)
+    D1 = synth.to_storage(synth.quantised_map(rng, 40, 50, 24), "f16")
+    D2 = synth.to_storage(synth.quantised_map(rng, 30, 70, 24), "f16")
+    lib = rnn._lib.load()
+    ws = torch.empty(lib.rnn_mnn_workspace_size(40, 50, 30, 70, 24), dtype=torch.uint8,
+                     device="cuda")
+    r = _stalled(lambda: rnn.mnn_exhaustive(dev(D1), dev(D2), workspace=ws, with_nn=True))
+    with pytest.raises(rnn.RNNError) as e:
+        rnn.workspace_status(ws)
+    assert e.value.name == "RNN_ETIMEOUT"
+    ra, ca = r.rowarg.cpu().numpy(), r.colarg.cpu().numpy()
+    assert ra.min() >= 0 and ra.max() < 30 * 70 and ca.min() >= 0 and ca.max() < 40 * 50
+    r = rnn.mnn_exhaustive(dev(D1), dev(D2), workspace=ws, with_nn=True)
+    rnn.workspace_status(ws)
+    ref = oracle.mnn(D1, D2)
+    assert np.array_equal(r.rowarg.cpu().numpy(), ref.row.arg)
+    assert np.array_equal(r.colarg.cpu().numpy(), ref.col.arg)
+    assert np.array_equal(r.trimmed().cpu().numpy(), ref.pairs)
