@@ -416,19 +416,29 @@ rnn_status rnn_pts_frm_match(int B, const float *P1, int64_t p1_batch_stride, co
  * no allocator.
  *
  *   nq > RNN_NN_NOALLOC_MAX_QUERIES  -> RNN_EUNSUPPORTED (nothing launched).
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture.
+ *   The call looks up the array's device address with the caller's device
+ *   current (on a stream that is being captured it reuses the address the
+ *   device's last other call found, so make the first call on a device before
+ *   any stream capture).
  *   All calls share the one array, which keeps the last call's contents (each
  *   call clears what must start at zero): calls that overlap on the GPU, on
  *   any streams, race and give undefined results.  Serialise them.
- *   rnn_workspace_status() does not apply; a timed-out wait shows as an
- *   undefined result only.
+ *   rnn_workspace_status() does not apply: rnn_nn_argmax_noalloc_status()
+ *   reads the array's status word instead.
  */
 #define RNN_NN_NOALLOC_MAX_QUERIES 65536
 rnn_status rnn_nn_argmax_noalloc(const void *Q, int64_t nq, const void *X, int64_t nx, int d,
                                  rnn_dtype dtype, int32_t *idx_out, float *score_out,
                                  rnn_stream_t stream);
+
+/* Status of the last rnn_nn_argmax_noalloc call on the current device:
+ * RNN_ETIMEOUT if one of its bounded device-side waits ran out (its indices
+ * are then undefined, though in range), else RNN_OK.  Reads the status word
+ * of the shared array (4 bytes to the host) and synchronises `stream`; it
+ * allocates nothing.  Like the call itself, this has no counterpart on the
+ * source pages.
+ *   RNN_ECUDA  -> the copy or the synchronisation failed. */
+rnn_status rnn_nn_argmax_noalloc_status(rnn_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Diagnostics for benchmarking (no effect on results).

@@ -28,6 +28,7 @@ EXPORTS = (
     "rnn_launch_count",
     "rnn_set_kernel_timer",
     "rnn_nn_argmax_noalloc",
+    "rnn_nn_argmax_noalloc_status",
     "rnn_nn_workspace_size_ex",
     "rnn_nn_argmax_ex",
     "rnn_mnn_workspace_size_ex",
@@ -108,6 +109,7 @@ def load():
         "rnn_launch_count": (ctypes.c_uint64, []),
         "rnn_set_kernel_timer": (None, [P, P, I, P]),
         "rnn_nn_argmax_noalloc": (I, [P, I64, P, I64, I, I, P, P, P]),
+        "rnn_nn_argmax_noalloc_status": (I, [P]),
         "rnn_nn_workspace_size_ex": (SZ, [I64, I64, I, I]),
         "rnn_nn_argmax_ex": (I, [P, I64, P, I64, I, I, I, P, P, P, SZ, P]),
         "rnn_mnn_workspace_size_ex": (SZ, [I, I, I, I, I, I]),
