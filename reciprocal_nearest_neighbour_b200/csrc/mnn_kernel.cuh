@@ -42,27 +42,30 @@
 // maxima with a strict '>' in increasing order, so the kept chunk is the
 // first that holds the maximum.
 //
-// Warp roles (18 warps):
+// Warp roles (19 warps):
 //   warp 0       TMA producer: the bm query tiles of a unit (four 32-row
 //                boxes each) once per unit, the candidate tile once per n-tile
-//   warp 1       MMA issuer (one warp: every commit then covers every MMA
-//                that read a shared-memory slot before it is refilled)
-//   warps 2..17  epilogue, quadrant q = warp % 4, part p = (warp - 2) / 4
+//   warps 1-2    MMA issuers, one per accumulator (tile l of an n-pass uses
+//                accumulator l % 2).  Each waits for its own accumulator, so
+//                the two turnarounds (commit, wake-up, release, re-issue)
+//                overlap.  A shared-memory slot is refilled once both warps
+//                have committed after its last reader; that is safe while a
+//                slot's reuse period is at least 5 tiles (a warp can run at
+//                most 4 tiles ahead of the other), so small units use warp 1
+//                alone (nmma = 1).
+//   warps 3..18  epilogue, quadrant q = warp % 4, part p = (warp - 3) / 4
 #pragma once
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include "nn_kernel.cuh"
 #include "ptx.cuh"
 
-#ifndef RNN_OP_PIPE
-#define RNN_OP_PIPE 0
-#endif
-
 namespace rnn {
 
-constexpr int kOpEpiWarp0 = 2;
+constexpr int kOpEpiWarp0 = 3;
 constexpr int kOpEpiWarps = 16;
-constexpr int kOpThreads = (kOpEpiWarp0 + kOpEpiWarps) * 32;  // 576
+constexpr int kOpThreads = (kOpEpiWarp0 + kOpEpiWarps) * 32;  // 608
 constexpr int kOpBlockN = 256;
 constexpr int kOpMaxBm = 16;      // query tiles a unit holds in shared memory
 constexpr int kOpMaxBn = 8;       // candidate tiles per unit (row chunk ids are bytes)
@@ -71,7 +74,8 @@ constexpr int kOpRowChunk = 64;   // columns of a row chunk (one epilogue warp's
 struct OnePassParams {
   int n1, n2;            // image-1 rows (tensor-memory lanes), image-2 rows (columns)
   int kpad;              // K of the tiles: 16, 32 or 64 (one K-block, swizzle 2*kpad bytes)
-  int bm, bn;            // m-tiles and n-tiles of a unit
+  int bm, bn;            // m-tiles (a power of two) and n-tiles of a unit
+  int nmma;              // MMA-issuing warps: 2, or 1 for small units
   int mblocks, nblocks;  // units = mblocks * nblocks; unit u -> (u % mblocks, u / mblocks)
   uint32_t idesc;
   unsigned long long* rowk;  // [n1] (score, first column of the row chunk), atomicMax
@@ -97,10 +101,27 @@ __host__ __device__ inline OnePassSmem onepass_smem(int kpad, int bm) {
   s.colred_off = (s.rchunk_off + static_cast<uint32_t>(bm) * 4u * 128u + 15u) & ~15u;
   s.bar_off = s.colred_off + 2u * 4u * 256u * 4u;                   // float [2][4][256]
   // a_full[16], a_empty[16], b_full[2], b_empty[2], acc_full[2], acc_empty[2],
-  // colbar[4], rowbar, drain
-  s.misc_off = s.bar_off + (2u * kOpMaxBm + 14u) * 8u;
+  // colbar[4], rowbar, drain[2]
+  s.misc_off = s.bar_off + (2u * kOpMaxBm + 15u) * 8u;
   s.total = s.misc_off + 16u;
   return s;
+}
+
+// Row state of one (m-tile, row, part) slot: the best score over the
+// n-tiles so far and the first n-tile that reached it.  At n = 0 the slot is
+// written whatever it held (also when y is NaN: a part wholly past the last
+// image-2 row); later a strictly larger y replaces it.  Branch-free.
+__device__ __forceinline__ void row_state_update(uint32_t slot, uint32_t cslot, float y, int n) {
+  asm volatile(
+      "{\n\t.reg .pred p, z;\n\t.reg .f32 o;\n\t"
+      "ld.shared.f32 o, [%0];\n\t"
+      "setp.gt.f32 p, %2, o;\n\t"
+      "setp.eq.s32 z, %3, 0;\n\t"
+      "or.pred p, p, z;\n\t"
+      "@p st.shared.f32 [%0], %2;\n\t"
+      "@p st.shared.u8 [%1], %3;\n\t}" ::"r"(slot),
+      "r"(cslot), "f"(y), "r"(n)
+      : "memory");
 }
 
 // Keep one of two values and send the other to the partner lane `mask`
@@ -134,7 +155,7 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* colbar = acc_empty + 2;
   uint64_t* rowbar = colbar + 4;
-  uint64_t* drain_bar = rowbar + 1;
+  uint64_t* drain_bar = rowbar + 1;  // [2], one per MMA warp
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
@@ -147,17 +168,18 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
   if (threadIdx.x == 0) {
     for (int l = 0; l < bm; ++l) {
       mbar_init(smem_u32(&a_full[l]), 1);
-      mbar_init(smem_u32(&a_empty[l]), 1);
+      mbar_init(smem_u32(&a_empty[l]), p.nmma);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&b_full[i]), 1);
-      mbar_init(smem_u32(&b_empty[i]), 1);
+      mbar_init(smem_u32(&b_empty[i]), p.nmma);
       mbar_init(smem_u32(&acc_full[i]), 1);
       mbar_init(smem_u32(&acc_empty[i]), kOpEpiWarps);
     }
     for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&colbar[i]), 4);
     mbar_init(smem_u32(rowbar), kOpEpiWarps);
-    mbar_init(smem_u32(drain_bar), 1);
+    mbar_init(smem_u32(&drain_bar[0]), 1);
+    mbar_init(smem_u32(&drain_bar[1]), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -242,11 +264,13 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    long long T = 0, b_cnt = 0;
+  } else if (warp <= 2) {
+    // ------------------------------------------------------ MMA issuers
+    const int mw = warp - 1;
+    long long b_cnt = 0;
     int a_it = 0;
-    bool ok = true, any = false;
+    uint32_t ph = 0;  // phase of this warp's accumulator's next use (bit per accumulator)
+    bool ok = mw < p.nmma, any = false;
     const uint64_t a_desc0 = make_sdesc(smem_u32(a_tiles), p.kpad);
     const uint64_t b_desc0 = make_sdesc(smem_u32(b_tiles), p.kpad);
     const uint32_t a_step = a_bytes >> 4, b_step = b_bytes >> 4;
@@ -256,37 +280,42 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
       for (int n = 0; n < bn && ok; ++n, ++b_cnt) {
         const int bs = static_cast<int>(b_cnt & 1);
         const uint32_t bpar = static_cast<uint32_t>((b_cnt >> 1) & 1);
-        for (int l = 0; l < bm; ++l, ++T) {
-          const int acc = static_cast<int>(T & 1);
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(smem_u32(&a_full[l]), static_cast<uint32_t>(a_it & 1),
-                                    abort_flag, p.err, kErrWaitMma, lim) &&
-                              mbar_wait(smem_u32(&b_full[bs]), bpar, abort_flag, p.err,
-                                        kErrWaitMma, lim) &&
-                              mbar_wait_sleep(smem_u32(&acc_empty[acc]),
-                                              static_cast<uint32_t>((T >> 1) & 1) ^ 1u,
-                                              abort_flag, p.err, kErrWaitMma, lim));
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kOpBlockN);
-          const uint64_t a = a_desc0 + static_cast<uint64_t>(l) * a_step;
-          const uint64_t b = b_desc0 + static_cast<uint64_t>(bs) * b_step;
-          for (int k = 0; k < ksteps; ++k)
-            umma_f16_warp(d_tmem, a + 2 * k, b + 2 * k, idesc, k > 0 ? 1u : 0u);
-          umma_commit_warp(smem_u32(&acc_full[acc]));
-          if (n == bn - 1) umma_commit_warp(smem_u32(&a_empty[l]));  // last read of slot l
-          if (l == bm - 1) umma_commit_warp(smem_u32(&b_empty[bs]));  // last read of slot bs
+        for (int l = 0; l < bm; ++l) {
+          const int acc = l & 1;
+          if (p.nmma == 1 || acc == mw) {
+            const uint32_t aph = (ph >> acc) & 1u;
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&a_full[l]), static_cast<uint32_t>(a_it & 1),
+                                      abort_flag, p.err, kErrWaitMma, lim) &&
+                                mbar_wait(smem_u32(&b_full[bs]), bpar, abort_flag, p.err,
+                                          kErrWaitMma, lim) &&
+                                mbar_wait_sleep(smem_u32(&acc_empty[acc]), aph ^ 1u, abort_flag,
+                                                p.err, kErrWaitMma, lim));
+            if (!ok) break;
+            ph ^= 1u << acc;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kOpBlockN);
+            const uint64_t a = a_desc0 + static_cast<uint64_t>(l) * a_step;
+            const uint64_t b = b_desc0 + static_cast<uint64_t>(bs) * b_step;
+            for (int k = 0; k < ksteps; ++k)
+              umma_f16_warp(d_tmem, a + 2 * k, b + 2 * k, idesc, k > 0 ? 1u : 0u);
+            umma_commit_warp(smem_u32(&acc_full[acc]));
+            any = true;
+          }
+          // every MMA warp commits after the last reader of a slot (each
+          // commit covers that warp's MMAs so far)
+          if (n == bn - 1) umma_commit_warp(smem_u32(&a_empty[l]));
+          if (l == bm - 1) umma_commit_warp(smem_u32(&b_empty[bs]));
           __syncwarp();
-          any = true;
         }
       }
     }
-    if (!ok && any) {
-      // let every MMA issued finish before tensor memory is released
-      umma_commit_warp(smem_u32(drain_bar));
+    if (mw < p.nmma && !ok && any) {
+      // let every MMA this warp issued finish before tensor memory is released
+      umma_commit_warp(smem_u32(&drain_bar[mw]));
       __syncwarp();
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(drain_bar), 0)) {
+      while (!mbar_try_wait(smem_u32(&drain_bar[mw]), 0)) {
         if (globaltimer_ns() - t0 > lim) {
           if (lane == 0) atomicOr(p.err, kErrDrain);
           break;
@@ -301,121 +330,78 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
     const int g = lane >> 2, s = lane & 3;
     const bool s0 = (lane & 1) != 0, s1 = (lane & 2) != 0;
     const bool g0 = (lane & 4) != 0, g1 = (lane & 8) != 0, g2 = (lane & 16) != 0;
+    const bool lane0 = lane == 0;
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                         static_cast<uint32_t>(64 * part);
     // this lane's row-state slot: row 32q + g + 8s of part `part`, per m-tile l
     const int rslot = part * 128 + 32 * q + g + 8 * s;
     const uint32_t rb_s = smem_u32(rbest) + 4u * rslot, rc_s = smem_u32(rchunk) + rslot;
     const uint32_t cr_s = smem_u32(colred);
+    const uint32_t full0 = smem_u32(&acc_full[0]), full1 = smem_u32(&acc_full[1]);
+    const uint32_t empty0 = smem_u32(&acc_empty[0]), empty1 = smem_u32(&acc_empty[1]);
     const float ninf = -__int_as_float(0x7f800000);
-    uint32_t T = 0;  // tile sequence of this CTA (only its two low bits are used)
+    uint32_t eph = 0;  // bit a: phase of accumulator a's next result
     int flushes = 0, rowphase = 0;
     bool ok = true;
-    // Software pipeline over the tiles of this CTA: each tile is read in two
-    // halves (rows g, g+8 into va; rows g+16, g+24 into vb).  The read of vb
-    // runs while va is folded, and the read of the next tile's va runs while
-    // vb is folded, so the tensor-memory latency hides behind the folds with
-    // 64 value registers.  `pend`: va's read for tile T is already issued.
-    float va[32], vb[32];
-    bool pend = false;
-#if !RNN_OP_PIPE
-    constexpr bool kPipe = false;
-#else
-    constexpr bool kPipe = true;
-#endif
+    float pm[16];      // running maxima of this thread's 16 columns over its rows
+
+    // One tile (query tile l of the n-pass, candidate tile n) in accumulator
+    // kAcc: read the 4 x 16 block (rows g, g+8 into va, rows g+16, g+24 into
+    // vb), hand the accumulator back, fold it.
+    auto tile = [&](auto acc_c, int l, int n) -> bool {
+      constexpr int kAcc = decltype(acc_c)::value;
+      if (!mbar_wait_sleep(kAcc ? full1 : full0, (eph >> kAcc) & 1u, abort_flag, p.err,
+                           kErrWaitEpilogue, lim))
+        return false;
+      eph ^= 1u << kAcc;
+      tc_fence_after();
+      float va[32], vb[32];
+      const uint32_t ta = tq + static_cast<uint32_t>(kAcc * kOpBlockN);
+      tmem_ld16x256_x8(ta, va);
+      tmem_ld16x256_x8(ta + (16u << 16), vb);
+      tmem_wait_ld_regs(va);
+      reg_fence(vb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane0) mbar_arrive(kAcc ? empty1 : empty0);
+      reg_fence(va);
+      reg_fence(vb);
+      // columns: two three-input maxima per column; rows: one chain per row
+      float r0 = fmaxf(va[0], va[1]), r1 = fmaxf(va[2], va[3]);
+      float r2 = fmaxf(vb[0], vb[1]), r3 = fmaxf(vb[2], vb[3]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          pm[2 * j + h] = fmax3(pm[2 * j + h], va[4 * j + h], va[4 * j + 2 + h]);
+          pm[2 * j + h] = fmax3(pm[2 * j + h], vb[4 * j + h], vb[4 * j + 2 + h]);
+        }
+        if (j > 0) {
+          r0 = fmax3(r0, va[4 * j], va[4 * j + 1]);
+          r1 = fmax3(r1, va[4 * j + 2], va[4 * j + 3]);
+          r2 = fmax3(r2, vb[4 * j], vb[4 * j + 1]);
+          r3 = fmax3(r3, vb[4 * j + 2], vb[4 * j + 3]);
+        }
+      }
+      // across the 4 lanes holding the same rows: lane s ends with row g + 8s
+      const float x0 = swap_max(r0, r1, s0, 1);  // row (s & 1)
+      const float x1 = swap_max(r2, r3, s0, 1);  // row 2 + (s & 1)
+      const float y = swap_max(x0, x1, s1, 2);   // row s
+      row_state_update(rb_s + 2048u * l, rc_s + 512u * l, y, n);
+      return true;
+    };
+
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int mb = u % p.mblocks, nb = u / p.mblocks;
       const int row_base = mb * 128 * bm;
       for (int n = 0; n < bn && ok; ++n) {
         const int col0 = (nb * bn + n) * kOpBlockN + 64 * part;  // first column of this part
-        float pm[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) pm[c] = ninf;
-        for (int l = 0; l < bm; ++l, ++T) {
-          const uint32_t ta = tq + static_cast<uint32_t>((T & 1u) * kOpBlockN);
-          if (!pend) {
-            if (!mbar_wait_sleep(smem_u32(&acc_full[T & 1u]), (T >> 1) & 1u, abort_flag, p.err,
-                                 kErrWaitEpilogue, lim)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            tmem_ld16x256_x8(ta, va);
-          }
-          if (!kPipe) tmem_ld16x256_x8(ta + (16u << 16), vb);
-          tmem_wait_ld_regs(va);
-          if (!kPipe) {
-            reg_fence(vb);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[T & 1u]));
-          } else {
-            tmem_ld16x256_x8(ta + (16u << 16), vb);
-          }
-          reg_fence(va);
-          // first half: columns over rows g, g+8; rows g and g+8 over this thread's 16 columns
-          // (column by column, so that each group of four values dies early)
-          float r0 = fmaxf(va[0], va[1]), r1 = fmaxf(va[2], va[3]);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              pm[2 * j + h] = fmax3(pm[2 * j + h], va[4 * j + h], va[4 * j + 2 + h]);
-            if (j > 0) {
-              r0 = fmax3(r0, va[4 * j], va[4 * j + 1]);
-              r1 = fmax3(r1, va[4 * j + 2], va[4 * j + 3]);
-            }
-          }
-          // the first half's folds before the wait for the second half
-#pragma unroll
-          for (int c = 0; c < 16; ++c) keep_order(pm[c]);
-          keep_order(r0);
-          keep_order(r1);
-          if (kPipe) {
-            tmem_wait_ld_regs(vb);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[T & 1u]));
-          }
-          // the next tile's first half, read during this tile's second fold
-          // (within the candidate tile: its column flush comes first)
-          pend = false;
-          if (kPipe && l != bm - 1) {
-            const uint32_t T1 = T + 1u;
-            if (!mbar_wait_sleep(smem_u32(&acc_full[T1 & 1u]), (T1 >> 1) & 1u, abort_flag, p.err,
-                                 kErrWaitEpilogue, lim)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            tmem_ld16x256_x8(tq + static_cast<uint32_t>((T1 & 1u) * kOpBlockN), va);
-            pend = true;
-          }
-          reg_fence(vb);
-          // second half: rows g+16, g+24
-          float r2 = fmaxf(vb[0], vb[1]), r3 = fmaxf(vb[2], vb[3]);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              pm[2 * j + h] = fmax3(pm[2 * j + h], vb[4 * j + h], vb[4 * j + 2 + h]);
-            if (j > 0) {
-              r2 = fmax3(r2, vb[4 * j], vb[4 * j + 1]);
-              r3 = fmax3(r3, vb[4 * j + 2], vb[4 * j + 3]);
-            }
-          }
-          // across the 4 lanes holding the same rows: lane s ends with row g + 8s
-          const float x0 = swap_max(r0, r1, s0, 1);  // row (s & 1)
-          const float x1 = swap_max(r2, r3, s0, 1);  // row 2 + (s & 1)
-          const float y = swap_max(x0, x1, s1, 2);   // row s
-          const uint32_t slot = rb_s + 2048u * l, cslot = rc_s + 512u * l;
-          if (n == 0) {
-            sts_f32(slot, y);
-            sts_u8(cslot, 0u);
-          } else if (y > lds_f32(slot)) {
-            sts_f32(slot, y);
-            sts_u8(cslot, static_cast<uint32_t>(n));
-          }
+        // tile l of an n-pass uses accumulator l % 2 (bm is a power of two)
+        for (int l = 0; l < bm && ok; l += 2) {
+          ok = tile(std::integral_constant<int, 0>{}, l, n);
+          if (ok && l + 1 < bm) ok = tile(std::integral_constant<int, 1>{}, l + 1, n);
         }
         if (!ok) break;
         // ---- column flush: over the 8 lanes of this quadrant holding the same columns
@@ -487,9 +473,6 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
       }
       ++rowphase;
     }
-    // an abort after the next tile's read was issued: let it land before the
-    // tensor memory is released
-    if (pend) tmem_wait_ld();
   }
 
   tc_fence_before();

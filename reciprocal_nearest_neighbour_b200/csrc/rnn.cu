@@ -2043,24 +2043,29 @@ size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2, int d) {
 
 // ---------------------------------------------------- one-pass exhaustive M
 struct OnePassPlan {
-  int bm, bn, mblocks, nblocks;
+  int bm, bn, mblocks, nblocks, nmma;
 };
 
 // Unit shape: the largest that shared memory holds (bm query tiles of
-// 128 x kpad, 8 candidate tiles), halved along the longer side until there
-// are at least two units per SM.
+// 128 x kpad, bm a power of two; 8 candidate tiles), halved along the longer
+// side until there are at least two units per SM.  Two MMA-issuing warps when
+// every shared-memory slot's reuse period is at least 5 tiles (2*bm for a
+// candidate slot, bm*bn for a query slot).
 static OnePassPlan onepass_plan(int64_t n1, int64_t n2, int kpad, int sms) {
   const int mt = static_cast<int>((n1 + 127) / 128);
   const int nt = static_cast<int>((n2 + kOpBlockN - 1) / kOpBlockN);
   auto blocks = [](int t, int b) { return (t + b - 1) / b; };
-  int bm = std::min(kpad == 64 ? 8 : kOpMaxBm, mt), bn = std::min(kOpMaxBn, nt);
+  int bm = kpad == 64 ? 8 : kOpMaxBm;
+  while (bm > 1 && bm > mt) bm >>= 1;
+  int bn = std::min(kOpMaxBn, nt);
   while (static_cast<int64_t>(blocks(mt, bm)) * blocks(nt, bn) < 2LL * sms && (bm > 1 || bn > 1)) {
     if (bn >= bm && bn > 1)
       bn = (bn + 1) / 2;
     else
-      bm = (bm + 1) / 2;
+      bm >>= 1;
   }
-  return {bm, bn, blocks(mt, bm), blocks(nt, bn)};
+  const int nmma = (bm >= 4 && bm * bn >= 8) ? 2 : 1;
+  return {bm, bn, blocks(mt, bm), blocks(nt, bn), nmma};
 }
 
 template <bool kBf16>
@@ -2121,6 +2126,7 @@ static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2
   p.bn = pl.bn;
   p.mblocks = pl.mblocks;
   p.nblocks = pl.nblocks;
+  p.nmma = pl.nmma;
   p.idesc = make_idesc(dtype, kOpBlockN);
   p.rowk = w.rowk;
   p.colk = w.colk;
