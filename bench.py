@@ -770,6 +770,22 @@ def run_nn_case(nq, d, nx):
     return 0
 
 
+def run_mnn_case(mode):
+    """The exhaustive set at 512x384, d=24 three times (for an ncu capture of
+    the one-pass kernel): mode "q" quantised maps, "f" unit-norm fp16 maps."""
+    import torch
+    import reciprocal_nearest_neighbour_b200 as rnn
+    from reciprocal_nearest_neighbour_b200 import synth
+    w = synth.WORKLOADS["mnn_512x384_q" if mode == "q" else "mnn_512x384_f"]
+    a, b = synth.make_workload_storage(w, "f16", pairs=[0])
+    a, b = a[0].cuda(), b[0].cuda()
+    for _ in range(3):
+        r = rnn.mnn_exhaustive(a, b)
+    torch.cuda.synchronize()
+    print(f"mnn-case {w.name}: |M| = {int(r.count.item())}")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -788,7 +804,12 @@ def main(argv=None):
     ap.add_argument("--nn-case", type=int, nargs=3, metavar=("NQ", "D", "NX"),
                     help="profiling aid: run nn_argmax three times on seeded fp16 "
                          "queries/candidates of these sizes and exit (no timing)")
+    ap.add_argument("--mnn-case", choices=["q", "f"],
+                    help="profiling aid: run the 512x384 exhaustive set three times on the "
+                         "quantised (q) or fp16 (f) maps and exit (no timing)")
     args = ap.parse_args(argv)
+    if args.mnn_case:
+        return run_mnn_case(args.mnn_case)
     if args.leg:
         return run_leg(args.leg, args.steps, args.warmup)
     if args.nn_case:

@@ -17,8 +17,9 @@
 // Loop order.  A work unit is bm m-tiles (image-1 rows) x bn n-tiles (image-2
 // rows).  For each n-tile, the m-tiles go by in the inner loop, so every
 // thread keeps the running maximum of its 16 columns in registers over the
-// whole inner loop (two three-input maxima per column and tile) and merges
-// across lanes and quadrants once per n-tile.  Row partials (one per row and
+// whole inner loop (two three-input maxima per column and tile), merges
+// them across its 8 lanes once per n-tile and writes them to the global keys
+// with atomicMax (one chunk per quadrant, so no meeting between warps).  Row partials (one per row and
 // 64-column part, after a two-step shuffle across 4 lanes) go to shared
 // memory, where each (m-tile, row, part) slot keeps the best over the n-tiles
 // with the first n-tile that reached it; they are merged and written once
@@ -87,7 +88,7 @@ struct OnePassParams {
 
 // Shared-memory layout, offsets from the 1024-byte aligned base.
 struct OnePassSmem {
-  uint32_t a_off, b_off, rbest_off, rchunk_off, colred_off, bar_off, misc_off, total;
+  uint32_t a_off, b_off, rbest_off, rchunk_off, bar_off, misc_off, total;
 };
 
 __host__ __device__ inline OnePassSmem onepass_smem(int kpad, int bm) {
@@ -98,11 +99,10 @@ __host__ __device__ inline OnePassSmem onepass_smem(int kpad, int bm) {
   s.b_off = s.a_off + static_cast<uint32_t>(bm) * a_bytes;
   s.rbest_off = s.b_off + 2u * b_bytes;                             // float [bm][4][128]
   s.rchunk_off = s.rbest_off + static_cast<uint32_t>(bm) * 4u * 128u * 4u;  // u8 [bm][4][128]
-  s.colred_off = (s.rchunk_off + static_cast<uint32_t>(bm) * 4u * 128u + 15u) & ~15u;
-  s.bar_off = s.colred_off + 2u * 4u * 256u * 4u;                   // float [2][4][256]
+  s.bar_off = (s.rchunk_off + static_cast<uint32_t>(bm) * 4u * 128u + 15u) & ~15u;
   // a_full[16], a_empty[16], b_full[2], b_empty[2], acc_full[2], acc_empty[2],
-  // colbar[4], rowbar, drain[2]
-  s.misc_off = s.bar_off + (2u * kOpMaxBm + 15u) * 8u;
+  // rowbar, drain[2]
+  s.misc_off = s.bar_off + (2u * kOpMaxBm + 11u) * 8u;
   s.total = s.misc_off + 16u;
   return s;
 }
@@ -145,7 +145,6 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
   uint8_t* b_tiles = smem + L.b_off;
   float* rbest = reinterpret_cast<float*>(smem + L.rbest_off);
   uint8_t* rchunk = smem + L.rchunk_off;
-  float* colred = reinterpret_cast<float*>(smem + L.colred_off);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + kOpMaxBm;
@@ -153,8 +152,7 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
   uint64_t* b_empty = b_full + 2;
   uint64_t* acc_full = b_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* colbar = acc_empty + 2;
-  uint64_t* rowbar = colbar + 4;
+  uint64_t* rowbar = acc_empty + 2;
   uint64_t* drain_bar = rowbar + 1;  // [2], one per MMA warp
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -176,7 +174,6 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
       mbar_init(smem_u32(&acc_full[i]), 1);
       mbar_init(smem_u32(&acc_empty[i]), kOpEpiWarps);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&colbar[i]), 4);
     mbar_init(smem_u32(rowbar), kOpEpiWarps);
     mbar_init(smem_u32(&drain_bar[0]), 1);
     mbar_init(smem_u32(&drain_bar[1]), 1);
@@ -280,18 +277,25 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
       for (int n = 0; n < bn && ok; ++n, ++b_cnt) {
         const int bs = static_cast<int>(b_cnt & 1);
         const uint32_t bpar = static_cast<uint32_t>((b_cnt >> 1) & 1);
+        bool b_seen = false;  // this warp has seen the candidate tile of this pass land
         for (int l = 0; l < bm; ++l) {
           const int acc = l & 1;
           if (p.nmma == 1 || acc == mw) {
             const uint32_t aph = (ph >> acc) & 1u;
+            // a query slot lands once per unit (this warp's slots are the same
+            // in every pass: bm is even when two warps issue), the candidate
+            // tile once per pass
             ok = __all_sync(0xffffffffu,
-                            mbar_wait(smem_u32(&a_full[l]), static_cast<uint32_t>(a_it & 1),
-                                      abort_flag, p.err, kErrWaitMma, lim) &&
-                                mbar_wait(smem_u32(&b_full[bs]), bpar, abort_flag, p.err,
-                                          kErrWaitMma, lim) &&
+                            (n > 0 || mbar_wait_sleep(smem_u32(&a_full[l]),
+                                                      static_cast<uint32_t>(a_it & 1),
+                                                      abort_flag, p.err, kErrWaitMma, lim)) &&
+                                (b_seen || mbar_wait_sleep(smem_u32(&b_full[bs]), bpar,
+                                                           abort_flag, p.err, kErrWaitMma,
+                                                           lim)) &&
                                 mbar_wait_sleep(smem_u32(&acc_empty[acc]), aph ^ 1u, abort_flag,
                                                 p.err, kErrWaitMma, lim));
             if (!ok) break;
+            b_seen = true;
             ph ^= 1u << acc;
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kOpBlockN);
@@ -336,12 +340,11 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
     // this lane's row-state slot: row 32q + g + 8s of part `part`, per m-tile l
     const int rslot = part * 128 + 32 * q + g + 8 * s;
     const uint32_t rb_s = smem_u32(rbest) + 4u * rslot, rc_s = smem_u32(rchunk) + rslot;
-    const uint32_t cr_s = smem_u32(colred);
     const uint32_t full0 = smem_u32(&acc_full[0]), full1 = smem_u32(&acc_full[1]);
     const uint32_t empty0 = smem_u32(&acc_empty[0]), empty1 = smem_u32(&acc_empty[1]);
     const float ninf = -__int_as_float(0x7f800000);
     uint32_t eph = 0;  // bit a: phase of accumulator a's next result
-    int flushes = 0, rowphase = 0;
+    int rowphase = 0;
     bool ok = true;
     float pm[16];      // running maxima of this thread's 16 columns over its rows
 
@@ -412,32 +415,17 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
         for (int i = 0; i < 4; ++i) y4[i] = swap_max(x[i], x[i + 4], g1, 8);
 #pragma unroll
         for (int i = 0; i < 2; ++i) z[i] = swap_max(y4[i], y4[i + 2], g0, 4);
-        // z[h]: column 8g + 2s + h of this part, over the quadrant's 32*bm rows
-        const uint32_t cr = cr_s + 4096u * (flushes & 1);
-        sts_v2f32(cr + 4u * (q * 256 + 64 * part + 8 * g + 2 * s), z[0], z[1]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&colbar[part]));
-        if (!mbar_wait(smem_u32(&colbar[part]), static_cast<uint32_t>(flushes & 1), abort_flag,
-                       p.err, kErrWaitEpilogue, lim)) {
-          ok = false;
-          break;
+        // z[h]: column 8g + 2s + h of this part, over the quadrant's 32*bm rows:
+        // the chunk (m-block, quadrant).  Each warp merges its own maxima into
+        // the global keys (no meeting with the other quadrants' warps); a
+        // quadrant wholly past the last image-1 row holds NaN and is skipped.
+        {
+          const int c = col0 + 8 * g + 2 * s;
+          const int chunk_row = row_base + 32 * bm * q;
+          if (c < p.n2 && z[0] == z[0]) atomicMax(p.colk + c, pack_key(z[0], chunk_row));
+          if (c + 1 < p.n2 && z[1] == z[1])
+            atomicMax(p.colk + c + 1, pack_key(z[1], chunk_row));
         }
-        if (lane < 16) {
-          const int c = 16 * q + lane;  // this warp's share of the part's columns
-          float best = lds_f32(cr + 4u * (64 * part + c));
-          int bq = 0;
-#pragma unroll
-          for (int qq = 1; qq < 4; ++qq) {
-            const float v = lds_f32(cr + 4u * (qq * 256 + 64 * part + c));
-            if (v > best) {
-              best = v;
-              bq = qq;
-            }
-          }
-          if (col0 + c < p.n2)
-            atomicMax(p.colk + col0 + c, pack_key(best, row_base + 32 * bm * bq));
-        }
-        ++flushes;
       }
       if (!ok) break;
       // ---- row flush: every epilogue warp has written its slots for this unit
