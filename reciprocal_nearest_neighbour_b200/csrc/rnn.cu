@@ -752,7 +752,10 @@ __global__ void mutual_write_kernel(const int32_t* rowarg, int64_t n1, const int
 // shared memory and serve all of its queries.  Four launches: count per
 // chunk, scan, scatter of the query ids, and the resolve over items of at
 // most kLocItem queries of one chunk.
-constexpr int kLocItem = 256;
+constexpr int kLocItem = 64;     // queries per item of the resolve
+constexpr int kLocSlices = 4;    // candidate slices per item (one thread each per query)
+constexpr int kLocPad = 8;       // ints between counters: one 32-byte sector each, so that
+                                 // the atomics on different chunks do not queue on one line
 
 struct LocParams {
   unsigned long long* rowk;  // [n1] row keys, chunks of lr columns (image 2)
@@ -760,10 +763,10 @@ struct LocParams {
   int64_t n1, n2;
   int lr, lc;
   int nch_r, nch;            // row chunks; all chunks (row chunks first)
-  int* cnt;                  // [nch] queries per chunk
+  int* cnt;                  // [nch * kLocPad] queries per chunk (padded stride)
   int* start;                // [nch + 1] first list position of each chunk
   int* items;                // [nch + 1] first item of each chunk
-  int* cursor;               // [nch] fill counters of the scatter
+  int* cursor;               // [nch * kLocPad] fill counters of the scatter (padded stride)
   uint32_t* list;            // [n1 + n2] query ids: image-1 row i, or n1 + image-2 row j
   const uint16_t* X1;        // rows of image 1 and image 2, ld elements apart
   const uint16_t* X2;
@@ -816,9 +819,7 @@ __global__ void loc_count_kernel(LocParams P) {
   const int64_t n = P.n1 + P.n2, stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += stride) {
-    const int c = loc_chunk(P, i);
-    const unsigned m = __match_any_sync(__activemask(), c);
-    if ((threadIdx.x & 31) == __ffs(m) - 1) atomicAdd(P.cnt + c, __popc(m));
+    atomicAdd(P.cnt + kLocPad * loc_chunk(P, i), 1);
   }
 }
 
@@ -831,8 +832,8 @@ __global__ void loc_scan_kernel(LocParams P) {
   for (int k = 0; k < per; ++k) {
     const int c = b0 + k;
     if (c < n) {
-      sc += P.cnt[c];
-      si += (P.cnt[c] + kLocItem - 1) / kLocItem;
+      sc += P.cnt[kLocPad * c];
+      si += (P.cnt[kLocPad * c] + kLocItem - 1) / kLocItem;
     }
   }
   int tc, ti;
@@ -841,11 +842,12 @@ __global__ void loc_scan_kernel(LocParams P) {
   for (int k = 0; k < per; ++k) {
     const int c = b0 + k;
     if (c < n) {
+      const int k = P.cnt[kLocPad * c];
       P.start[c] = oc;
       P.items[c] = oi;
-      P.cursor[c] = 0;
-      oc += P.cnt[c];
-      oi += (P.cnt[c] + kLocItem - 1) / kLocItem;
+      P.cursor[kLocPad * c] = 0;
+      oc += k;
+      oi += (k + kLocItem - 1) / kLocItem;
     }
   }
   if (threadIdx.x == 0) {
@@ -856,29 +858,26 @@ __global__ void loc_scan_kernel(LocParams P) {
 
 __global__ void loc_scatter_kernel(LocParams P) {
   const int64_t n = P.n1 + P.n2, stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int lane = threadIdx.x & 31;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += stride) {
     const int c = loc_chunk(P, i);
-    const unsigned m = __match_any_sync(__activemask(), c);
-    const int leader = __ffs(m) - 1;
-    int base = 0;
-    if (lane == leader) base = atomicAdd(P.cursor + c, __popc(m));
-    base = __shfl_sync(m, base, leader);
-    const int rank = __popc(m & ((1u << lane) - 1u));
-    P.list[P.start[c] + base + rank] = static_cast<uint32_t>(i);
+    P.list[P.start[c] + atomicAdd(P.cursor + kLocPad * c, 1)] = static_cast<uint32_t>(i);
   }
 }
 
 // Items are slices of at most kLocItem queries of one chunk.  The block
-// stages the chunk's candidates as fp32 [len][kD] in shared memory; each
-// thread takes one query and scans them in increasing index with a strict
-// '>', so it keeps the lowest index reaching the largest recomputed score.
-// The key keeps the tensor cores' maximum as its score.
+// stages the chunk's candidates as fp32 [len][kD] in shared memory; thread t
+// takes query t % kLocItem and the candidate slice t / kLocItem, scans it in
+// increasing index with a strict '>' (so it keeps the lowest index reaching
+// its slice's largest recomputed score), and the slices meet in index order
+// in shared memory.  The key keeps the tensor cores' maximum as its score.
 template <bool kBf16, int kD>
-__global__ void __launch_bounds__(kLocItem) loc_resolve_kernel(LocParams P) {
+__global__ void __launch_bounds__(kLocItem* kLocSlices) loc_resolve_kernel(LocParams P) {
   extern __shared__ float cand[];
+  __shared__ float s_best[kLocSlices][kLocItem];
+  __shared__ int s_idx[kLocSlices][kLocItem];
   const int total = P.items[P.nch];
+  const int qt = threadIdx.x % kLocItem, slice = threadIdx.x / kLocItem;
   for (int it = blockIdx.x; it < total; it += gridDim.x) {
     int lo = 0, hi = P.nch;  // items[lo] <= it < items[hi]
     while (hi - lo > 1) {
@@ -892,17 +891,29 @@ __global__ void __launch_bounds__(kLocItem) loc_resolve_kernel(LocParams P) {
     const int64_t c0 = static_cast<int64_t>(rows ? c : c - P.nch_r) * L;
     const int len = static_cast<int>(ncand - c0 < L ? ncand - c0 : L);
     const uint16_t* X = rows ? P.X2 : P.X1;
-    __syncthreads();  // the previous item's readers are done with `cand`
-    for (int e = threadIdx.x; e < len * kD; e += blockDim.x) {
-      const int r = e / kD, ch = e - r * kD;
-      cand[e] = h2f(X[(c0 + r) * P.ld + ch], kBf16);
+    __syncthreads();  // the previous item's readers are done with `cand` and the slices
+    constexpr int kChunks = kD / 8;  // 16-byte pieces of a row
+    for (int e = threadIdx.x; e < len * kChunks; e += blockDim.x) {
+      const int r = e / kChunks, c8 = e - r * kChunks;
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(X + (c0 + r) * P.ld) + c8);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      float* dst = cand + r * kD + c8 * 8;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        dst[2 * k] = h2f(static_cast<uint16_t>(ws[k] & 0xFFFFu), kBf16);
+        dst[2 * k + 1] = h2f(static_cast<uint16_t>(ws[k] >> 16), kBf16);
+      }
     }
     __syncthreads();
     const int q0 = P.start[c] + (it - P.items[c]) * kLocItem;
-    const int qend = P.start[c] + P.cnt[c];
-    if (q0 + static_cast<int>(threadIdx.x) < qend) {
-      const uint32_t id = P.list[q0 + threadIdx.x];
-      const int64_t qi = rows ? static_cast<int64_t>(id) : static_cast<int64_t>(id) - P.n1;
+    const int qend = P.start[c] + P.cnt[kLocPad * c];
+    const bool live = q0 + qt < qend;
+    int64_t qi = 0;
+    float best = -__int_as_float(0x7f800000);
+    int bk = -1;
+    if (live) {
+      const uint32_t id = P.list[q0 + qt];
+      qi = rows ? static_cast<int64_t>(id) : static_cast<int64_t>(id) - P.n1;
       const uint16_t* qr = (rows ? P.X1 : P.X2) + qi * P.ld;
       float qv[kD];
 #pragma unroll
@@ -915,20 +926,53 @@ __global__ void __launch_bounds__(kLocItem) loc_resolve_kernel(LocParams P) {
           qv[ch + 2 * k + 1] = h2f(static_cast<uint16_t>(ws[k] >> 16), kBf16);
         }
       }
-      float best = -__int_as_float(0x7f800000);
-      int bk = 0;
-      for (int k = 0; k < len; ++k) {
+      const int per = (len + kLocSlices - 1) / kLocSlices;
+      const int k0 = slice * per, k1 = min(len, k0 + per);
+      int k = k0;
+      // two candidates at a time: independent sums, compared in index order;
+      // the rows come from shared memory as 16-byte vectors (one broadcast
+      // per four channels)
+      for (; k + 2 <= k1; k += 2) {
+        const float4* c0v = reinterpret_cast<const float4*>(cand + k * kD);
+        const float4* c1v = reinterpret_cast<const float4*>(cand + (k + 1) * kD);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < kD; ch += 4) {
+          const float4 x0 = c0v[ch / 4], x1 = c1v[ch / 4];
+          a0 = fmaf(qv[ch], x0.x, a0);
+          a0 = fmaf(qv[ch + 1], x0.y, a0);
+          a0 = fmaf(qv[ch + 2], x0.z, a0);
+          a0 = fmaf(qv[ch + 3], x0.w, a0);
+          a1 = fmaf(qv[ch], x1.x, a1);
+          a1 = fmaf(qv[ch + 1], x1.y, a1);
+          a1 = fmaf(qv[ch + 2], x1.z, a1);
+          a1 = fmaf(qv[ch + 3], x1.w, a1);
+        }
+        if (a0 > best) { best = a0; bk = k; }
+        if (a1 > best) { best = a1; bk = k + 1; }
+      }
+      for (; k < k1; ++k) {
         const float* cr = cand + k * kD;
         float acc = 0.f;
 #pragma unroll
         for (int ch = 0; ch < kD; ++ch) acc = fmaf(qv[ch], cr[ch], acc);
-        if (acc > best) {
-          best = acc;
-          bk = k;
+        if (acc > best) { best = acc; bk = k; }
+      }
+    }
+    s_best[slice][qt] = best;
+    s_idx[slice][qt] = bk;
+    __syncthreads();
+    if (slice == 0 && live) {
+      // slices in index order: a later slice wins only with a strictly larger score
+#pragma unroll
+      for (int sl = 1; sl < kLocSlices; ++sl) {
+        if (s_idx[sl][qt] >= 0 && s_best[sl][qt] > best) {
+          best = s_best[sl][qt];
+          bk = s_idx[sl][qt];
         }
       }
       unsigned long long* kp = rows ? P.rowk + qi : P.colk + qi;
-      *kp = pack_key(key_score(*kp), static_cast<int>(c0 + bk));
+      *kp = pack_key(key_score(*kp), static_cast<int>(c0 + (bk < 0 ? 0 : bk)));
     }
   }
 }
@@ -2002,8 +2046,8 @@ static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, rnn_metric met
   w->colk = c.take<unsigned long long>(n2 > 0 ? n2 : 1);
   w->counts = c.take<int>((n1 + kMnnChunk - 1) / kMnnChunk + 1);
   w->nch_max = (n2 + kOpRowChunk - 1) / kOpRowChunk + (n1 + 31) / 32;
-  w->loc_cnt = c.take<int>(w->nch_max + 1);
-  w->loc_cursor = c.take<int>(w->nch_max + 1);
+  w->loc_cnt = c.take<int>(kLocPad * (w->nch_max + 1));
+  w->loc_cursor = c.take<int>(kLocPad * (w->nch_max + 1));
   w->loc_start = c.take<int>(w->nch_max + 1);
   w->loc_items = c.take<int>(w->nch_max + 1);
   w->loc_list = c.take<uint32_t>(n1 + n2 > 0 ? n1 + n2 : 1);
@@ -2072,11 +2116,11 @@ template <bool kBf16>
 static rnn_status loc_resolve_launch(int d, const LocParams& P, int grid, size_t smem,
                                      cudaStream_t s) {
   switch (d) {
-    case 8: loc_resolve_kernel<kBf16, 8><<<grid, kLocItem, smem, s>>>(P); break;
-    case 16: loc_resolve_kernel<kBf16, 16><<<grid, kLocItem, smem, s>>>(P); break;
-    case 24: loc_resolve_kernel<kBf16, 24><<<grid, kLocItem, smem, s>>>(P); break;
-    case 32: loc_resolve_kernel<kBf16, 32><<<grid, kLocItem, smem, s>>>(P); break;
-    case 64: loc_resolve_kernel<kBf16, 64><<<grid, kLocItem, smem, s>>>(P); break;
+    case 8: loc_resolve_kernel<kBf16, 8><<<grid, kLocItem * kLocSlices, smem, s>>>(P); break;
+    case 16: loc_resolve_kernel<kBf16, 16><<<grid, kLocItem * kLocSlices, smem, s>>>(P); break;
+    case 24: loc_resolve_kernel<kBf16, 24><<<grid, kLocItem * kLocSlices, smem, s>>>(P); break;
+    case 32: loc_resolve_kernel<kBf16, 32><<<grid, kLocItem * kLocSlices, smem, s>>>(P); break;
+    case 64: loc_resolve_kernel<kBf16, 64><<<grid, kLocItem * kLocSlices, smem, s>>>(P); break;
     default: return RNN_EUNSUPPORTED;
   }
   return launched();
@@ -2159,7 +2203,8 @@ static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2
   P.X1 = X1;
   P.X2 = X2;
   P.ld = ld;
-  zero_words_kernel<<<grid_for(P.nch, di->sms), kSmallThreads, 0, s>>>(P.cnt, P.nch);
+  zero_words_kernel<<<grid_for(kLocPad * P.nch, di->sms), kSmallThreads, 0, s>>>(
+      P.cnt, static_cast<int64_t>(kLocPad) * P.nch);
   if ((r = launched()) != RNN_OK) return r;
   loc_count_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(P);
   if ((r = launched()) != RNN_OK) return r;
@@ -2168,7 +2213,7 @@ static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2
   loc_scatter_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(P);
   if ((r = launched()) != RNN_OK) return r;
   const int64_t max_items = P.nch + (n1 + n2) / kLocItem + 1;
-  const int rg = static_cast<int>(std::min<int64_t>(max_items, 4LL * di->sms));
+  const int rg = static_cast<int>(std::min<int64_t>(max_items, 8LL * di->sms));
   const size_t lsm = static_cast<size_t>(std::max(P.lr, P.lc)) * d * sizeof(float);
   return dtype == RNN_BF16 ? loc_resolve_launch<true>(d, P, rg, lsm, s)
                            : loc_resolve_launch<false>(d, P, rg, lsm, s);
