@@ -34,7 +34,7 @@ import time
 # first FRM call (20 launches averaged).  It belongs to the sources that
 # determine that kernel's memory traffic (see _kernel_sources_sha256): with any
 # other sources the bench reports traffic as null.
-TRAFFIC = {"sources_sha256": "479f6941dec8deb1efff62de04f96f9a84081885084d9d25211ee142715fa4fd",
+TRAFFIC = {"sources_sha256": "5da71dd25e046cadb30fecf30f2e10865058156d108a064e2a70365d10083178",
            "frm_nn_bytes_per_launch": 37.23e6}
 
 # What fixes the fused kernel's traffic: its own code and the PTX helpers,
