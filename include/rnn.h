@@ -92,6 +92,13 @@ rnn_status rnn_workspace_status(const void *workspace, rnn_stream_t stream);
 /* ------------------------------------------------------------------------
  * Nearest neighbours of a set of queries (the NN1 / NN2 operator).
  *
+ * NN2(D1_i) is the pixel of image 2 whose descriptor best matches D1_i, and
+ * NN1 the same from image 2 into image 1 (cv-learn.com "MASt3R" note,
+ * paragraph "Fast reciprocal matching (FRM)"; the staskaer.github.io
+ * DUSt3R/MASt3R blog, MASt3R matching section, where the quoted
+ * fast_reciprocal_NNs calls it on the active seeds at every half-step).
+ * Best = largest dot product, lowest index among equal scores.
+ *
  *   Q          [nq][d] query descriptors.
  *   X          [nx][d] candidate descriptors.
  *   idx_out    [nq] int32: NN of each query among the rows of X (lowest index
