@@ -34,7 +34,7 @@ import time
 # first FRM call (20 launches averaged).  It belongs to the sources that
 # determine that kernel's memory traffic (see _kernel_sources_sha256): with any
 # other sources the bench reports traffic as null.
-TRAFFIC = {"sources_sha256": "5da71dd25e046cadb30fecf30f2e10865058156d108a064e2a70365d10083178",
+TRAFFIC = {"sources_sha256": "c79b517a1c0f7c2021ec3a38a75d8ee4acaa70d655dc5012ea0c9e797f9aded7",
            "frm_nn_bytes_per_launch": 37.23e6}
 
 # What fixes the fused kernel's traffic: its own code and the PTX helpers,

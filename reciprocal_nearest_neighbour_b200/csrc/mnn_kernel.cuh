@@ -57,7 +57,10 @@
 //                slot's reuse period is at least 5 tiles (a warp can run at
 //                most 4 tiles ahead of the other), so small units use warp 1
 //                alone (nmma = 1).
-//   warps 3..18  epilogue, quadrant q = warp % 4, part p = (warp - 3) / 4
+//   warps 3..18  epilogue, quadrant q = warp % 4, part p = (warp - 3) / 4.
+//                They poll the accumulator barrier without suspending: a
+//                suspended wait wakes up later than a polled one, and the
+//                epilogue's wake-up is on every tile's critical path.
 #pragma once
 #include <cstdint>
 #include <type_traits>
@@ -357,7 +360,7 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
     // back, fold it.
     auto tile = [&](auto acc_c, int l, int n) -> bool {
       constexpr int kAcc = decltype(acc_c)::value;
-      if (!mbar_wait_fast(kAcc ? full1 : full0, (eph >> kAcc) & 1u, abort_flag, p.err,
+      if (!mbar_wait_spin(kAcc ? full1 : full0, (eph >> kAcc) & 1u, abort_flag, p.err,
                           kErrWaitEpilogue, lim))
         return false;
       eph ^= 1u << kAcc;

@@ -121,23 +121,27 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity,
   }
 }
 
-// mbar_wait_sleep with a non-blocking test first: a phase that has already
-// completed costs one instruction and no suspend.
-__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity,
+// Bounded wait that polls with the non-blocking test and never suspends:
+// for warps that wait on the critical path, where waking from a suspended
+// try_wait costs more than the issue slots the polling takes from the warps
+// beside them.  The abort flag and the time limit are looked at once every
+// 64 polls.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, int* err, int code,
                                                uint64_t limit_ns) {
-  return mbar_test_wait(bar, parity) ||
-         mbar_wait_sleep(bar, parity, abort_flag, err, code, limit_ns);
-}
-
-// Shared-memory fetch-and-add with acquire-release order at CTA scope.
-__device__ __forceinline__ uint32_t atom_add_acq_rel_shared(uint32_t addr, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "r"(addr), "r"(v)
-               : "memory");
-  return old;
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(err, code);
+      return false;
+    }
+  }
 }
 
 // 32-bit shared-memory accesses (addresses from smem_u32)
