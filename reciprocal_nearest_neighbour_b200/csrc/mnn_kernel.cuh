@@ -81,7 +81,7 @@ constexpr int kOpRowChunk = 64;   // columns of a row chunk (one epilogue warp's
 struct OnePassParams {
   int n1, n2;            // image-1 rows (tensor-memory lanes), image-2 rows (columns)
   int kpad;              // K of the tiles: 16, 32 or 64 (one K-block, swizzle 2*kpad bytes)
-  int bm, bn;            // m-tiles (a power of two) and n-tiles of a unit
+  int bm, bn;            // m-tiles (an even power of two) and n-tiles of a unit
   int nmma;              // MMA-issuing warps: 2, or 1 for small units
   int mblocks, nblocks;  // units = mblocks * nblocks; unit u -> (u % mblocks, u / mblocks)
   uint32_t idesc;
@@ -114,16 +114,22 @@ __host__ __device__ inline OnePassSmem onepass_smem(int kpad, int bm) {
 }
 
 // Row state of one (m-tile, row, part) slot: the best score over the
-// n-tiles so far and the first n-tile that reached it.  At n = 0 the slot is
-// written whatever it held (also when y is NaN: a part wholly past the last
-// image-2 row); later a strictly larger y replaces it.  Branch-free.
+// n-tiles so far and the first n-tile that reached it.  The first n-tile
+// writes the slot whatever it held (also when y is NaN: a part wholly past
+// the last image-2 row); a later n-tile n replaces it only with a strictly
+// larger y.  Branch-free.
+__device__ __forceinline__ void row_state_first(uint32_t slot, uint32_t cslot, float y) {
+  asm volatile(
+      "st.shared.f32 [%0], %2;\n\t"
+      "st.shared.u8 [%1], 0;" ::"r"(slot),
+      "r"(cslot), "f"(y)
+      : "memory");
+}
 __device__ __forceinline__ void row_state_update(uint32_t slot, uint32_t cslot, float y, int n) {
   asm volatile(
-      "{\n\t.reg .pred p, z;\n\t.reg .f32 o;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .f32 o;\n\t"
       "ld.shared.f32 o, [%0];\n\t"
       "setp.gt.f32 p, %2, o;\n\t"
-      "setp.eq.s32 z, %3, 0;\n\t"
-      "or.pred p, p, z;\n\t"
       "@p st.shared.f32 [%0], %2;\n\t"
       "@p st.shared.u8 [%1], %3;\n\t}" ::"r"(slot),
       "r"(cslot), "f"(y), "r"(n)
@@ -349,7 +355,9 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
     const uint32_t full0 = smem_u32(&acc_full[0]), full1 = smem_u32(&acc_full[1]);
     const uint32_t empty0 = smem_u32(&acc_empty[0]), empty1 = smem_u32(&acc_empty[1]);
     const float ninf = -__int_as_float(0x7f800000);
-    uint32_t eph = 0;  // bit a: phase of accumulator a's next result
+    // phase of the accumulators' next results: tiles alternate between the
+    // two (bm is even), so both accumulators' k-th uses share the parity k % 2
+    uint32_t ph = 0;
     int rowphase = 0;
     bool ok = true;
     float pm[16];      // running maxima of this thread's 16 columns over its rows
@@ -358,12 +366,12 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
     // kAcc: read the 4 x 16 block (rows g, g+8 into va, rows g+16, g+24 into
     // vb; column 4j + s in registers 2j and 2j + 1), hand the accumulator
     // back, fold it.
-    auto tile = [&](auto acc_c, int l, int n) -> bool {
+    auto tile = [&](auto acc_c, auto first_c, int l, int n) -> bool {
       constexpr int kAcc = decltype(acc_c)::value;
-      if (!mbar_wait_spin(kAcc ? full1 : full0, (eph >> kAcc) & 1u, abort_flag, p.err,
-                          kErrWaitEpilogue, lim))
+      constexpr bool kFirst = decltype(first_c)::value;  // n == 0
+      if (!mbar_wait_spin(kAcc ? full1 : full0, ph, abort_flag, p.err, kErrWaitEpilogue, lim))
         return false;
-      eph ^= 1u << kAcc;
+      if (kAcc) ph ^= 1u;
       tc_fence_after();
       float va[32], vb[32];
       const uint32_t ta = tq + static_cast<uint32_t>(kAcc * kOpBlockN);
@@ -394,7 +402,18 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
       const float x0 = swap_max(r0, r1, s0, 1);  // row (s & 1)
       const float x1 = swap_max(r2, r3, s0, 1);  // row 2 + (s & 1)
       const float y = swap_max(x0, x1, s1, 2);   // row s
-      row_state_update(rb_s + 2048u * l, rc_s + 512u * l, y, n);
+      if (kFirst)
+        row_state_first(rb_s + 2048u * l, rc_s + 512u * l, y);
+      else
+        row_state_update(rb_s + 2048u * l, rc_s + 512u * l, y, n);
+      return true;
+    };
+    // one n-pass: tile l uses accumulator l % 2
+    auto pass = [&](auto first_c, int n) -> bool {
+      for (int l = 0; l < bm; l += 2) {
+        if (!tile(std::integral_constant<int, 0>{}, first_c, l, n)) return false;
+        if (!tile(std::integral_constant<int, 1>{}, first_c, l + 1, n)) return false;
+      }
       return true;
     };
 
@@ -405,11 +424,7 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
         const int col0 = (nb * bn + n) * kOpBlockN + 64 * part;  // first column of this part
 #pragma unroll
         for (int c = 0; c < 16; ++c) pm[c] = ninf;
-        // tile l of an n-pass uses accumulator l % 2 (bm is a power of two)
-        for (int l = 0; l < bm && ok; l += 2) {
-          ok = tile(std::integral_constant<int, 0>{}, l, n);
-          if (ok && l + 1 < bm) ok = tile(std::integral_constant<int, 1>{}, l + 1, n);
-        }
+        ok = n == 0 ? pass(std::true_type{}, 0) : pass(std::false_type{}, n);
         if (!ok) break;
         // ---- column flush: over the 8 lanes of this quadrant holding the same columns
         float x[8], y4[4], z[2];

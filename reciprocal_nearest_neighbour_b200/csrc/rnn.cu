@@ -2091,8 +2091,10 @@ struct OnePassPlan {
 };
 
 // Unit shape: the largest that shared memory holds (bm query tiles of
-// 128 x kpad, bm a power of two; 8 candidate tiles), halved along the longer
-// side until there are at least two units per SM.  Two MMA-issuing warps when
+// 128 x kpad, bm a power of two and at least 2, so that the tiles of every
+// pass alternate between the two accumulators; query tiles past the last row
+// read the NaN tail; 8 candidate tiles), halved along the longer side until
+// there are at least two units per SM.  Two MMA-issuing warps when
 // every shared-memory slot's reuse period is at least 5 tiles (2*bm for a
 // candidate slot, bm*bn for a query slot).
 static OnePassPlan onepass_plan(int64_t n1, int64_t n2, int kpad, int sms) {
@@ -2100,10 +2102,10 @@ static OnePassPlan onepass_plan(int64_t n1, int64_t n2, int kpad, int sms) {
   const int nt = static_cast<int>((n2 + kOpBlockN - 1) / kOpBlockN);
   auto blocks = [](int t, int b) { return (t + b - 1) / b; };
   int bm = kpad == 64 ? 8 : kOpMaxBm;
-  while (bm > 1 && bm > mt) bm >>= 1;
+  while (bm > 2 && bm > mt) bm >>= 1;
   int bn = std::min(kOpMaxBn, nt);
-  while (static_cast<int64_t>(blocks(mt, bm)) * blocks(nt, bn) < 2LL * sms && (bm > 1 || bn > 1)) {
-    if (bn >= bm && bn > 1)
+  while (static_cast<int64_t>(blocks(mt, bm)) * blocks(nt, bn) < 2LL * sms && (bm > 2 || bn > 1)) {
+    if (bn > 1 && (bn >= bm || bm <= 2))
       bn = (bn + 1) / 2;
     else
       bm >>= 1;
