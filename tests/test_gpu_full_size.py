@@ -69,6 +69,24 @@ def test_mnn_full_size_quantised_bitexact():
     assert len(ref_pairs) > 1000
 
 
+def test_mnn_full_size_quantised_bf16_bitexact():
+    """The same quantised maps stored as bf16 (k/64 with |k| <= 127 has at
+    most 7 significant bits, so bf16 holds it exactly): the whole set equals
+    the oracle's, bit for bit."""
+    w, a, b = refs.mnn_inputs("q")
+    z = _mnn_ref("q", a, b)
+    a2, b2 = a.to(torch.bfloat16), b.to(torch.bfloat16)
+    assert torch.equal(a2.float(), a.float()) and torch.equal(b2.float(), b.float())
+    r = rnn.mnn_exhaustive(dev(a2), dev(b2), with_nn=True)
+    assert np.array_equal(r.rowarg.cpu().numpy(), z["rowarg"])
+    assert np.array_equal(r.colarg.cpu().numpy(), z["colarg"])
+    rowmax = r.rowmax.cpu().numpy().astype(np.float64) * 4096.0
+    colmax = r.colmax.cpu().numpy().astype(np.float64) * 4096.0
+    assert np.array_equal(rowmax, z["rowbest4096"].astype(np.float64))
+    assert np.array_equal(colmax, z["colbest4096"].astype(np.float64))
+    assert np.array_equal(r.trimmed().cpu().numpy(), _mutual_pairs(z["rowarg"], z["colarg"]))
+
+
 def test_mnn_full_size_fp16_tolerance():
     """The whole 512x384, d = 24 set on unit-norm fp16 maps: every index and
     score under the tolerance rule, and the pair list differing from the
