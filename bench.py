@@ -323,6 +323,7 @@ def run_native(args):
                 "unit": "TFLOP/s", "frac": round(achieved_tf / peak_tf, 4), "traffic": traffic,
                 "kernel": "nn_argmax_kernel", "launches": nrec,
                 "avg_launch_us": round(1e3 * sum(nn_ms) / max(nrec, 1), 3),
+                "flops_per_launch": round(flops / max(nrec, 1), -6),
                 "peak_source": f"bf16 burst, {peaks['source']}",
                 "active_queries_per_pair": queries_per_call / P}
 
