@@ -34,7 +34,7 @@ import time
 # first FRM call (20 launches averaged).  It belongs to the sources that
 # determine that kernel's memory traffic (see _kernel_sources_sha256): with any
 # other sources the bench reports traffic as null.
-TRAFFIC = {"sources_sha256": "c79b517a1c0f7c2021ec3a38a75d8ee4acaa70d655dc5012ea0c9e797f9aded7",
+TRAFFIC = {"sources_sha256": "c420dfd32bec45cd77db817ca97c9e7fc7813d08cf1aaca6d59ad29529010e7d",
            "frm_nn_bytes_per_launch": 37.23e6}
 
 # What fixes the fused kernel's traffic: its own code and the PTX helpers,
