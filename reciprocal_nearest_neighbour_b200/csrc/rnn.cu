@@ -153,14 +153,18 @@ static Geometry geometry(int d) {
 }
 
 // The one-pass kernel for the exhaustive set covers one K-block of 16, 32 or
-// 64 (d <= 32 or d = 64) with the dot metric; other shapes take the
-// two-sweep form.  Its copies of the maps carry kOpPadRows NaN rows past the
-// last pixel: enough for the last unit (bm*128 <= 2048 query rows, 8*256
-// candidate rows) to read nothing but NaN beyond the end.
+// 64; other shapes take the two-sweep form.  Its copies of the maps carry
+// kOpPadRows NaN rows past the last pixel: enough for the last unit
+// (bm*128 <= 2048 query rows, 8*256 candidate rows) to read nothing but NaN
+// beyond the end.  Under the Euclidean metric the copies carry six more
+// columns (op_copy_kernel), so that one score serves both directions.
 constexpr int64_t kOpPadRows = 2048;
-static bool onepass_fits(const Geometry& g, rnn_metric metric) {
-  return metric == RNN_DOT && g.nkb == 1 && g.block_n == kOpBlockN &&
-         (g.kpad == 16 || g.kpad == 32 || g.kpad == 64);
+constexpr int kOpAugCols = 6;
+static Geometry onepass_geometry(int d, rnn_metric metric) {
+  return geometry(d + (metric == RNN_L2 ? kOpAugCols : 0));
+}
+static bool onepass_fits(const Geometry& g) {
+  return g.nkb == 1 && g.block_n == kOpBlockN && (g.kpad == 16 || g.kpad == 32 || g.kpad == 64);
 }
 
 // Depth K of the tensor-core tiles for d channels (d rounded up to the
@@ -771,6 +775,7 @@ struct LocParams {
   const uint16_t* X1;        // rows of image 1 and image 2, ld elements apart
   const uint16_t* X2;
   int ld;
+  int l2;                    // Euclidean forms: report -2 x the score (the squared distance)
 };
 
 __device__ __forceinline__ int loc_chunk(const LocParams& P, int64_t i) {
@@ -794,21 +799,72 @@ __global__ void zero_words_kernel(int* a, int64_t n) {
 // The one-pass kernel's copy of a map: rows of kpad elements, the d channels
 // then zeros, and NaN rows from row n to ntot.  One thread per 16-byte chunk
 // of the output.
+// Copies of the maps for the one-pass kernel: rows of kpad channels (zeros
+// past d), then NaN rows up to ntot.  Under the Euclidean metric the first
+// chunk past the channels holds, for image 1 (form kOpFormA),
+//   1, 1, 1, p0, p1, p2
+// and for image 2 (form kOpFormB)
+//   p0, p1, p2, 1, 1, 1
+// where p0 + p1 + p2 = -|row|^2/2 (the row's own norm, split greedily into
+// three 16-bit parts as in prep_chunk).  The tensor cores then compute
+//   q.x - |x|^2/2 - |q|^2/2 = -|q - x|^2/2
+// for every pair: the largest value of a row is its nearest image-2 pixel and
+// the largest of a column its nearest image-1 pixel.  On k/64 inputs every
+// part and partial sum is a multiple of 2^-13 far inside fp32's range, so the
+// score is exact.
+constexpr int kOpFormDot = 0, kOpFormA = 1, kOpFormB = 2;
+template <bool kBf16>
+__device__ __forceinline__ uint4 op_aug_chunk(const uint4* __restrict__ row, int creal, int form) {
+  float n2 = 0.f;
+  for (int cc = 0; cc < creal; ++cc) {
+    const uint4 x = __ldg(row + cc);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = bits_to_f(static_cast<uint16_t>(w[e] & 0xFFFFu), kBf16);
+      const float hi = bits_to_f(static_cast<uint16_t>(w[e] >> 16), kBf16);
+      n2 = fmaf(lo, lo, n2);
+      n2 = fmaf(hi, hi, n2);
+    }
+  }
+  uint16_t part[3];
+  float rest = -0.5f * n2;
+#pragma unroll
+  for (int e = 0; e < 3; ++e) {
+    part[e] = f_to_bits(rest, kBf16);
+    rest -= bits_to_f(part[e], kBf16);
+  }
+  const uint32_t one = f_to_bits(1.0f, kBf16);
+  uint16_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int e = 0; e < 3; ++e) {
+    h[form == kOpFormA ? e : 3 + e] = static_cast<uint16_t>(one);
+    h[form == kOpFormA ? 3 + e : e] = part[e];
+  }
+  return make_uint4(h[0] | (static_cast<uint32_t>(h[1]) << 16),
+                    h[2] | (static_cast<uint32_t>(h[3]) << 16),
+                    h[4] | (static_cast<uint32_t>(h[5]) << 16),
+                    h[6] | (static_cast<uint32_t>(h[7]) << 16));
+}
+
+template <bool kBf16>
 __global__ void op_copy_kernel(const uint16_t* __restrict__ src, int64_t n, int d,
-                               uint16_t* __restrict__ dst, int kpad, int64_t ntot, int bf16) {
+                               uint16_t* __restrict__ dst, int kpad, int64_t ntot, int form) {
   const int cpr = kpad / 8, creal = d / 8;
-  const uint16_t nan16 = bf16 ? 0x7FC0u : 0x7E00u;
+  const uint16_t nan16 = kBf16 ? 0x7FC0u : 0x7E00u;
   const uint32_t nan2 = static_cast<uint32_t>(nan16) * 0x10001u;
   const int64_t total = ntot * cpr, stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += stride) {
     const int64_t r = i / cpr;
     const int c = static_cast<int>(i - r * cpr);
+    const uint4* row = reinterpret_cast<const uint4*>(src + r * d);
     uint4 v;
     if (r >= n)
       v = make_uint4(nan2, nan2, nan2, nan2);
     else if (c < creal)
-      v = __ldg(reinterpret_cast<const uint4*>(src + r * d) + c);
+      v = __ldg(row + c);
+    else if (c == creal && form != kOpFormDot)
+      v = op_aug_chunk<kBf16>(row, creal, form);
     else
       v = make_uint4(0u, 0u, 0u, 0u);
     reinterpret_cast<uint4*>(dst)[i] = v;
@@ -972,7 +1028,8 @@ __global__ void __launch_bounds__(kLocItem* kLocSlices) loc_resolve_kernel(LocPa
         }
       }
       unsigned long long* kp = rows ? P.rowk + qi : P.colk + qi;
-      *kp = pack_key(key_score(*kp), static_cast<int>(c0 + (bk < 0 ? 0 : bk)));
+      const float sc = key_score(*kp);
+      *kp = pack_key(P.l2 ? -2.f * sc : sc, static_cast<int>(c0 + (bk < 0 ? 0 : bk)));
     }
   }
 }
@@ -2053,9 +2110,9 @@ static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, rnn_metric met
   w->loc_list = c.take<uint32_t>(n1 + n2 > 0 ? n1 + n2 : 1);
   w->q1 = w->x1 = w->q2 = w->x2 = nullptr;
   const int mode = d > 0 ? copies_for(d, metric) : kCopiesNone;
-  if (d > 0 && onepass_fits(geometry(d), metric)) {
+  if (d > 0 && onepass_fits(onepass_geometry(d, metric))) {
     // one-pass form: padded rows, then kOpPadRows NaN rows
-    const int kpad = geometry(d).kpad;
+    const int kpad = onepass_geometry(d, metric).kpad;
     w->q1 = w->x1 = c.take<uint16_t>((n1 + kOpPadRows) * kpad);
     w->q2 = w->x2 = c.take<uint16_t>((n2 + kOpPadRows) * kpad);
   } else if (mode != kCopiesNone) {
@@ -2143,8 +2200,8 @@ static cudaError_t loc_resolve_attr(int smem) {
 // Keys of both directions from one pass over the scores, then the grouped
 // locate.  X1, X2: the rows the tensor maps read (ld elements apart).
 static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2, int64_t n2,
-                              int ld, int d, rnn_dtype dtype, const Geometry& g, const MnnWs& w,
-                              DeviceInfo* di, cudaStream_t s) {
+                              int ld, int d, bool l2, rnn_dtype dtype, const Geometry& g,
+                              const MnnWs& w, DeviceInfo* di, cudaStream_t s) {
   constexpr int kLocSmem = 64 * 1024;
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -2205,6 +2262,7 @@ static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2
   P.X1 = X1;
   P.X2 = X2;
   P.ld = ld;
+  P.l2 = l2 ? 1 : 0;
   zero_words_kernel<<<grid_for(kLocPad * P.nch, di->sms), kSmallThreads, 0, s>>>(
       P.cnt, static_cast<int64_t>(kLocPad) * P.nch);
   if ((r = launched()) != RNN_OK) return r;
@@ -2216,9 +2274,11 @@ static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2
   if ((r = launched()) != RNN_OK) return r;
   const int64_t max_items = P.nch + (n1 + n2) / kLocItem + 1;
   const int rg = static_cast<int>(std::min<int64_t>(max_items, 8LL * di->sms));
-  const size_t lsm = static_cast<size_t>(std::max(P.lr, P.lc)) * d * sizeof(float);
-  return dtype == RNN_BF16 ? loc_resolve_launch<true>(d, P, rg, lsm, s)
-                           : loc_resolve_launch<false>(d, P, rg, lsm, s);
+  // the Euclidean forms are recomputed over all their channels
+  const int kd = l2 ? ld : d;
+  const size_t lsm = static_cast<size_t>(std::max(P.lr, P.lc)) * kd * sizeof(float);
+  return dtype == RNN_BF16 ? loc_resolve_launch<true>(kd, P, rg, lsm, s)
+                           : loc_resolve_launch<false>(kd, P, rg, lsm, s);
 }
 
 extern "C" {
@@ -2251,20 +2311,34 @@ rnn_status rnn_mnn_exhaustive_ex(const void* D1, int H1, int W1, const void* D2,
 
   const bool l2 = metric == RNN_L2;
   const Geometry g = geometry(d + (l2 ? kAugCols : 0));
+  const Geometry og = onepass_geometry(d, metric);
   const int nb = nblk1 > nblk2 ? nblk1 : nblk2;
   zero_keys_kernel<<<grid_for(n1 + n2, di->sms), kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2,
                                                                         w.err);
   if ((r = launched()) != RNN_OK) return r;
-  if (onepass_fits(g, metric)) {
+  if (onepass_fits(og)) {
     // every score once, reduced by rows and by columns
-    const int bf = dtype == RNN_BF16 ? 1 : 0;
-    op_copy_kernel<<<grid_for((n1 + kOpPadRows) * g.kpad / 8, di->sms), kSmallThreads, 0, s>>>(
-        static_cast<const uint16_t*>(D1), n1, d, w.q1, g.kpad, n1 + kOpPadRows, bf);
+    const uint16_t* s1 = static_cast<const uint16_t*>(D1);
+    const uint16_t* s2 = static_cast<const uint16_t*>(D2);
+    const int f1 = l2 ? kOpFormA : kOpFormDot, f2 = l2 ? kOpFormB : kOpFormDot;
+    const int g1 = grid_for((n1 + kOpPadRows) * og.kpad / 8, di->sms);
+    const int g2 = grid_for((n2 + kOpPadRows) * og.kpad / 8, di->sms);
+    if (dtype == RNN_BF16) {
+      op_copy_kernel<true><<<g1, kSmallThreads, 0, s>>>(s1, n1, d, w.q1, og.kpad,
+                                                        n1 + kOpPadRows, f1);
+      if ((r = launched()) != RNN_OK) return r;
+      op_copy_kernel<true><<<g2, kSmallThreads, 0, s>>>(s2, n2, d, w.q2, og.kpad,
+                                                        n2 + kOpPadRows, f2);
+    } else {
+      op_copy_kernel<false><<<g1, kSmallThreads, 0, s>>>(s1, n1, d, w.q1, og.kpad,
+                                                         n1 + kOpPadRows, f1);
+      if ((r = launched()) != RNN_OK) return r;
+      op_copy_kernel<false><<<g2, kSmallThreads, 0, s>>>(s2, n2, d, w.q2, og.kpad,
+                                                         n2 + kOpPadRows, f2);
+    }
     if ((r = launched()) != RNN_OK) return r;
-    op_copy_kernel<<<grid_for((n2 + kOpPadRows) * g.kpad / 8, di->sms), kSmallThreads, 0, s>>>(
-        static_cast<const uint16_t*>(D2), n2, d, w.q2, g.kpad, n2 + kOpPadRows, bf);
-    if ((r = launched()) != RNN_OK) return r;
-    if ((r = mnn_onepass(w.q1, n1, w.q2, n2, g.kpad, d, dtype, g, w, di, s)) != RNN_OK) return r;
+    if ((r = mnn_onepass(w.q1, n1, w.q2, n2, og.kpad, d, l2, dtype, og, w, di, s)) != RNN_OK)
+      return r;
     mnn_count_kernel<<<nb, kSmallThreads, 0, s>>>(w.rowk, n1, w.colk, n2, w.counts, nblk1,
                                                   rowarg_out, rowmax_out, colarg_out, colmax_out);
     if ((r = launched()) != RNN_OK) return r;

@@ -67,9 +67,13 @@ def test_workspace_sizes(lib):
             >= 2 * n * 8 + 2 * (n + 2048) * 64)
     assert (lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24)
             == lib.rnn_mnn_workspace_size(384, 512, 384, 512, 32))
-    # the Euclidean metric keeps the two-sweep form: a query and a candidate form per map
+    # the Euclidean metric takes the one-pass kernel too (d = 24: 24 channels and six
+    # form columns in 32), on the same copies; at d = 64 it keeps the two sweeps with
+    # a query and a candidate form per map (67 columns padded to 80, 160-byte rows)
     assert (lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, 1)
-            >= 2 * n * 8 + 4 * n * 64)
+            == lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24))
+    assert (lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 64, 1)
+            >= 2 * n * 8 + 4 * n * 160)
     one = lib.rnn_frm_workspace_size(1, 384, 512, 384, 512, 32, 8)
     many = lib.rnn_frm_workspace_size(64, 288, 512, 288, 512, 32, 8)
     assert one > 0 and many > 64 * 2304 * 8
@@ -148,10 +152,10 @@ def test_frm_argument_errors(lib):
 def test_ex_workspace_sizes(lib):
     dot = lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, _lib.RNN_DOT)
     assert dot == lib.rnn_mnn_workspace_size(384, 512, 384, 512, 24)
-    # the Euclidean metric keeps a query and a candidate form of each map (the
-    # dot metric holds one padded copy of each, with a tail of 2048 rows)
+    # both metrics run the one-pass kernel at d = 24 on one padded copy of each
+    # map (the Euclidean forms fit their six columns in the same 32 channels)
     l2 = lib.rnn_mnn_workspace_size_ex(384, 512, 384, 512, 24, _lib.RNN_L2)
-    assert l2 >= dot + 2 * 384 * 512 * 32 * 2 - 2 * 2048 * 32 * 2
+    assert l2 == dot
     assert lib.rnn_nn_workspace_size_ex(100, 5000, 24, _lib.RNN_DOT) == \
         lib.rnn_nn_workspace_size(100)
     assert lib.rnn_nn_workspace_size_ex(100, 5000, 24, _lib.RNN_L2) >= \

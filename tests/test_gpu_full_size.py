@@ -168,6 +168,21 @@ def test_mnn_multi_unit_ragged_bitexact(dt):
     assert np.array_equal(r.trimmed().cpu().numpy(), ref.pairs.reshape(-1, 2))
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_mnn_l2_multi_unit_ragged_bitexact(dt):
+    """The Euclidean metric on the same multi-unit ragged shapes: nearest
+    neighbours by distance in both directions, squared distances, bit for bit."""
+    D1, D2 = synth.quantised_pair(78, 160, 161, 190, 257, 24)
+    a, b = synth.to_storage(D1, dt), synth.to_storage(D2, dt)
+    r = rnn.mnn_exhaustive(dev(a), dev(b), with_nn=True, metric="l2")
+    ref = oracle.mnn(a, b, metric="l2")
+    assert np.array_equal(r.rowarg.cpu().numpy(), ref.row.arg)
+    assert np.array_equal(r.colarg.cpu().numpy(), ref.col.arg)
+    assert np.array_equal(r.rowmax.cpu().numpy().astype(np.float64), -ref.row.best)
+    assert np.array_equal(r.colmax.cpu().numpy().astype(np.float64), -ref.col.best)
+    assert np.array_equal(r.trimmed().cpu().numpy(), ref.pairs.reshape(-1, 2))
+
+
 @pytest.mark.parametrize("d", [8, 16, 24, 32, 64])
 def test_mnn_ties_across_chunks(d):
     """Rows copied far from their originals in both maps (other quadrants,

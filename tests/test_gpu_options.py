@@ -64,8 +64,11 @@ def test_nn_l2_unit_fp16_tolerance():
 
 
 @pytest.mark.parametrize("s1,s2,d", [((32, 32), (32, 32), 16), ((37, 41), (29, 53), 24),
-                                     ((20, 30), (25, 21), 32)])
+                                     ((20, 30), (25, 21), 32), ((9, 7), (11, 5), 8),
+                                     ((31, 33), (27, 35), 56), ((24, 26), (22, 28), 64)])
 def test_mnn_l2_quantised_bitexact(s1, s2, d):
+    """Under the Euclidean metric d <= 56 runs the one-pass kernel on the
+    symmetric forms (-|q - x|^2/2 for every pair), d = 64 the two sweeps."""
     rng = np.random.default_rng(5 + d)
     D1 = synth.to_storage(synth.quantised_map(rng, *s1, d), "f16")
     D2 = synth.to_storage(synth.quantised_map(rng, *s2, d), "f16")
