@@ -67,7 +67,7 @@ typedef enum rnn_dtype { RNN_F16 = 0, RNN_BF16 = 1 } rnn_dtype;
  *            note, section "Method and architecture").
  *   RNN_L2   the smallest Euclidean distance |D1_i - D2_j|, which is what the
  *            brute-force matcher of the quoted fast_reciprocal_NNs computes
- *            ("every distance, then the minimum"; staskaer.github.io
+ *            (all distances, the smallest kept; staskaer.github.io
  *            DUSt3R/MASt3R blog, MASt3R matching section).
  * Ties go to the lowest index under either metric.
  */

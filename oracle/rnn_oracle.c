@@ -52,7 +52,7 @@ static double score(const double *a, const double *b, int d)
  * Metric of the nearest-neighbour query.  METRIC_DOT: the largest dot
  * product (the reading used throughout).  METRIC_L2: the smallest Euclidean
  * distance, which is what the quoted function's brute-force matcher computes
- * ("compute every distance and take the minimum"); it is scored here as the
+ * (it forms all the distances and keeps the smallest); it is scored here as the
  * negated squared distance so that "largest score" still means "nearest".
  */
 enum { METRIC_DOT = 0, METRIC_L2 = 1 };
