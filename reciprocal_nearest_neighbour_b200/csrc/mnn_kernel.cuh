@@ -22,11 +22,16 @@
 // thread keeps the running maximum of its 16 columns in registers over the
 // whole inner loop (two three-input maxima per column and tile), merges
 // them across its 8 lanes once per n-tile and writes them to the global keys
-// with atomicMax (one chunk per quadrant, so no meeting between warps).  Row partials (one per row and
-// 64-column part, after a two-step shuffle across 4 lanes) go to shared
-// memory, where each (m-tile, row, part) slot keeps the best over the n-tiles
-// with the first n-tile that reached it; they are merged and written once
-// per unit.
+// with atomicMax (one chunk per quadrant, so no meeting between warps).  Row
+// partials (one per row and 64-column part, after a two-step shuffle across
+// 4 lanes) go to shared memory, where each (m-tile, row, part) slot keeps the
+// best over the n-tiles with the first n-tile that reached it; they are
+// merged and written once per unit.
+//
+// Metric.  The kernel takes the largest score of rows and columns of
+// whatever the copies of the maps give: the dot product, or under the
+// Euclidean metric the copies' extra columns make every score
+// -|q - x|^2 / 2, symmetric in the two maps (op_copy_kernel in rnn.cu).
 //
 // Ragged edges.  The maps are read from copies whose rows past the last
 // pixel (up to a whole unit) are NaN, so every score there is NaN, and the
