@@ -63,9 +63,11 @@
 //                most 4 tiles ahead of the other), so small units use warp 1
 //                alone (nmma = 1).
 //   warps 3..18  epilogue, quadrant q = warp % 4, part p = (warp - 3) / 4.
-//                They poll the accumulator barrier without suspending: a
-//                suspended wait wakes up later than a polled one, and the
-//                epilogue's wake-up is on every tile's critical path.
+//                The epilogue warps beside the MMA warps (q = 1, 2) run about
+//                a tile behind the others and their releases gate every next
+//                MMA: they poll the accumulator barrier without suspending (a
+//                suspended wait wakes up later).  The warps of q = 0, 3 wait
+//                ahead of them and suspend.
 #pragma once
 #include <cstdint>
 #include <type_traits>
@@ -347,6 +349,7 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
     // --------------------------------------------------------- epilogue
     const int e = warp - kOpEpiWarp0;
     const int q = warp & 3;        // tensor-memory lane quadrant this warp may read
+    const bool spin = q == 1 || q == 2;  // shares its sub-partition with an MMA warp
     const int part = e >> 2;       // 64-column part of the tile
     const int g = lane >> 2, s = lane & 3;
     const bool s0 = (lane & 1) != 0, s1 = (lane & 2) != 0;
@@ -374,7 +377,12 @@ mnn_onepass_kernel(const __grid_constant__ OnePassParams p,
     auto tile = [&](auto acc_c, auto first_c, int l, int n) -> bool {
       constexpr int kAcc = decltype(acc_c)::value;
       constexpr bool kFirst = decltype(first_c)::value;  // n == 0
-      if (!mbar_wait_spin(kAcc ? full1 : full0, ph, abort_flag, p.err, kErrWaitEpilogue, lim))
+      // the sub-partitions of the two MMA warps (q = 1, 2) set the tile period
+      // and poll; the other two wait ahead of them, and suspend so that their
+      // polling adds nothing to the barrier traffic
+      const uint32_t fb = kAcc ? full1 : full0;
+      if (!(spin ? mbar_wait_spin(fb, ph, abort_flag, p.err, kErrWaitEpilogue, lim)
+                 : mbar_wait_sleep(fb, ph, abort_flag, p.err, kErrWaitEpilogue, lim)))
         return false;
       if (kAcc) ph ^= 1u;
       tc_fence_after();
