@@ -15,6 +15,9 @@ Files (``tests/golden/full_size/``):
   ``colarg`` (NN2 of every image-1 pixel, NN1 of every image-2 pixel) and
   ``rowbest4096``, ``colbest4096``: the best scores times 4096, which are
   integers (every score is a multiple of 2^-12).
+* ``mnn_512x384_q_l2.npz``: the quantised maps under the Euclidean metric
+  (nearest by |a - b|^2, lowest index on ties); the best scores (-|a - b|^2)
+  times 4096, integers as above.
 * ``mnn_512x384_f.npz``: the unit-norm fp16 maps.  ``rowarg``, ``colarg``,
   ``rowbest``, ``colbest`` and the top-2 gaps ``rowgap``, ``colgap``.  The
   scores are stored as float32: the tolerance rule compares them with a
@@ -24,8 +27,8 @@ Files (``tests/golden/full_size/``):
   queries made, converged flag and the smallest top-2 gap along the seed's
   trajectory; the pairs follow from the converged seeds.
 
-Usage: ``python tests/golden/make_full_size_refs.py [mnn_q] [mnn_f] [frm64]``
-(default: all three).
+Usage: ``python tests/golden/make_full_size_refs.py [mnn_q] [mnn_q_l2] [mnn_f] [frm64]``
+(default: all four).
 """
 from __future__ import annotations
 
@@ -83,12 +86,12 @@ def path(name: str) -> str:
     return os.path.join(OUT, name + ".npz")
 
 
-def write_mnn(mode: str) -> str:
+def write_mnn(mode: str, metric: str = "dot") -> str:
     import oracle
 
     w, a, b = mnn_inputs(mode)
     t0 = time.time()
-    ref = oracle.mnn(a, b)
+    ref = oracle.mnn(a, b, metric=metric)
     dt = time.time() - t0
     meta = dict(inputs_sha256=inputs_sha256(a, b), oracle_sha256=oracle_sha256(),
                 workload=w.name, oracle_seconds=dt, threads=oracle.max_threads())
@@ -102,7 +105,7 @@ def write_mnn(mode: str) -> str:
         arrs.update(rowbest=ref.row.best.astype(np.float32), colbest=ref.col.best.astype(np.float32),
                     rowgap=ref.row.gap.astype(np.float32), colgap=ref.col.gap.astype(np.float32))
     os.makedirs(OUT, exist_ok=True)
-    name = "mnn_512x384_" + mode
+    name = "mnn_512x384_" + mode + ("" if metric == "dot" else "_" + metric)
     np.savez_compressed(path(name), **arrs, **{k: np.array(v) for k, v in meta.items()})
     return f"{name}: |M| = {len(ref.pairs)}, oracle {dt:.0f} s"
 
@@ -143,10 +146,12 @@ def load(name: str, *tensors):
 
 
 def main(argv) -> None:
-    jobs = argv or ["mnn_q", "mnn_f", "frm64"]
+    jobs = argv or ["mnn_q", "mnn_q_l2", "mnn_f", "frm64"]
     for j in jobs:
         if j == "mnn_q":
             print(write_mnn("q"), flush=True)
+        elif j == "mnn_q_l2":
+            print(write_mnn("q", "l2"), flush=True)
         elif j == "mnn_f":
             print(write_mnn("f"), flush=True)
         elif j == "frm64":

@@ -37,11 +37,11 @@ def _mutual_pairs(rowarg, colarg):
     return np.stack([i, rowarg[i]], axis=1).astype(np.int32).reshape(-1, 2)
 
 
-def _mnn_ref(mode, a, b):
-    z = refs.load("mnn_512x384_" + mode, a, b)
+def _mnn_ref(mode, a, b, metric="dot"):
+    z = refs.load("mnn_512x384_" + mode + ("" if metric == "dot" else "_" + metric), a, b)
     if z is not None:
         return z
-    r = oracle.mnn(a, b)
+    r = oracle.mnn(a, b, metric=metric)
     z = dict(rowarg=r.row.arg, colarg=r.col.arg)
     if mode == "q":
         z.update(rowbest4096=np.round(r.row.best * 4096).astype(np.int32),
@@ -84,6 +84,23 @@ def test_mnn_full_size_quantised_bf16_bitexact():
     colmax = r.colmax.cpu().numpy().astype(np.float64) * 4096.0
     assert np.array_equal(rowmax, z["rowbest4096"].astype(np.float64))
     assert np.array_equal(colmax, z["colbest4096"].astype(np.float64))
+    assert np.array_equal(r.trimmed().cpu().numpy(), _mutual_pairs(z["rowarg"], z["colarg"]))
+
+
+def test_mnn_full_size_l2_quantised_bitexact():
+    """The whole 512x384, d = 24 set on k/64 maps under the Euclidean metric
+    (the one-pass kernel on the symmetric forms): every nearest index by
+    distance, every squared distance and the pair list, bit for bit."""
+    w, a, b = refs.mnn_inputs("q")
+    z = _mnn_ref("q", a, b, metric="l2")
+    r = rnn.mnn_exhaustive(dev(a), dev(b), with_nn=True, metric="l2")
+    assert np.array_equal(r.rowarg.cpu().numpy(), z["rowarg"])
+    assert np.array_equal(r.colarg.cpu().numpy(), z["colarg"])
+    # the oracle scores -|a - b|^2, the library reports |a - b|^2
+    rowmax = r.rowmax.cpu().numpy().astype(np.float64) * 4096.0
+    colmax = r.colmax.cpu().numpy().astype(np.float64) * 4096.0
+    assert np.array_equal(rowmax, -z["rowbest4096"].astype(np.float64))
+    assert np.array_equal(colmax, -z["colbest4096"].astype(np.float64))
     assert np.array_equal(r.trimmed().cpu().numpy(), _mutual_pairs(z["rowarg"], z["colarg"]))
 
 
