@@ -124,9 +124,11 @@ rnn_status rnn_nn_argmax(const void *Q, int64_t nq, const void *X, int64_t nx, i
  *   colarg_out [H2*W2] NN1 of every D2 pixel, colmax_out its score;
  *              each of these four may be NULL.
  *   workspace  at least rnn_mnn_workspace_size(H1, W1, H2, W2, d) bytes,
- *              256-byte aligned.  When d is not a whole number of the
- *              tensor-core K-blocks (d = 8, 24, 40, ...) it also holds
- *              zero-padded copies of both maps, made by the call.
+ *              256-byte aligned.  For d <= 64 it holds copies of both maps
+ *              made by the call (rows zero-padded to the K-block, then 2048
+ *              NaN rows past the last pixel), which one pass of the fused
+ *              kernel reduces by rows and by columns; larger d keeps the
+ *              rows as given (two sweeps, one per direction).
  */
 size_t rnn_mnn_workspace_size(int H1, int W1, int H2, int W2, int d);
 rnn_status rnn_mnn_exhaustive(const void *D1, int H1, int W1, const void *D2, int H2, int W2,
@@ -194,10 +196,13 @@ rnn_status rnn_frm_match_batched(int B, const void *D1, int64_t d1_batch_stride,
  * rnn_nn_argmax_ex / rnn_mnn_exhaustive_ex: as rnn_nn_argmax /
  * rnn_mnn_exhaustive.  With RNN_L2 the scores written (score_out, rowmax_out,
  * colmax_out) are squared distances |q - x|^2 of the chosen neighbours.
- * Their workspace sizes depend on the metric (the Euclidean metric keeps
- * augmented copies of the maps in it: rows [x, -|x|^2/2 in three 16-bit
- * parts] and [q, 1, 1, 1], whose dot product q.x - |x|^2/2 the tensor cores
- * maximise).
+ * Their workspace sizes depend on the metric.  The Euclidean metric keeps
+ * augmented copies of the maps in it: for rnn_nn_argmax_ex (and the
+ * exhaustive set with d > 56) rows [x, -|x|^2/2 in three 16-bit parts] and
+ * [q, 1, 1, 1], whose dot product q.x - |x|^2/2 the tensor cores maximise;
+ * for the exhaustive set with d <= 56 rows [q, 1, 1, 1, -|q|^2/2] of image 1
+ * and [x, -|x|^2/2, 1, 1, 1] of image 2, whose dot product -|q - x|^2/2 is
+ * maximised over rows and over columns in one pass.
  *
  * rnn_frm_match_ex: FRM over B pairs (as rnn_frm_match_batched) with
  *   init_xy1     NULL: seeds on the grid of stride seed_stride (>= 1).
