@@ -770,6 +770,7 @@ struct LocParams {
   int* cnt;                  // [nch * kLocPad] queries per chunk (padded stride)
   int* start;                // [nch + 1] first list position of each chunk
   int* items;                // [nch + 1] first item of each chunk
+  int* item_chunk;           // [items] the chunk of each item
   int* cursor;               // [nch * kLocPad] fill counters of the scatter (padded stride)
   uint32_t* list;            // [n1 + n2] query ids: image-1 row i, or n1 + image-2 row j
   const uint16_t* X1;        // rows of image 1 and image 2, ld elements apart
@@ -899,11 +900,13 @@ __global__ void loc_scan_kernel(LocParams P) {
     const int c = b0 + k;
     if (c < n) {
       const int k = P.cnt[kLocPad * c];
+      const int ni = (k + kLocItem - 1) / kLocItem;
       P.start[c] = oc;
       P.items[c] = oi;
       P.cursor[kLocPad * c] = 0;
+      for (int j = 0; j < ni; ++j) P.item_chunk[oi + j] = c;
       oc += k;
-      oi += (k + kLocItem - 1) / kLocItem;
+      oi += ni;
     }
   }
   if (threadIdx.x == 0) {
@@ -935,12 +938,7 @@ __global__ void __launch_bounds__(kLocItem* kLocSlices) loc_resolve_kernel(LocPa
   const int total = P.items[P.nch];
   const int qt = threadIdx.x % kLocItem, slice = threadIdx.x / kLocItem;
   for (int it = blockIdx.x; it < total; it += gridDim.x) {
-    int lo = 0, hi = P.nch;  // items[lo] <= it < items[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (P.items[mid] <= it) lo = mid; else hi = mid;
-    }
-    const int c = lo;
+    const int c = P.item_chunk[it];
     const bool rows = c < P.nch_r;
     const int L = rows ? P.lr : P.lc;
     const int64_t ncand = rows ? P.n2 : P.n1;
@@ -2092,7 +2090,7 @@ struct MnnWs {
   // grouped locate of the one-pass path (chunks: at most n2/64 row chunks and
   // n1/32 column chunks)
   int64_t nch_max;
-  int *loc_cnt, *loc_start, *loc_items, *loc_cursor;
+  int *loc_cnt, *loc_start, *loc_items, *loc_item_chunk, *loc_cursor;
   uint32_t* loc_list;
 };
 
@@ -2107,6 +2105,8 @@ static size_t mnn_layout(void* ws, int64_t n1, int64_t n2, int d, rnn_metric met
   w->loc_cursor = c.take<int>(kLocPad * (w->nch_max + 1));
   w->loc_start = c.take<int>(w->nch_max + 1);
   w->loc_items = c.take<int>(w->nch_max + 1);
+  // items: at most one per chunk beyond the full ones
+  w->loc_item_chunk = c.take<int>(w->nch_max + (n1 + n2) / kLocItem + 2);
   w->loc_list = c.take<uint32_t>(n1 + n2 > 0 ? n1 + n2 : 1);
   w->q1 = w->x1 = w->q2 = w->x2 = nullptr;
   const int mode = d > 0 ? copies_for(d, metric) : kCopiesNone;
@@ -2257,6 +2257,7 @@ static rnn_status mnn_onepass(const uint16_t* X1, int64_t n1, const uint16_t* X2
   P.cnt = w.loc_cnt;
   P.start = w.loc_start;
   P.items = w.loc_items;
+  P.item_chunk = w.loc_item_chunk;
   P.cursor = w.loc_cursor;
   P.list = w.loc_list;
   P.X1 = X1;
